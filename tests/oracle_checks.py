@@ -1,0 +1,320 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each ``check_*`` takes an ``oracle.Oracle`` and raises AssertionError on failure.  The pin
+tests run them on the oracle as built; the planted-mistake tests run them on copies of the
+oracle with one plausible mistake each and require that some check fails.
+
+What pins what:
+  * SpMV       -- closed-form eigenpairs of the 1D/2D/3D Dirichlet Laplacians (the 2D one
+                  is the Poisson model problem of the torch-sla page's experiments); a dense
+                  matvec (numpy) on random rectangular matrices.
+  * transpose  -- dense transpose.
+  * PCG        -- the defining optimality of CG: the k-th iterate is the A-norm-optimal
+                  point of the Krylov space K_k(M^-1 A, M^-1 b) (Galerkin condition), built
+                  here with dense QR and a dense solve; one-step convergence on an
+                  eigenvector; m-step termination for m distinct eigenvalues; agreement
+                  with a dense LU solve; invariance under scaling of b; status codes.
+  * SPAI apply -- the dense product (G G^T + eps I) r.
+  * adjoint    -- A lam = w; w.x = lam.b; sum A_ij g_ij = -L; central finite differences
+                  of L = w.A^-1 b (dense LU) in single stored entries and in b.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import sla_workloads as W
+
+TOL_TIGHT = 1e-13
+
+
+# ------------------------------------------------------------------------------ helpers
+def dense(A) -> np.ndarray:
+    D = np.zeros((A.n_rows, A.n_cols), dtype=np.float64)
+    rows = A.rows_of_entries()
+    D[rows, A.col.astype(np.int64)] = A.val.astype(np.float64)
+    return D
+
+
+def csr_from_dense(D: np.ndarray) -> W.CSR:
+    n_rows, n_cols = D.shape
+    rp = [0]
+    ci, v = [], []
+    for i in range(n_rows):
+        nz = np.nonzero(D[i])[0]
+        ci.extend(nz.tolist())
+        v.extend(D[i, nz].tolist())
+        rp.append(len(ci))
+    return W.CSR(n_rows, n_cols, np.array(rp, np.int32), np.array(ci, np.int32),
+                 np.array(v, np.float64))
+
+
+def random_sparse(rng, n_rows, n_cols, density=0.3) -> np.ndarray:
+    D = rng.uniform(-1, 1, size=(n_rows, n_cols))
+    D[rng.uniform(size=D.shape) > density] = 0.0
+    return D
+
+
+def random_spd(n: int, seed: int) -> W.CSR:
+    """Small SPD matrix with a random pattern and a non-constant diagonal."""
+    A = W.random_spd_list(1, n, pairs_per_row=2.0, shift=0.5, seed=seed, dtype=np.float64)
+    A.sys_row_off = None
+    return A
+
+
+def rel(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    den = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
+
+
+def lap_eig_1d(N, j):
+    p = np.arange(1, N + 1)
+    return np.sin(j * np.pi * p / (N + 1)), 2.0 - 2.0 * np.cos(j * np.pi / (N + 1))
+
+
+def dense_minv(ora, A, kind, G=None, eps=0.0) -> np.ndarray:
+    n = A.n_rows
+    if kind == "none":
+        return np.eye(n)
+    if kind == "jacobi":
+        return np.diag(1.0 / np.diag(dense(A)))
+    Gd = dense(G)
+    return Gd @ Gd.T + eps * np.eye(n)
+
+
+# ------------------------------------------------------------------------------ SpMV
+def check_spmv_closed_form(ora):
+    # 1D: tridiag(-1, 2, -1), eigenvalue 2 - 2cos(j pi/(N+1))
+    N = 37
+    A = W.poisson1d(N)
+    for j in (1, 5, 36):
+        v, lam = lap_eig_1d(N, j)
+        assert rel(ora.spmv(A, v), lam * v) < 1e-12, "1D Laplacian eigenpair"
+    # 2D: 5-point, eigenvalue 4 - 2cos(j pi/(N+1)) - 2cos(k pi/(N+1)), v = v_j (x) v_k
+    N = 19
+    A = W.poisson2d(N)
+    for j, k in ((1, 1), (3, 7), (19, 2)):
+        vj, lj = lap_eig_1d(N, j)
+        vk, lk = lap_eig_1d(N, k)
+        v = np.outer(vj, vk).ravel()
+        assert rel(ora.spmv(A, v), (lj + lk) * v) < 1e-12, "2D Poisson eigenpair"
+    # 3D heat step: A = I + dt L7, eigenvalue 1 + dt (sum of three 1D eigenvalues)
+    N, dt = 9, 0.1
+    A = W.heat3d(N, dt, np.float64)
+    for j, k, l in ((1, 1, 1), (2, 5, 9)):
+        vj, lj = lap_eig_1d(N, j)
+        vk, lk = lap_eig_1d(N, k)
+        vl, ll = lap_eig_1d(N, l)
+        v = np.einsum("a,b,c->abc", vj, vk, vl).ravel()
+        assert rel(ora.spmv(A, v), (1 + dt * (lj + lk + ll)) * v) < 1e-12, "3D heat eigenpair"
+
+
+def check_spmv_dense(ora):
+    rng = np.random.default_rng(11)
+    for shape in ((30, 30), (20, 33), (41, 7)):
+        D = random_sparse(rng, *shape)
+        D[3, :] = 0.0                       # an empty row
+        A = csr_from_dense(D)
+        x = rng.standard_normal(shape[1])
+        assert rel(ora.spmv(A, x), D @ x) < 1e-14, f"SpMV vs dense {shape}"
+
+
+def check_transpose(ora):
+    rng = np.random.default_rng(12)
+    D = random_sparse(rng, 17, 23, 0.35)
+    At = ora.transpose(csr_from_dense(D))
+    assert At.n_rows == 23 and At.n_cols == 17
+    assert np.array_equal(dense(At), D.T), "transpose vs dense"
+    for i in range(At.n_rows):
+        seg = At.col[At.row_ptr[i]:At.row_ptr[i + 1]]
+        assert np.all(np.diff(seg) > 0), "transpose keeps columns ascending"
+
+
+def check_spai_apply(ora):
+    rng = np.random.default_rng(13)
+    A = random_spd(30, 101)
+    G = W.spai_factor_G(A, seed=7, dtype=np.float64)
+    r = rng.standard_normal(A.n_rows)
+    for eps in (3e-3, 0.25):
+        z = ora.precond_apply(A, r, "spai", G=G, eps=eps)
+        Gd = dense(G)
+        assert rel(z, (Gd @ Gd.T + eps * np.eye(A.n_rows)) @ r) < 1e-14, "SPAI apply vs dense"
+    zj = ora.precond_apply(A, r, "jacobi")
+    assert rel(zj, r / np.diag(dense(A))) < 1e-15, "Jacobi apply vs dense"
+
+
+# ------------------------------------------------------------------------------ PCG
+def check_pcg_krylov_optimal(ora):
+    """x_k is the Galerkin (A-norm optimal) point of K_k(M^-1 A, M^-1 b), for k = 1..5."""
+    rng = np.random.default_rng(14)
+    A = random_spd(14, 202)
+    Ad = dense(A)
+    G = W.spai_factor_G(A, seed=9, dtype=np.float64)
+    b = rng.standard_normal(A.n_rows)
+    for kind in ("none", "jacobi", "spai"):
+        Minv = dense_minv(ora, A, kind, G, 0.01)
+        v = Minv @ b
+        basis = []
+        for k in range(1, 6):
+            basis.append(v / np.linalg.norm(v))
+            v = Minv @ (Ad @ basis[-1])
+            Q, _ = np.linalg.qr(np.array(basis).T)
+            x_ref = Q @ np.linalg.solve(Q.T @ Ad @ Q, Q.T @ b)
+            res = ora.pcg(A, b, precond=kind, G=G, eps=0.01, fixed_iters=k)
+            assert res.iters == k
+            assert rel(res.x, x_ref) < 1e-10, f"{kind}: iterate {k} is not Krylov-optimal"
+            true_rel = np.linalg.norm(b - Ad @ res.x) / np.linalg.norm(b)
+            assert abs(res.relres - true_rel) <= 1e-12, f"{kind}: recursive residual drifts at {k}"
+
+
+def check_pcg_eigvec_one_step(ora):
+    N = 16
+    A = W.poisson2d(N)
+    vj, lj = lap_eig_1d(N, 3)
+    vk, lk = lap_eig_1d(N, 5)
+    b = np.outer(vj, vk).ravel()
+    res = ora.pcg(A, b, "jacobi", tol=1e-12)
+    assert res.iters == 1, f"eigenvector rhs needs one step, took {res.iters}"
+    assert rel(res.x, b / (lj + lk)) < 1e-13, "x = v / lambda"
+
+
+def check_pcg_m_distinct(ora):
+    N = 16
+    A = W.poisson2d(N)
+    pairs = [(1, 1), (1, 2), (2, 3), (4, 4), (7, 9)]        # distinct eigenvalues
+    lams = []
+    b = np.zeros(N * N)
+    for c, (j, k) in enumerate(pairs):
+        vj, lj = lap_eig_1d(N, j)
+        vk, lk = lap_eig_1d(N, k)
+        lams.append(lj + lk)
+        b += (1.0 + c) * np.outer(vj, vk).ravel()
+    assert len(set(np.round(lams, 12))) == len(pairs)
+    res = ora.pcg(A, b, "jacobi", tol=1e-10)
+    assert res.iters == len(pairs), f"{len(pairs)} distinct eigenvalues, {res.iters} steps"
+
+
+def check_pcg_dense_solve(ora):
+    rng = np.random.default_rng(15)
+    for n, seed in ((8, 1), (33, 2), (64, 3)):
+        A = random_spd(n, 300 + seed)
+        Ad = dense(A)
+        G = W.spai_factor_G(A, seed=seed, dtype=np.float64)
+        b = rng.uniform(-1, 1, n)
+        x_ref = np.linalg.solve(Ad, b)
+        kappa = np.linalg.cond(Ad)
+        for kind in ("none", "jacobi", "spai"):
+            res = ora.pcg(A, b, precond=kind, G=G, eps=3e-3, tol=1e-12)
+            assert res.status == 0, f"{kind} n={n} status {res.status}"
+            assert res.iters <= n + 5, f"{kind} n={n}: {res.iters} steps"
+            assert rel(res.x, x_ref) < 10 * kappa * 1e-12, f"{kind} n={n} vs dense solve"
+
+
+def check_pcg_scaling(ora):
+    A = random_spd(40, 404)
+    b = np.random.default_rng(16).standard_normal(40)
+    r1 = ora.pcg(A, b, "jacobi", tol=1e-9)
+    r2 = ora.pcg(A, 1e6 * b, "jacobi", tol=1e-9)
+    assert r1.iters == r2.iters, "the stopping test is relative to ||b||"
+    assert rel(r2.x, 1e6 * r1.x) < 1e-12
+
+
+def check_pcg_status(ora):
+    A = W.poisson2d(12)
+    n = A.n_rows
+    res = ora.pcg(A, np.zeros(n), "jacobi", tol=1e-10)
+    assert res.status == 0 and res.iters == 0 and not res.x.any(), "b = 0 gives x = 0, 0 steps"
+    b = np.random.default_rng(17).uniform(-1, 1, n)
+    res = ora.pcg(A, b, "jacobi", tol=1e-14, maxit=3)
+    assert res.status == 1 and res.iters == 3, "maxit reached -> not converged"
+    ind = csr_from_dense(np.diag([1.0, -1.0]))
+    res = ora.pcg(ind, np.array([1.0, 1.0]), "none", tol=1e-10)
+    assert res.status == 2, "p.q = 0 on an indefinite matrix -> breakdown"
+
+
+# ------------------------------------------------------------------------------ adjoint
+def _loss_dense(Ad, b, w):
+    return float(w @ np.linalg.solve(Ad, b))
+
+
+def check_adjoint_identities(ora):
+    rng = np.random.default_rng(18)
+    for A in (W.poisson2d(14), random_spd(50, 505)):
+        n = A.n_rows
+        b = rng.uniform(-1, 1, n)
+        w = rng.uniform(-1, 1, n)
+        fw = ora.pcg(A, b, "jacobi", tol=1e-13)
+        adj = ora.adjoint(A, fw.x, w, "jacobi", tol=1e-13)
+        L = float(w @ fw.x)
+        assert rel(ora.spmv(A, adj.lam), w) < 1e-12, "A^T lam = w"
+        assert abs(float(adj.lam @ b) - L) <= 1e-10 * max(1.0, abs(L)), "lam.b = w.x"
+        s = float(np.sum(A.val.astype(np.float64) * adj.grad))
+        assert abs(s + L) <= 1e-10 * max(1.0, abs(L)), "sum A_ij g_ij = -L"
+
+
+def check_grad_fd(ora):
+    """Central differences of L = w.A^-1 b in single stored entries (dense LU)."""
+    rng = np.random.default_rng(19)
+    A = random_spd(15, 606)
+    Ad = dense(A)
+    b = rng.uniform(-1, 1, 15)
+    w = rng.uniform(-1, 1, 15)
+    fw = ora.pcg(A, b, "jacobi", tol=1e-14)
+    adj = ora.adjoint(A, fw.x, w, "jacobi", tol=1e-14)
+    rows = A.rows_of_entries()
+    picks = rng.choice(A.nnz, size=12, replace=False)
+    for kk in picks:
+        i, j = int(rows[kk]), int(A.col[kk])
+        h = 1e-6 * max(1.0, abs(Ad[i, j]))
+        Ap = Ad.copy(); Ap[i, j] += h
+        Am = Ad.copy(); Am[i, j] -= h
+        fd = (_loss_dense(Ap, b, w) - _loss_dense(Am, b, w)) / (2 * h)
+        assert abs(adj.grad[kk] - fd) <= 1e-7 * max(1.0, abs(fd)), f"dL/dA[{i},{j}]"
+    for i in rng.choice(15, size=5, replace=False):
+        h = 1e-6
+        bp = b.copy(); bp[i] += h
+        bm = b.copy(); bm[i] -= h
+        fd = (_loss_dense(Ad, bp, w) - _loss_dense(Ad, bm, w)) / (2 * h)
+        assert abs(adj.lam[i] - fd) <= 1e-7 * max(1.0, abs(fd)), f"dL/db[{i}]"
+
+
+def check_grad_fd_symmetric(ora):
+    """A symmetric perturbation of (i,j) and (j,i), L evaluated by tight CG, matches g_ij + g_ji."""
+    rng = np.random.default_rng(20)
+    A = W.poisson2d(8)
+    n = A.n_rows
+    b = rng.uniform(-1, 1, n)
+    w = rng.uniform(-1, 1, n)
+    fw = ora.pcg(A, b, "jacobi", tol=1e-14)
+    adj = ora.adjoint(A, fw.x, w, "jacobi", tol=1e-14)
+    rows = A.rows_of_entries()
+    index = {(int(rows[k]), int(A.col[k])): k for k in range(A.nnz)}
+    for (i, j) in ((0, 1), (9, 17), (30, 30)):
+        h = 1e-5
+        def L_of(delta):
+            B = W.CSR(A.n_rows, A.n_cols, A.row_ptr, A.col, A.val.astype(np.float64).copy())
+            B.val[index[(i, j)]] += delta
+            if i != j:
+                B.val[index[(j, i)]] += delta
+            return float(w @ ora.pcg(B, b, "jacobi", tol=1e-14).x)
+        fd = (L_of(h) - L_of(-h)) / (2 * h)
+        g = adj.grad[index[(i, j)]] + (adj.grad[index[(j, i)]] if i != j else 0.0)
+        assert abs(g - fd) <= 1e-6 * max(1.0, abs(fd)), f"symmetric dL/dA[{i},{j}]"
+
+
+def check_list_blocks(ora):
+    A = W.random_spd_list(4, 30, seed=21, dtype=np.float64)
+    Ad = dense(A)
+    b = np.random.default_rng(22).uniform(-1, 1, A.n_rows)
+    x, out = ora.pcg_list(A, b, precond="jacobi", tol=1e-13)
+    assert all(r.status == 0 for r in out)
+    assert rel(x, np.linalg.solve(Ad, b)) < 1e-10, "block-diagonal list vs dense solve"
+
+
+ALL_CHECKS = [
+    check_spmv_closed_form, check_spmv_dense, check_transpose, check_spai_apply,
+    check_pcg_krylov_optimal, check_pcg_eigvec_one_step, check_pcg_m_distinct,
+    check_pcg_dense_solve, check_pcg_scaling, check_pcg_status, check_adjoint_identities,
+    check_grad_fd, check_grad_fd_symmetric, check_list_blocks,
+]
