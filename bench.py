@@ -1,0 +1,455 @@
+"""Benchmark: PCG iterations/s of the differentiable sparse SPD solve on B200.
+
+One step = the whole hot path on one batch of synthetic input: the forward PCG solve
+x = A^-1 b, the adjoint solve A lambda = w (w = dL/dx for L = w.x) and the pattern
+gradient dL/dA_ij = -lambda_i x_j.  The default workload is the SPAI-preconditioned 2D
+Poisson problem (1024 x 1024 grid, fp32 values and vectors, fp64 reductions,
+M^-1 = G G^T + 3e-3 I, tolerance 1e-6).  value = PCG iterations (forward + adjoint) per
+second over all ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..5]
+
+Multi-GPU (torchrun): every rank solves its own replica (the single-system solve does not
+shard here), weak scaling; time is the max over ranks.  --impl reference times the fp64
+CPU oracle on the host cores (bounded sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "PCG iterations/sec and SpMV HBM GB/s (fraction of ~8 TB/s) at 1 B200"
+UNIT = "iterations/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--size", default="full", choices=["full", "small", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-reps", type=int, default=20)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------- byte model
+def vbytes(dtype) -> int:
+    return np.dtype(dtype).itemsize
+
+
+def matrix_bytes(n, nnz, sv) -> int:
+    """Algorithmic bytes to stream one CSR matrix: values + column indices + row_ptr."""
+    return nnz * (sv + 4) + (n + 1) * 4
+
+
+def kernel_bytes(w) -> dict:
+    """Algorithmic bytes per launch of each kernel of one PCG iteration (K right-hand sides)."""
+    A = w.A
+    n, nnz, sv = A.n_rows, A.nnz, vbytes(w.dtype)
+    K = w.nrhs
+    out = {"q_spmv": matrix_bytes(n, nnz, sv) + 4 * n * K * sv}   # read z, p_old; write p_new, q
+    if w.precond == "spai":
+        ng = w.G.nnz
+        out["update_gt_spmv"] = matrix_bytes(n, ng, sv) + 7 * n * K * sv   # r,q gathered; p,x; write r,x,y
+        out["z_g_spmv"] = matrix_bytes(n, ng, sv) + 3 * n * K * sv         # y gathered, r; write z
+    else:
+        out["update_jacobi"] = 8 * n * K * sv + n * sv                     # x,p,r,q,(D^-1); write x,r,z
+    return out
+
+
+# ------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines: list[str] = []
+        self.t = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(smax)) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_bus_id(dev: int) -> str | None:
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------------- helpers
+def measured_peaks() -> tuple[float, str]:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "differentiable_sparse_linear_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str) -> int | None:
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    for ln in open(path):
+        parts = ln.split()
+        if len(parts) >= 4 and not ln.startswith("#") and parts[0] == kernel and parts[1] == workload:
+            if parts[3] == src:
+                return int(float(parts[2]))
+    return None
+
+
+def cpu_baseline(w, budget_s: float = 15.0) -> dict:
+    """The fp64 oracle (single-threaded C) on a bounded sample: fixed PCG iterations."""
+    import oracle
+    ora = oracle.get()
+    B = w.B if w.B.ndim == 1 else w.B[:, 0]
+    A = w.A
+    if A.sys_row_off is not None:
+        A = ora.system(A, 0)
+        B = B[: A.n_rows]
+    kw = dict(precond=w.precond, G=w.G, eps=w.eps)
+    t0 = time.perf_counter()
+    ora.pcg(A, B, fixed_iters=5, **kw)
+    per = (time.perf_counter() - t0) / 5
+    iters = int(max(5, min(5000, budget_s / max(per, 1e-9))))
+    t0 = time.perf_counter()
+    r = ora.pcg(A, B, fixed_iters=iters, **kw)
+    dt = time.perf_counter() - t0
+    return {"value": r.iters / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{r.iters} fixed PCG iterations of the forward solve on the same "
+                      f"{'system 0 of the ' if w.A.sys_row_off is not None else ''}workload "
+                      f"({dt:.1f} s, one host thread)"}
+
+
+# ------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import sla_workloads as W
+    w = W.workload(args.config, args.size)
+    import oracle
+    ora = oracle.get()
+    B = w.B if w.B.ndim == 1 else w.B[:, 0]
+    A = w.A
+    if A.sys_row_off is not None:
+        A = ora.system(A, 0)
+        B = B[: A.n_rows]
+    kw = dict(precond=w.precond, G=w.G, eps=w.eps)
+    t0 = time.perf_counter()
+    ora.pcg(A, B, fixed_iters=3, **kw)
+    per = (time.perf_counter() - t0) / 3
+    per_step = int(max(3, min(2000, 2.0 / max(per, 1e-9))))     # about 2 s of CPU per step
+    for _ in range(args.warmup):
+        ora.pcg(A, B, fixed_iters=per_step, **kw)
+    t0 = time.perf_counter()
+    total = 0
+    for _ in range(args.steps):
+        total += ora.pcg(A, B, fixed_iters=per_step, **kw).iters
+    dt = time.perf_counter() - t0
+    value = total / dt
+    sample = (f"{per_step} fixed forward PCG iterations per step of the fp64 oracle on "
+              f"{w.name} (one host thread)")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "n": int(A.n_rows), "nnz": int(A.nnz)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import differentiable_sparse_linear_b200 as sla
+    import sla_workloads as W
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = W.workload(args.config, args.size)
+    A = w.A
+    t_setup = time.perf_counter()
+    rp = torch.from_numpy(A.row_ptr).to(dev)
+    ci = torch.from_numpy(A.col).to(dev)
+    va = torch.from_numpy(A.val).to(dev)
+    is_list = A.sys_row_off is not None
+    if is_list:
+        Ad = sla.sla_csr_create_list(list(A.sys_row_off), rp, ci, va)
+    else:
+        Ad = sla.sla_csr_create(rp, ci, va)
+    Gd = None
+    if w.precond == "spai":
+        Gd = sla.sla_csr_create(torch.from_numpy(w.G.row_ptr).to(dev), torch.from_numpy(w.G.col).to(dev),
+                                torch.from_numpy(w.G.val).to(dev))
+        M = sla.sla_precond_spai(Ad, Gd, w.eps)
+    else:
+        M = sla.sla_precond_jacobi(Ad)
+    b = torch.from_numpy(np.ascontiguousarray(w.B)).to(dev)
+    wl = torch.from_numpy(np.ascontiguousarray(w.W)).to(dev)
+    X = torch.empty_like(b)
+    torch.cuda.synchronize()
+    setup_s = time.perf_counter() - t_setup
+    nrhs = w.nrhs
+    multi = is_list or nrhs > 1
+    body_kernels = 6 if w.precond == "spai" else 4       # two iterations per graph loop body
+    prologue = 2 if w.precond == "spai" else 1
+
+    def launches(iters: int) -> int:
+        """Kernels one solve launches: init, prologue, loop bodies (two iterations each), copy-out."""
+        return 2 + prologue + body_kernels * ((iters + 1) // 2)
+
+    def step(bv, wv, x_out):
+        if multi:
+            x, inf = sla.sla_pcg_solve_batched(Ad, M, bv, x_out, rtol=w.tol)
+            lam, g, ainf = sla.sla_pcg_adjoint_batched(Ad, M, x, wv, rtol=w.tol)
+            if is_list:
+                return sum(i.iters for i in inf) + sum(i.iters for i in ainf), 2, x, lam
+            it = max(i.iters for i in inf), max(i.iters for i in ainf)
+            return (sum(i.iters for i in inf) + sum(i.iters for i in ainf),
+                    launches(it[0]) + launches(it[1]) + 1, x, lam)
+        x, inf = sla.sla_pcg_solve(Ad, M, bv, x_out, rtol=w.tol)
+        lam, g, ainf = sla.sla_pcg_adjoint(Ad, M, x, wv, rtol=w.tol)
+        if inf.status != 0 or ainf.status != 0:
+            raise RuntimeError(f"solve did not converge: {inf} {ainf}")
+        return inf.iters + ainf.iters, launches(inf.iters) + launches(ainf.iters) + 1, x, lam
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step(b, wl, X)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    clocks = ClockSampler(gpu_bus_id(local) if rank == 0 else None)
+    barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    total_iters = 0
+    total_launch = 0
+    ev0.record()
+    for _ in range(args.steps):
+        flush.zero_()
+        it, nl, _, _ = step(b, wl, X)
+        total_iters += it
+        total_launch += nl + 1
+    ev1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if rank == 0 else {}
+    ms = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms, float(total_iters)], dtype=torch.float64, device=dev)
+    if world > 1:
+        tm = t.clone()
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ti = t.clone()
+        dist.all_reduce(ti, op=dist.ReduceOp.SUM)
+        ms_max, iters_all = float(tm[0]), float(ti[1])
+    else:
+        ms_max, iters_all = ms, float(total_iters)
+    value = iters_all / (ms_max / 1e3)
+
+    # end to end: host inputs in pinned memory, result read back every step
+    hb = torch.from_numpy(np.ascontiguousarray(w.B)).pin_memory()
+    hw = torch.from_numpy(np.ascontiguousarray(w.W)).pin_memory()
+    hx = torch.empty(hb.shape, dtype=hb.dtype).pin_memory()
+    hl = torch.empty(hb.shape, dtype=hb.dtype).pin_memory()
+    bd = torch.empty_like(b)
+    wd = torch.empty_like(wl)
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e_iters = 0
+    e0.record()
+    for _ in range(args.steps):
+        flush.zero_()
+        bd.copy_(hb, non_blocking=True)
+        wd.copy_(hw, non_blocking=True)
+        it, _, x, lam = step(bd, wd, X)
+        hx.copy_(x, non_blocking=True)
+        hl.copy_(lam, non_blocking=True)
+        e_iters += it
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ems = e0.elapsed_time(e1)
+    te = torch.tensor([ems, float(e_iters)], dtype=torch.float64, device=dev)
+    if world > 1:
+        tm = te.clone()
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ti = te.clone()
+        dist.all_reduce(ti, op=dist.ReduceOp.SUM)
+        ems, e_iters = float(tm[0]), float(ti[1])
+    e2e = {"value": e_iters / (ems / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": int(hb.numel() * hb.element_size() + hw.numel() * hw.element_size()),
+           "d2h_bytes_per_step": int(hx.numel() * hx.element_size() + hl.numel() * hl.element_size())}
+
+    # dominant kernel: per-launch device time inside the iteration sequence
+    peak, peak_kind = measured_peaks()
+    roofline = None
+    kernels = {}
+    spmv = None
+    if not is_list:
+        kt = sla.sla_pcg_kernel_times(Ad, M, nrhs, reps=args.kernel_reps)
+        names = list(kernel_bytes(w))
+        kb = kernel_bytes(w)
+        for i, nm in enumerate(names):
+            kernels[nm] = {"ms": kt[i], "bytes": kb[nm], "gbs": kb[nm] / (kt[i] * 1e6) if kt[i] > 0 else None}
+        dom = max(names, key=lambda k: kernels[k]["ms"])
+        ach = kernels[dom]["gbs"]
+        tr = profiled_traffic(dom, w.name)
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
+                    "frac": ach / peak, "traffic": tr, "peak_source": peak_kind,
+                    "algorithmic_bytes": kb[dom], "ms_per_launch": kernels[dom]["ms"]}
+        # standalone SpMV y = A x, L2 flushed before each launch
+        xs = torch.randn(A.n_rows * nrhs, dtype=va.dtype, device=dev).reshape(b.shape)
+        ys = torch.empty_like(xs)
+        tot = 0.0
+        reps = 20
+        for r in range(reps + 2):
+            flush.zero_()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record()
+            if nrhs > 1:
+                sla.sla_spmv_multi(Ad, xs, ys)
+            else:
+                sla.sla_spmv(Ad, xs, ys)
+            s1.record()
+            torch.cuda.synchronize()
+            if r >= 2:
+                tot += s0.elapsed_time(s1)
+        sb = matrix_bytes(A.n_rows, A.nnz, vbytes(w.dtype)) + 2 * A.n_rows * nrhs * vbytes(w.dtype)
+        sp_ms = tot / reps
+        spmv = {"gbs": sb / (sp_ms * 1e6), "frac": sb / (sp_ms * 1e6) / peak, "ms": sp_ms, "bytes": sb,
+                "l2": "flushed before each launch"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        iters_per_step = total_iters / args.steps
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if w.dtype == np.float32 else "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "n": int(A.n_rows), "nnz": int(A.nnz),
+                       "nnz_G": int(w.G.nnz) if w.G is not None else 0, "nrhs": nrhs,
+                       "batch": int(A.batch), "precond": w.precond, "tol": w.tol,
+                       "iters_per_step": iters_per_step,
+                       "step": "forward PCG solve + adjoint PCG solve + pattern gradient",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed between steps (512 MiB write)", "setup_s": setup_s},
+            "roofline": roofline, "spmv": spmv, "kernels": kernels,
+            "gpu_launches": total_launch, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,322 @@
+"""Differentiable sparse SPD solve on B200: Python binding of libsla (include/sla.h).
+
+Every computation runs in libsla's CUDA kernels; this module only marshals torch tensors
+(device pointers, the current CUDA stream) into the C ABI and back.  There is no CPU or
+PyTorch fallback: without the built library, or without a CUDA device, calls raise.
+
+Functions keep the C names (``sla_spmv``, ``sla_pcg_solve``, ``sla_pcg_adjoint`` ...).
+``solve(A, b, M)`` is the differentiable entry point: its backward pass is the adjoint of
+"torch-sla: Differentiable Sparse Linear Algebra with Adjoint Solvers and Sparse Tensor
+Parallelism for PyTorch", Methodology §2 (Linear Systems): one solve with A^T = A,
+dL/db = lambda, dL/dA_ij = -lambda_i x_j on A's pattern; only x is saved for backward.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import (SLA_BREAKDOWN, SLA_ERR_CUDA, SLA_ERR_INVALID_ARG, SLA_ERR_INVALID_CSR,
+                   SLA_ERR_OOM, SLA_ERR_UNSUPPORTED, SLA_F32, SLA_F64, SLA_NOT_CONVERGED,
+                   SLA_SPD, SLA_SUCCESS, SLA_VALIDATE)
+
+__all__ = [
+    "SlaError", "Matrix", "Preconditioner", "PcgInfo", "lib",
+    "sla_version", "sla_csr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
+    "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
+    "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
+    "sla_workspace_bytes", "sla_pcg_kernel_times", "solve",
+]
+
+
+def lib() -> C.CDLL:
+    return _lib.load()
+
+
+class SlaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        L = lib()
+        name = L.sla_status_string(status).decode()
+        detail = L.sla_last_error().decode()
+        super().__init__(f"{where}: {name}: {detail}")
+        self.status = status
+
+
+def _check(status: int, where: str) -> int:
+    if status < 0:
+        raise SlaError(status, where)
+    return status
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libsla takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libsla takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return SLA_F32
+    if dt == torch.float64:
+        return SLA_F64
+    raise ValueError(f"values must be float32 or float64, got {dt}")
+
+
+@dataclass
+class PcgInfo:
+    iters: int
+    relres: float
+    status: int
+
+    @property
+    def converged(self) -> bool:
+        return self.status == SLA_SUCCESS
+
+
+def _infos(arr) -> list[PcgInfo]:
+    return [PcgInfo(int(a.iters), float(a.relres), int(a.status)) for a in arr]
+
+
+def _opts(rtol: float, maxit: int) -> _lib.sla_pcg_opts:
+    o = _lib.sla_pcg_opts()
+    o.rtol = float(rtol)
+    o.maxit = int(maxit)
+    return o
+
+
+def sla_version() -> str:
+    return lib().sla_version().decode()
+
+
+class Matrix:
+    """Handle on a CSR matrix held in CUDA tensors (int32 row_ptr/col, fp32/fp64 values).
+
+    The tensors are borrowed by the library; this object keeps them alive.
+    """
+
+    def __init__(self, handle: int, row_ptr, col, val, sys_row_off=None):
+        self._h = C.c_void_p(handle)
+        self.row_ptr, self.col, self.val = row_ptr, col, val
+        self.sys_row_off = sys_row_off
+        self.n = row_ptr.numel() - 1
+        self.nnz = col.numel()
+        self.dtype = val.dtype
+        self.batch = 1 if sys_row_off is None else len(sys_row_off) - 1
+
+    @property
+    def handle(self) -> C.c_void_p:
+        if self._h is None or not self._h.value:
+            raise ValueError("matrix handle is closed")
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().sla_csr_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def matvec(self, x: torch.Tensor) -> torch.Tensor:
+        return sla_spmv(self, x)
+
+
+class Preconditioner:
+    def __init__(self, handle: int, kind: str, A: Matrix, G: Optional[Matrix] = None, eps: float = 0.0):
+        self._h = C.c_void_p(handle)
+        self.kind, self.A, self.G, self.eps = kind, A, G, eps
+
+    @property
+    def handle(self) -> C.c_void_p:
+        if self._h is None or not self._h.value:
+            raise ValueError("preconditioner handle is closed")
+        return self._h
+
+    def refresh(self, stream=None):
+        _check(lib().sla_precond_refresh(self.handle, _stream(stream)), "sla_precond_refresh")
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().sla_precond_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _mh(M: Optional[Preconditioner]):
+    return None if M is None else M.handle
+
+
+def sla_csr_create(row_ptr: torch.Tensor, col: torch.Tensor, val: torch.Tensor, *,
+                   validate: bool = True, spd: bool = True, stream=None) -> Matrix:
+    """sla_csr_create: one square CSR matrix (n = row_ptr.numel() - 1)."""
+    n = row_ptr.numel() - 1
+    if row_ptr.dtype != torch.int32 or col.dtype != torch.int32:
+        raise ValueError("row_ptr and col must be int32")
+    h = C.c_void_p()
+    flags = (SLA_VALIDATE if validate else 0) | (SLA_SPD if spd else 0)
+    _check(lib().sla_csr_create(C.byref(h), n, n, col.numel(), _ptr(row_ptr), _ptr(col), _ptr(val),
+                                _dtype_code(val.dtype), flags, _stream(stream)), "sla_csr_create")
+    return Matrix(h.value, row_ptr, col, val)
+
+
+def sla_csr_create_list(sys_row_off: Sequence[int], row_ptr: torch.Tensor, col: torch.Tensor,
+                        val: torch.Tensor, *, validate: bool = True, spd: bool = True,
+                        stream=None) -> Matrix:
+    """sla_csr_create_list: independent systems as one block-diagonal CSR (global columns)."""
+    off = (C.c_int64 * len(sys_row_off))(*[int(v) for v in sys_row_off])
+    h = C.c_void_p()
+    flags = (SLA_VALIDATE if validate else 0) | (SLA_SPD if spd else 0)
+    _check(lib().sla_csr_create_list(C.byref(h), len(sys_row_off) - 1, off, col.numel(), _ptr(row_ptr),
+                                     _ptr(col), _ptr(val), _dtype_code(val.dtype), flags,
+                                     _stream(stream)), "sla_csr_create_list")
+    return Matrix(h.value, row_ptr, col, val, sys_row_off=list(sys_row_off))
+
+
+def sla_spmv(A: Matrix, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    y = torch.empty(A.n, dtype=A.dtype, device=x.device) if y is None else y
+    _check(lib().sla_spmv(A.handle, _ptr(x), _ptr(y), _stream(stream)), "sla_spmv")
+    return y
+
+
+def sla_spmv_multi(A: Matrix, X: torch.Tensor, Y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    nrhs = X.shape[1]
+    Y = torch.empty_like(X) if Y is None else Y
+    _check(lib().sla_spmv_multi(A.handle, nrhs, _ptr(X), _ptr(Y), _stream(stream)), "sla_spmv_multi")
+    return Y
+
+
+def sla_precond_jacobi(A: Matrix, stream=None) -> Preconditioner:
+    h = C.c_void_p()
+    _check(lib().sla_precond_jacobi(C.byref(h), A.handle, _stream(stream)), "sla_precond_jacobi")
+    return Preconditioner(h.value, "jacobi", A)
+
+
+def sla_precond_spai(A: Matrix, G: Matrix, eps: float = 3e-3, stream=None) -> Preconditioner:
+    h = C.c_void_p()
+    _check(lib().sla_precond_spai(C.byref(h), A.handle, G.handle, float(eps), _stream(stream)),
+           "sla_precond_spai")
+    return Preconditioner(h.value, "spai", A, G, eps)
+
+
+def sla_pcg_solve(A: Matrix, M: Optional[Preconditioner], b: torch.Tensor,
+                  x: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
+                  stream=None) -> tuple[torch.Tensor, PcgInfo]:
+    x = torch.empty_like(b) if x is None else x
+    info = _lib.sla_pcg_info()
+    opts = _opts(rtol, maxit)
+    _check(lib().sla_pcg_solve(A.handle, _mh(M), _ptr(b), _ptr(x), C.byref(opts), C.byref(info),
+                               _stream(stream)), "sla_pcg_solve")
+    return x, _infos([info])[0]
+
+
+def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLdx: torch.Tensor, *,
+                    want_dA: bool = True, rtol: float = 0.0, maxit: int = 0, stream=None):
+    """Returns (dL/db, dL/dA on A's pattern or None, info)."""
+    dLdb = torch.empty_like(dLdx)
+    dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdx.device) if want_dA else None
+    info = _lib.sla_pcg_info()
+    opts = _opts(rtol, maxit)
+    _check(lib().sla_pcg_adjoint(A.handle, _mh(M), _ptr(x), _ptr(dLdx), _ptr(dLdb), _ptr(dLdA),
+                                 C.byref(opts), C.byref(info), _stream(stream)), "sla_pcg_adjoint")
+    return dLdb, dLdA, _infos([info])[0]
+
+
+def sla_pcg_solve_batched(A: Matrix, M: Optional[Preconditioner], B: torch.Tensor,
+                          X: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
+                          stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
+    """Shared matrix: B is [n, nrhs].  List handle: B is the concatenated [n_total] vector."""
+    nrhs = 1 if (B.dim() == 1 or A.batch > 1) else B.shape[1]
+    count = A.batch if A.batch > 1 else nrhs
+    X = torch.empty_like(B) if X is None else X
+    infos = (_lib.sla_pcg_info * count)()
+    opts = _opts(rtol, maxit)
+    _check(lib().sla_pcg_solve_batched(A.handle, _mh(M), nrhs, _ptr(B), _ptr(X), C.byref(opts),
+                                       infos, _stream(stream)), "sla_pcg_solve_batched")
+    return X, _infos(infos)
+
+
+def sla_pcg_adjoint_batched(A: Matrix, M: Optional[Preconditioner], X: torch.Tensor, dLdX: torch.Tensor,
+                            *, want_dA: bool = True, rtol: float = 0.0, maxit: int = 0, stream=None):
+    nrhs = 1 if (dLdX.dim() == 1 or A.batch > 1) else dLdX.shape[1]
+    count = A.batch if A.batch > 1 else nrhs
+    dLdB = torch.empty_like(dLdX)
+    dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdX.device) if want_dA else None
+    infos = (_lib.sla_pcg_info * count)()
+    opts = _opts(rtol, maxit)
+    _check(lib().sla_pcg_adjoint_batched(A.handle, _mh(M), nrhs, _ptr(X), _ptr(dLdX), _ptr(dLdB),
+                                         _ptr(dLdA), C.byref(opts), infos, _stream(stream)),
+           "sla_pcg_adjoint_batched")
+    return dLdB, dLdA, _infos(infos)
+
+
+def sla_pattern_grad(A: Matrix, lam: torch.Tensor, x: torch.Tensor, g: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    nrhs = 1 if lam.dim() == 1 else lam.shape[1]
+    g = torch.empty(A.nnz, dtype=A.dtype, device=lam.device) if g is None else g
+    _check(lib().sla_pattern_grad(A.handle, nrhs, _ptr(lam), _ptr(x), _ptr(g), _stream(stream)),
+           "sla_pattern_grad")
+    return g
+
+
+def sla_pcg_kernel_times(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1, reps: int = 20,
+                         stream=None) -> list[float]:
+    """Mean ms per launch of the iteration's kernels: [q = A p, x/r update, z = G y + eps r]."""
+    out = (C.c_double * 3)()
+    _check(lib().sla_pcg_kernel_times(A.handle, _mh(M), nrhs, reps, out, _stream(stream)),
+           "sla_pcg_kernel_times")
+    return list(out)
+
+
+def sla_workspace_bytes(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1) -> int:
+    return int(lib().sla_workspace_bytes(A.handle, _mh(M), nrhs))
+
+
+class _Solve(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, val, b, A, M, rtol, maxit):
+        x, info = sla_pcg_solve(A, M, b, rtol=rtol, maxit=maxit)
+        if info.status == SLA_BREAKDOWN:
+            raise SlaError(SLA_BREAKDOWN, "solve")
+        ctx.A, ctx.M, ctx.rtol, ctx.maxit = A, M, rtol, maxit
+        ctx.info = info
+        ctx.save_for_backward(x)
+        return x
+
+    @staticmethod
+    def backward(ctx, gx):
+        (x,) = ctx.saved_tensors
+        need_A = ctx.needs_input_grad[0]
+        dLdb, dLdA, info = sla_pcg_adjoint(ctx.A, ctx.M, x, gx.contiguous(), want_dA=need_A,
+                                           rtol=ctx.rtol, maxit=ctx.maxit)
+        return dLdA, dLdb, None, None, None, None
+
+
+def solve(A: Matrix, b: torch.Tensor, M: Optional[Preconditioner] = None, *, rtol: float = 0.0,
+          maxit: int = 0) -> torch.Tensor:
+    """x = A^-1 b, differentiable in A's values (A.val) and in b.
+
+    Gradients flow to ``A.val`` if it requires grad; the backward pass is one adjoint PCG
+    solve and one pattern-gradient pass, independent of the forward iteration count.
+    """
+    return _Solve.apply(A.val, b, A, M, rtol, maxit)

@@ -1,0 +1,708 @@
+// C ABI of libsla: argument checks, handles, tile partitions, solve plans.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "sla.h"
+#include "sla_internal.cuh"
+
+#define SLA_VERSION_STRING "sla-b200 0.1.0 (sm_100a)"
+
+namespace sla {
+
+static thread_local std::string g_last_error;
+
+void set_error(const std::string &msg) { g_last_error = msg; }
+
+sla_status fail(sla_status code, const std::string &msg)
+{
+    set_error(msg);
+    return code;
+}
+
+sla_status cuda_fail(cudaError_t e, const char *what)
+{
+    std::string m = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+    set_error(m);
+    return e == cudaErrorMemoryAllocation ? SLA_ERR_OOM : SLA_ERR_CUDA;
+}
+
+static size_t vbytes(sla_dtype d) { return d == SLA_F32 ? 4 : 8; }
+
+// Rows grouped into tiles of at most D items (rows + entries); a row with more than D-1
+// entries forms a tile of its own.
+sla_status ensure_tiles(sla_csr *A, int D, cudaStream_t s, const TilePart **out)
+{
+    auto it = A->tiles.find(D);
+    if (it != A->tiles.end()) {
+        *out = &it->second;
+        return SLA_SUCCESS;
+    }
+    std::vector<int32_t> t;
+    t.reserve((size_t)(A->n + A->nnz) / (size_t)D + 16);
+    t.push_back(0);
+    int64_t items = 0;
+    for (int64_t r = 0; r < A->n; ++r) {
+        const int64_t len = (int64_t)A->h_rp[r + 1] - A->h_rp[r];
+        if (len + 1 > D) {
+            if (items > 0) {
+                t.push_back((int32_t)r);
+                items = 0;
+            }
+            t.push_back((int32_t)(r + 1));
+            continue;
+        }
+        if (items + len + 1 > D) {
+            t.push_back((int32_t)r);
+            items = 0;
+        }
+        items += len + 1;
+    }
+    if (items > 0)
+        t.push_back((int32_t)A->n);
+    TilePart tp;
+    tp.D = D;
+    tp.n_tiles = (int)t.size() - 1;
+    SLA_CUDA_TRY(cudaMalloc((void **)&tp.d_tile_row, t.size() * sizeof(int32_t)));
+    SLA_CUDA_TRY(cudaMemcpyAsync(tp.d_tile_row, t.data(), t.size() * sizeof(int32_t),
+                                 cudaMemcpyHostToDevice, s));
+    SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    auto ins = A->tiles.emplace(D, tp);
+    *out = &ins.first->second;
+    return SLA_SUCCESS;
+}
+
+static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K)
+{
+    (void)M;
+    const size_t vec = align256((size_t)A->n * (size_t)K * vbytes(A->dtype));
+    const size_t parts = align256((size_t)A->num_sms * 32 * 2 * KMAX * sizeof(double));
+    return 8 * vec + parts + align256(sizeof(PcgState));
+}
+
+void destroy_plan(Plan *p)
+{
+    if (!p)
+        return;
+    if (p->exec)
+        cudaGraphExecDestroy(p->exec);
+    if (p->graph)
+        cudaGraphDestroy(p->graph);
+    if (p->cs)
+        cudaStreamDestroy(p->cs);
+    if (p->cs2)
+        cudaStreamDestroy(p->cs2);
+    if (p->ws)
+        cudaFree(p->ws);
+    if (p->h_st)
+        cudaFreeHost(p->h_st);
+    delete p;
+}
+
+sla_status get_plan(sla_csr *A, const sla_precond *M, int K, Plan **out)
+{
+    for (Plan *p : A->plans)
+        if (p->M == M && p->K == K) {
+            *out = p;
+            return SLA_SUCCESS;
+        }
+    Plan *p = new Plan();
+    p->M = M;
+    p->K = K;
+    p->kind = M ? M->kind : 0;
+    p->ws_bytes = plan_bytes(A, M, K);
+    auto cleanup = [&](sla_status st) {
+        destroy_plan(p);
+        return st;
+    };
+    cudaError_t e = cudaMalloc(&p->ws, p->ws_bytes);
+    if (e != cudaSuccess)
+        return cleanup(cuda_fail(e, "solver workspace"));
+    e = cudaMallocHost((void **)&p->h_st, sizeof(PcgState));
+    if (e != cudaSuccess)
+        return cleanup(cuda_fail(e, "pinned solver state"));
+    const size_t vec = align256((size_t)A->n * (size_t)K * vbytes(A->dtype));
+    char *b = (char *)p->ws;
+    void **vs[8] = {&p->x, &p->ra, &p->rb, &p->pa, &p->pb, &p->q, &p->z, &p->y};
+    for (int i = 0; i < 8; ++i) {
+        *vs[i] = b;
+        b += vec;
+    }
+    p->partials = (double *)b;
+    b += align256((size_t)A->num_sms * 32 * 2 * KMAX * sizeof(double));
+    p->st = (PcgState *)b;
+    e = cudaStreamCreateWithFlags(&p->cs, cudaStreamNonBlocking);
+    if (e == cudaSuccess)
+        e = cudaStreamCreateWithFlags(&p->cs2, cudaStreamNonBlocking);
+    if (e != cudaSuccess)
+        return cleanup(cuda_fail(e, "capture streams"));
+    sla_status st = capture_plan_graph(A, p);
+    if (st != SLA_SUCCESS)
+        return cleanup(st);
+    A->plans.push_back(p);
+    *out = p;
+    return SLA_SUCCESS;
+}
+
+static sla_status current_device(sla_csr *A)
+{
+    SLA_CUDA_TRY(cudaGetDevice(&A->device));
+    SLA_CUDA_TRY(cudaDeviceGetAttribute(&A->num_sms, cudaDevAttrMultiProcessorCount, A->device));
+    return SLA_SUCCESS;
+}
+
+// Copy row_ptr to the host, check it (always: the kernels rely on it), and optionally
+// check the column pattern on the device.
+static sla_status setup_pattern(sla_csr *A, uint32_t flags, cudaStream_t s)
+{
+    A->h_rp.resize((size_t)A->n + 1);
+    SLA_CUDA_TRY(cudaMemcpyAsync(A->h_rp.data(), A->rp, ((size_t)A->n + 1) * sizeof(int32_t),
+                                 cudaMemcpyDeviceToHost, s));
+    SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    if (A->h_rp[0] != 0)
+        return fail(SLA_ERR_INVALID_CSR, "row_ptr[0] must be 0");
+    if ((int64_t)A->h_rp[(size_t)A->n] != A->nnz)
+        return fail(SLA_ERR_INVALID_CSR, "row_ptr[n] must equal nnz");
+    int64_t mx = 0;
+    for (int64_t r = 0; r < A->n; ++r) {
+        const int64_t len = (int64_t)A->h_rp[r + 1] - A->h_rp[r];
+        if (len < 0)
+            return fail(SLA_ERR_INVALID_CSR, "row_ptr must be non-decreasing (row " + std::to_string(r) + ")");
+        mx = std::max(mx, len);
+    }
+    A->max_row_len = mx;
+    if (flags & SLA_VALIDATE) {
+        int *d_err = nullptr;
+        SLA_CUDA_TRY(cudaMallocAsync((void **)&d_err, sizeof(int), s));
+        SLA_CUDA_TRY(cudaMemsetAsync(d_err, 0, sizeof(int), s));
+        sla_status st = launch_validate(A, d_err, s);
+        int h_err = 0;
+        if (st == SLA_SUCCESS) {
+            cudaError_t e = cudaMemcpyAsync(&h_err, d_err, sizeof(int), cudaMemcpyDeviceToHost, s);
+            if (e == cudaSuccess)
+                e = cudaStreamSynchronize(s);
+            if (e != cudaSuccess)
+                st = cuda_fail(e, "validation");
+        }
+        cudaFreeAsync(d_err, s);
+        if (st != SLA_SUCCESS)
+            return st;
+        if (h_err)
+            return fail(SLA_ERR_INVALID_CSR,
+                        "column index out of range, unsorted or repeated within a row");
+    }
+    return SLA_SUCCESS;
+}
+
+static void free_csr(sla_csr *A)
+{
+    if (!A)
+        return;
+    for (Plan *p : A->plans)
+        destroy_plan(p);
+    A->plans.clear();
+    for (auto &kv : A->tiles)
+        cudaFree(kv.second.d_tile_row);
+    if (A->d_sys_off)
+        cudaFree(A->d_sys_off);
+    if (A->own_rp)
+        cudaFree(A->own_rp);
+    if (A->own_ci)
+        cudaFree(A->own_ci);
+    if (A->own_val)
+        cudaFree(A->own_val);
+    delete A;
+}
+
+}  // namespace sla
+
+using namespace sla;
+
+extern "C" {
+
+const char *sla_version(void) { return SLA_VERSION_STRING; }
+
+const char *sla_status_string(sla_status s)
+{
+    switch (s) {
+    case SLA_SUCCESS: return "SLA_SUCCESS";
+    case SLA_NOT_CONVERGED: return "SLA_NOT_CONVERGED";
+    case SLA_BREAKDOWN: return "SLA_BREAKDOWN";
+    case SLA_ERR_INVALID_ARG: return "SLA_ERR_INVALID_ARG";
+    case SLA_ERR_INVALID_CSR: return "SLA_ERR_INVALID_CSR";
+    case SLA_ERR_CUDA: return "SLA_ERR_CUDA";
+    case SLA_ERR_OOM: return "SLA_ERR_OOM";
+    case SLA_ERR_UNSUPPORTED: return "SLA_ERR_UNSUPPORTED";
+    default: return "SLA_UNKNOWN_STATUS";
+    }
+}
+
+const char *sla_last_error(void) { return g_last_error.c_str(); }
+
+sla_status sla_csr_create(sla_csr **out, int64_t n_rows, int64_t n_cols, int64_t nnz,
+                          const int32_t *d_row_ptr, const int32_t *d_col, const void *d_val,
+                          sla_dtype dtype, uint32_t flags, void *stream)
+{
+    if (!out)
+        return fail(SLA_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (n_rows < 0 || nnz < 0 || n_rows != n_cols)
+        return fail(SLA_ERR_INVALID_ARG, "matrix must be square with n >= 0 and nnz >= 0");
+    if (n_rows >= (int64_t)INT32_MAX || nnz >= (int64_t)INT32_MAX)
+        return fail(SLA_ERR_INVALID_ARG, "n and nnz must fit int32 indices");
+    if (dtype != SLA_F32 && dtype != SLA_F64)
+        return fail(SLA_ERR_INVALID_ARG, "dtype must be SLA_F32 or SLA_F64");
+    if (!d_row_ptr || (nnz > 0 && (!d_col || !d_val)))
+        return fail(SLA_ERR_INVALID_ARG, "NULL row_ptr, col or val");
+    cudaStream_t s = (cudaStream_t)stream;
+    sla_csr *A = new sla_csr();
+    A->n = n_rows;
+    A->nnz = nnz;
+    A->dtype = dtype;
+    A->flags = flags;
+    A->rp = d_row_ptr;
+    A->ci = d_col;
+    A->val = d_val;
+    A->max_sys_n = n_rows;
+    A->max_sys_nnz = nnz;
+    sla_status st = current_device(A);
+    if (st == SLA_SUCCESS)
+        st = setup_pattern(A, flags, s);
+    if (st != SLA_SUCCESS) {
+        free_csr(A);
+        return st;
+    }
+    *out = A;
+    return SLA_SUCCESS;
+}
+
+sla_status sla_csr_create_list(sla_csr **out, int32_t batch, const int64_t *h_sys_row_off,
+                               int64_t nnz_total, const int32_t *d_row_ptr, const int32_t *d_col,
+                               const void *d_val, sla_dtype dtype, uint32_t flags, void *stream)
+{
+    if (!out)
+        return fail(SLA_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (batch < 1 || !h_sys_row_off)
+        return fail(SLA_ERR_INVALID_ARG, "batch must be >= 1 with system offsets");
+    if (h_sys_row_off[0] != 0)
+        return fail(SLA_ERR_INVALID_ARG, "system offsets must start at 0");
+    for (int32_t i = 0; i < batch; ++i)
+        if (h_sys_row_off[i + 1] < h_sys_row_off[i])
+            return fail(SLA_ERR_INVALID_ARG, "system offsets must be non-decreasing");
+    const int64_t n = h_sys_row_off[batch];
+    sla_csr *A = nullptr;
+    sla_status st = sla_csr_create(&A, n, n, nnz_total, d_row_ptr, d_col, d_val, dtype,
+                                   flags & ~SLA_VALIDATE, stream);
+    if (st != SLA_SUCCESS)
+        return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    A->batch = batch;
+    A->sys_off.assign(h_sys_row_off, h_sys_row_off + batch + 1);
+    A->max_sys_n = 0;
+    A->max_sys_nnz = 0;
+    for (int32_t i = 0; i < batch; ++i) {
+        A->max_sys_n = std::max<int64_t>(A->max_sys_n, h_sys_row_off[i + 1] - h_sys_row_off[i]);
+        A->max_sys_nnz = std::max<int64_t>(
+            A->max_sys_nnz, (int64_t)A->h_rp[(size_t)h_sys_row_off[i + 1]] - A->h_rp[(size_t)h_sys_row_off[i]]);
+    }
+    cudaError_t e = cudaMalloc((void **)&A->d_sys_off, sizeof(int64_t) * (size_t)(batch + 1));
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(A->d_sys_off, h_sys_row_off, sizeof(int64_t) * (size_t)(batch + 1),
+                            cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        st = cuda_fail(e, "system offsets");
+        free_csr(A);
+        return st;
+    }
+    if (flags & SLA_VALIDATE) {
+        A->flags = flags;
+        st = setup_pattern(A, flags, s);
+        if (st != SLA_SUCCESS) {
+            free_csr(A);
+            return st;
+        }
+    }
+    *out = A;
+    return SLA_SUCCESS;
+}
+
+sla_status sla_csr_destroy(sla_csr *A)
+{
+    free_csr(A);
+    return SLA_SUCCESS;
+}
+
+sla_status sla_csr_shape(const sla_csr *A, int64_t *n_rows, int64_t *nnz, int32_t *batch)
+{
+    if (!A)
+        return fail(SLA_ERR_INVALID_ARG, "NULL handle");
+    if (n_rows)
+        *n_rows = A->n;
+    if (nnz)
+        *nnz = A->nnz;
+    if (batch)
+        *batch = A->batch;
+    return SLA_SUCCESS;
+}
+
+sla_status sla_spmv(const sla_csr *A, const void *d_x, void *d_y, void *stream)
+{
+    if (!A)
+        return fail(SLA_ERR_INVALID_ARG, "NULL handle");
+    if (A->n > 0 && (!d_x || !d_y))
+        return fail(SLA_ERR_INVALID_ARG, "NULL vector");
+    if (A->n > 0 && d_x == d_y)
+        return fail(SLA_ERR_INVALID_ARG, "x and y must not overlap");
+    return launch_spmv(A, 1, d_x, d_y, (cudaStream_t)stream);
+}
+
+sla_status sla_spmv_multi(const sla_csr *A, int32_t nrhs, const void *d_X, void *d_Y, void *stream)
+{
+    if (!A)
+        return fail(SLA_ERR_INVALID_ARG, "NULL handle");
+    if (nrhs < 1 || nrhs > KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    if (A->n > 0 && (!d_X || !d_Y || d_X == d_Y))
+        return fail(SLA_ERR_INVALID_ARG, "NULL or overlapping X/Y");
+    return launch_spmv(A, nrhs, d_X, d_Y, (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------------ preconditioners
+static sla_status jacobi_setup(sla_precond *M, cudaStream_t s)
+{
+    const sla_csr *A = M->A;
+    int *d_err = nullptr;
+    SLA_CUDA_TRY(cudaMallocAsync((void **)&d_err, sizeof(int), s));
+    SLA_CUDA_TRY(cudaMemsetAsync(d_err, 0, sizeof(int), s));
+    sla_status st = launch_jacobi_dinv(A, M->d_dinv, d_err, s);
+    int h_err = 0;
+    if (st == SLA_SUCCESS) {
+        cudaError_t e = cudaMemcpyAsync(&h_err, d_err, sizeof(int), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess)
+            e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess)
+            st = cuda_fail(e, "Jacobi set-up");
+    }
+    cudaFreeAsync(d_err, s);
+    if (st != SLA_SUCCESS)
+        return st;
+    if (h_err)
+        return fail(SLA_ERR_INVALID_ARG, "Jacobi needs a stored, positive diagonal entry in every row");
+    return SLA_SUCCESS;
+}
+
+sla_status sla_precond_jacobi(sla_precond **out, const sla_csr *A, void *stream)
+{
+    if (!out || !A)
+        return fail(SLA_ERR_INVALID_ARG, "NULL argument");
+    *out = nullptr;
+    cudaStream_t s = (cudaStream_t)stream;
+    sla_precond *M = new sla_precond();
+    M->kind = 1;
+    M->A = A;
+    cudaError_t e = cudaMalloc(&M->d_dinv, (size_t)std::max<int64_t>(A->n, 1) * vbytes(A->dtype));
+    if (e != cudaSuccess) {
+        delete M;
+        return cuda_fail(e, "Jacobi D^-1");
+    }
+    sla_status st = jacobi_setup(M, s);
+    if (st != SLA_SUCCESS) {
+        cudaFree(M->d_dinv);
+        delete M;
+        return st;
+    }
+    *out = M;
+    return SLA_SUCCESS;
+}
+
+// G^T by a counting sort of G's entries by column on the host (set-up only): row j of G^T
+// lists the rows i of G holding column j in increasing i.  perm[k] = position in G of the
+// k-th entry of G^T, so a later change of G's values is one device gather.
+static sla_status spai_transpose(sla_precond *M, cudaStream_t s)
+{
+    const sla_csr *G = M->G;
+    const int64_t n = G->n, nnz = G->nnz;
+    std::vector<int32_t> ci((size_t)nnz);
+    if (nnz > 0) {
+        SLA_CUDA_TRY(cudaMemcpyAsync(ci.data(), G->ci, (size_t)nnz * sizeof(int32_t),
+                                     cudaMemcpyDeviceToHost, s));
+        SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    }
+    std::vector<int32_t> rpT((size_t)n + 1, 0), ciT((size_t)nnz), perm((size_t)nnz);
+    for (int64_t k = 0; k < nnz; ++k) {
+        if (ci[(size_t)k] < 0 || ci[(size_t)k] >= n)
+            return fail(SLA_ERR_INVALID_CSR, "G: column index out of range");
+        rpT[(size_t)ci[(size_t)k] + 1] += 1;
+    }
+    for (int64_t j = 0; j < n; ++j)
+        rpT[(size_t)j + 1] += rpT[(size_t)j];
+    std::vector<int32_t> fill(rpT.begin(), rpT.end() - 1);
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t k = G->h_rp[(size_t)i]; k < G->h_rp[(size_t)i + 1]; ++k) {
+            const int32_t dst = fill[(size_t)ci[(size_t)k]]++;
+            ciT[(size_t)dst] = (int32_t)i;
+            perm[(size_t)dst] = (int32_t)k;
+        }
+    sla_csr *GT = new sla_csr();
+    GT->n = n;
+    GT->nnz = nnz;
+    GT->dtype = G->dtype;
+    GT->device = G->device;
+    GT->num_sms = G->num_sms;
+    GT->max_sys_n = n;
+    GT->h_rp = rpT;
+    M->GT = GT;
+    int64_t mx = 0;
+    for (int64_t j = 0; j < n; ++j)
+        mx = std::max<int64_t>(mx, (int64_t)rpT[(size_t)j + 1] - rpT[(size_t)j]);
+    GT->max_row_len = mx;
+    SLA_CUDA_TRY(cudaMalloc((void **)&GT->own_rp, ((size_t)n + 1) * sizeof(int32_t)));
+    SLA_CUDA_TRY(cudaMalloc((void **)&GT->own_ci, (size_t)std::max<int64_t>(nnz, 1) * sizeof(int32_t)));
+    SLA_CUDA_TRY(cudaMalloc(&GT->own_val, (size_t)std::max<int64_t>(nnz, 1) * vbytes(G->dtype)));
+    SLA_CUDA_TRY(cudaMalloc((void **)&M->d_perm, (size_t)std::max<int64_t>(nnz, 1) * sizeof(int32_t)));
+    GT->rp = GT->own_rp;
+    GT->ci = GT->own_ci;
+    GT->val = GT->own_val;
+    SLA_CUDA_TRY(cudaMemcpyAsync(GT->own_rp, rpT.data(), ((size_t)n + 1) * sizeof(int32_t),
+                                 cudaMemcpyHostToDevice, s));
+    if (nnz > 0) {
+        SLA_CUDA_TRY(cudaMemcpyAsync(GT->own_ci, ciT.data(), (size_t)nnz * sizeof(int32_t),
+                                     cudaMemcpyHostToDevice, s));
+        SLA_CUDA_TRY(cudaMemcpyAsync(M->d_perm, perm.data(), (size_t)nnz * sizeof(int32_t),
+                                     cudaMemcpyHostToDevice, s));
+    }
+    SLA_TRY(refresh_transpose_values(G, GT, M->d_perm, s));
+    SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    return SLA_SUCCESS;
+}
+
+static void free_precond(sla_precond *M)
+{
+    if (!M)
+        return;
+    if (M->A) {
+        sla_csr *A = const_cast<sla_csr *>(M->A);
+        std::vector<Plan *> keep;
+        for (Plan *p : A->plans) {
+            if (p->M == M)
+                destroy_plan(p);
+            else
+                keep.push_back(p);
+        }
+        A->plans.swap(keep);
+    }
+    if (M->d_dinv)
+        cudaFree(M->d_dinv);
+    if (M->d_perm)
+        cudaFree(M->d_perm);
+    if (M->GT)
+        free_csr(M->GT);
+    delete M;
+}
+
+sla_status sla_precond_spai(sla_precond **out, const sla_csr *A, const sla_csr *G, double eps,
+                            void *stream)
+{
+    if (!out || !A || !G)
+        return fail(SLA_ERR_INVALID_ARG, "NULL argument");
+    *out = nullptr;
+    if (G->n != A->n || G->dtype != A->dtype)
+        return fail(SLA_ERR_INVALID_ARG, "G must match A's size and dtype");
+    if (!(eps >= 0.0))
+        return fail(SLA_ERR_INVALID_ARG, "eps must be >= 0");
+    sla_precond *M = new sla_precond();
+    M->kind = 2;
+    M->A = A;
+    M->G = G;
+    M->eps = eps;
+    sla_status st = spai_transpose(M, (cudaStream_t)stream);
+    if (st != SLA_SUCCESS) {
+        M->A = nullptr;
+        free_precond(M);
+        return st;
+    }
+    *out = M;
+    return SLA_SUCCESS;
+}
+
+sla_status sla_precond_refresh(sla_precond *M, void *stream)
+{
+    if (!M)
+        return fail(SLA_ERR_INVALID_ARG, "NULL preconditioner");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (M->kind == 1)
+        return jacobi_setup(M, s);
+    SLA_TRY(refresh_transpose_values(M->G, M->GT, M->d_perm, s));
+    SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    return SLA_SUCCESS;
+}
+
+sla_status sla_precond_destroy(sla_precond *M)
+{
+    free_precond(M);
+    return SLA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ solves
+static sla_status check_solve(const sla_csr *A, const sla_precond *M)
+{
+    if (!A)
+        return fail(SLA_ERR_INVALID_ARG, "NULL matrix handle");
+    if (M && M->A != A)
+        return fail(SLA_ERR_INVALID_ARG, "the preconditioner was built for another matrix handle");
+    return SLA_SUCCESS;
+}
+
+sla_status sla_pcg_solve(const sla_csr *A, const sla_precond *M, const void *d_b, void *d_x,
+                         const sla_pcg_opts *opts, sla_pcg_info *info, void *stream)
+{
+    SLA_TRY(check_solve(A, M));
+    if (A->batch > 1)
+        return fail(SLA_ERR_INVALID_ARG, "list handles are solved with sla_pcg_solve_batched");
+    if (A->n > 0 && (!d_b || !d_x || d_b == d_x))
+        return fail(SLA_ERR_INVALID_ARG, "NULL or overlapping b/x");
+    if (A->n == 0) {
+        if (info) {
+            info->iters = 0;
+            info->relres = 0.0;
+            info->status = SLA_SUCCESS;
+        }
+        return SLA_SUCCESS;
+    }
+    Plan *p = nullptr;
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, 1, &p));
+    return run_plan(const_cast<sla_csr *>(A), p, 1, d_b, d_x, opts, info, nullptr, nullptr,
+                    (cudaStream_t)stream);
+}
+
+sla_status sla_pcg_adjoint(const sla_csr *A, const sla_precond *M, const void *d_x,
+                           const void *d_dLdx, void *d_dLdb, void *d_dLdA,
+                           const sla_pcg_opts *opts, sla_pcg_info *info, void *stream)
+{
+    SLA_TRY(check_solve(A, M));
+    if (A->batch > 1)
+        return fail(SLA_ERR_INVALID_ARG, "list handles use sla_pcg_adjoint_batched");
+    if (A->n > 0 && (!d_x || !d_dLdx || !d_dLdb || d_dLdx == d_dLdb))
+        return fail(SLA_ERR_INVALID_ARG, "NULL or overlapping adjoint vectors");
+    if (A->n == 0)
+        return SLA_SUCCESS;
+    Plan *p = nullptr;
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, 1, &p));
+    return run_plan(const_cast<sla_csr *>(A), p, 1, d_dLdx, d_dLdb, opts, info, d_x, d_dLdA,
+                    (cudaStream_t)stream);
+}
+
+sla_status sla_pcg_solve_batched(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                 const void *d_B, void *d_X, const sla_pcg_opts *opts,
+                                 sla_pcg_info *h_info, void *stream)
+{
+    SLA_TRY(check_solve(A, M));
+    if (!h_info)
+        return fail(SLA_ERR_INVALID_ARG, "h_info is required");
+    if (A->n > 0 && (!d_B || !d_X || d_B == d_X))
+        return fail(SLA_ERR_INVALID_ARG, "NULL or overlapping B/X");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (A->batch > 1 || A->d_sys_off) {
+        if (nrhs != 1)
+            return fail(SLA_ERR_INVALID_ARG, "list handles take nrhs = 1");
+        return run_list_solve(A, M, d_B, d_X, nullptr, nullptr, opts, h_info, s);
+    }
+    if (nrhs < 1 || nrhs > KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    if (A->n == 0) {
+        for (int c = 0; c < nrhs; ++c)
+            h_info[c] = sla_pcg_info{0, 0.0, SLA_SUCCESS, 0};
+        return SLA_SUCCESS;
+    }
+    int K = 1;
+    while (K < nrhs)
+        K <<= 1;
+    Plan *p = nullptr;
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, &p));
+    return run_plan(const_cast<sla_csr *>(A), p, nrhs, d_B, d_X, opts, h_info, nullptr, nullptr,
+                    s);
+}
+
+sla_status sla_pcg_adjoint_batched(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                   const void *d_X, const void *d_dLdX, void *d_dLdB,
+                                   void *d_dLdA, const sla_pcg_opts *opts, sla_pcg_info *h_info,
+                                   void *stream)
+{
+    SLA_TRY(check_solve(A, M));
+    if (!h_info)
+        return fail(SLA_ERR_INVALID_ARG, "h_info is required");
+    if (A->n > 0 && (!d_X || !d_dLdX || !d_dLdB || d_dLdX == d_dLdB))
+        return fail(SLA_ERR_INVALID_ARG, "NULL or overlapping adjoint blocks");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (A->batch > 1 || A->d_sys_off) {
+        if (nrhs != 1)
+            return fail(SLA_ERR_INVALID_ARG, "list handles take nrhs = 1");
+        return run_list_solve(A, M, d_dLdX, d_dLdB, d_X, d_dLdA, opts, h_info, s);
+    }
+    if (nrhs < 1 || nrhs > KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    if (A->n == 0)
+        return SLA_SUCCESS;
+    int K = 1;
+    while (K < nrhs)
+        K <<= 1;
+    Plan *p = nullptr;
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, &p));
+    return run_plan(const_cast<sla_csr *>(A), p, nrhs, d_dLdX, d_dLdB, opts, h_info, d_X, d_dLdA,
+                    s);
+}
+
+sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *d_lam, const void *d_x,
+                            void *d_g, void *stream)
+{
+    if (!A)
+        return fail(SLA_ERR_INVALID_ARG, "NULL handle");
+    if (nrhs < 1)
+        return fail(SLA_ERR_INVALID_ARG, "nrhs must be >= 1");
+    if (A->nnz > 0 && (!d_lam || !d_x || !d_g))
+        return fail(SLA_ERR_INVALID_ARG, "NULL vector");
+    if (A->nnz == 0)
+        return SLA_SUCCESS;
+    return launch_pattern_grad(A, nrhs, d_lam, d_x, d_g, (cudaStream_t)stream);
+}
+
+sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t nrhs, int32_t reps,
+                                double *h_ms, void *stream)
+{
+    SLA_TRY(check_solve(A, M));
+    if (!h_ms || reps < 1)
+        return fail(SLA_ERR_INVALID_ARG, "h_ms is required and reps must be >= 1");
+    if (A->batch > 1)
+        return fail(SLA_ERR_UNSUPPORTED, "kernel timing covers the single-matrix solver");
+    if (nrhs < 1 || nrhs > KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    if (A->n == 0)
+        return fail(SLA_ERR_INVALID_ARG, "empty matrix");
+    int K = 1;
+    while (K < nrhs)
+        K <<= 1;
+    Plan *p = nullptr;
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, &p));
+    return kernel_times(const_cast<sla_csr *>(A), p, nrhs, reps, h_ms, (cudaStream_t)stream);
+}
+
+size_t sla_workspace_bytes(const sla_csr *A, const sla_precond *M, int32_t nrhs)
+{
+    if (!A || nrhs < 1 || nrhs > KMAX)
+        return 0;
+    int K = 1;
+    while (K < nrhs)
+        K <<= 1;
+    return plan_bytes(A, M, K);
+}
+
+}  // extern "C"

@@ -1,0 +1,261 @@
+// PCG over a batch of independent small SPD systems with distinct patterns (the
+// SparseTensorList batch of "torch-sla: Differentiable Sparse Linear Algebra with Adjoint
+// Solvers and Sparse Tensor Parallelism for PyTorch", Methodology §1), forward and adjoint.
+//
+// One block owns one system for its whole solve: the system's vectors (x, r, p, q, z,
+// D^-1, and for the adjoint the forward x) live in shared memory, so the only HBM traffic
+// is the system's matrix (re-read from L2 after the first iteration), b, and the results.
+// Dot products are block reductions in fp64 with a fixed order; each system has its own
+// stopping test, iteration count and status.  There is no grid-wide dependency, so the
+// whole batch is one launch and needs no graph.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "sla_internal.cuh"
+
+namespace sla {
+
+constexpr int LIST_T = 512;
+
+// Sum two values over the block; every thread receives both totals.
+__device__ __forceinline__ void list_sum2(double &a, double &b, double *s_red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        a += __shfl_down_sync(0xffffffffu, a, off);
+        b += __shfl_down_sync(0xffffffffu, b, off);
+    }
+    if (lane == 0) {
+        s_red[2 * warp] = a;
+        s_red[2 * warp + 1] = b;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double ta = 0.0, tb = 0.0;
+        for (int w = 0; w < LIST_T / 32; ++w) {
+            ta += s_red[2 * w];
+            tb += s_red[2 * w + 1];
+        }
+        s_red[2 * (LIST_T / 32)] = ta;
+        s_red[2 * (LIST_T / 32) + 1] = tb;
+    }
+    __syncthreads();
+    a = s_red[2 * (LIST_T / 32)];
+    b = s_red[2 * (LIST_T / 32) + 1];
+    __syncthreads();
+}
+
+// q = A p on one system (rows [0, ns), local columns = global - o0), S lanes per row;
+// returns this thread's share of p.q (only the first lane of each row group contributes).
+template <typename V, int S>
+__device__ __forceinline__ double list_spmv(int ns, int64_t o0, const int32_t *rp, const int32_t *ci,
+                                            const V *val, const V *p, V *q)
+{
+    const int lane = threadIdx.x & (S - 1);
+    const int grp = threadIdx.x / S;
+    constexpr int NG = LIST_T / S;
+    double part = 0.0;
+    for (int i = grp; i < ns; i += NG) {
+        const int64_t k0 = rp[o0 + i], k1 = rp[o0 + i + 1];
+        double acc = 0.0;
+        for (int64_t k = k0 + lane; k < k1; k += S)
+            acc = __fma_rn((double)val[k], (double)p[ci[k] - o0], acc);
+#pragma unroll
+        for (int off = S / 2; off > 0; off >>= 1)
+            acc += __shfl_xor_sync(0xffffffffu, acc, off, S);
+        if (lane == 0) {
+            const V qv = (V)acc;
+            q[i] = qv;
+            part += (double)p[i] * (double)qv;
+        }
+    }
+    return part;
+}
+
+template <typename V, int S>
+__global__ void __launch_bounds__(LIST_T)
+k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sys_off, int batch,
+           const V *B, V *X, const V *dinv, const V *Xf, V *Gout, double tol, long long maxit_opt,
+           sla_pcg_info *info)
+{
+    extern __shared__ __align__(16) unsigned char s_raw[];
+    __shared__ double s_red[2 * (LIST_T / 32) + 2];
+    const int tid = threadIdx.x;
+    for (int s = blockIdx.x; s < batch; s += gridDim.x) {
+        const int64_t o0 = sys_off[s];
+        const int ns = (int)(sys_off[s + 1] - o0);
+        V *x = (V *)s_raw;
+        V *r = x + ns;
+        V *p = r + ns;
+        V *q = p + ns;
+        V *z = q + ns;
+        V *dv = z + ns;
+        V *xf = dv + ns;
+        const long long maxit = maxit_opt > 0 ? maxit_opt : 10LL * (ns > 0 ? ns : 1);
+
+        double bb = 0.0, rz = 0.0;
+        for (int i = tid; i < ns; i += LIST_T) {
+            const V bi = B[o0 + i];
+            const V di = dinv ? dinv[o0 + i] : (V)1;
+            const V zi = (V)((double)bi * (double)di);
+            x[i] = (V)0;
+            r[i] = bi;
+            dv[i] = di;
+            z[i] = zi;
+            p[i] = zi;
+            if (Xf)
+                xf[i] = Xf[o0 + i];
+            bb += (double)bi * (double)bi;
+            rz += (double)bi * (double)zi;
+        }
+        list_sum2(bb, rz, s_red);
+        const double bnorm = sqrt(bb);
+        double rho = rz;
+        long long it = 0;
+        double relres = bnorm > 0.0 ? 1.0 : 0.0;
+        int status = SLA_NOT_CONVERGED;
+        if (!isfinite(bnorm))
+            status = SLA_BREAKDOWN;
+        else if (bnorm == 0.0)
+            status = SLA_SUCCESS;
+        else if (!(rho > 0.0) || !isfinite(rho))
+            status = SLA_BREAKDOWN;
+        else {
+            while (it < maxit) {
+                ++it;
+                double pq = list_spmv<V, S>(ns, o0, rp, ci, val, p, q), dummy = 0.0;
+                list_sum2(pq, dummy, s_red);
+                if (!(pq > 0.0) || !isfinite(pq)) {
+                    status = SLA_BREAKDOWN;
+                    break;
+                }
+                const double alpha = rho / pq;
+                double rr = 0.0, rzn = 0.0;
+                for (int i = tid; i < ns; i += LIST_T) {
+                    x[i] = (V)__fma_rn(alpha, (double)p[i], (double)x[i]);
+                    const V rn = (V)__fma_rn(-alpha, (double)q[i], (double)r[i]);
+                    r[i] = rn;
+                    const V zn = (V)((double)rn * (double)dv[i]);
+                    z[i] = zn;
+                    rr += (double)rn * (double)rn;
+                    rzn += (double)rn * (double)zn;
+                }
+                list_sum2(rr, rzn, s_red);
+                relres = sqrt(rr) / bnorm;
+                if (!isfinite(relres)) {
+                    status = SLA_BREAKDOWN;
+                    break;
+                }
+                if (relres <= tol) {
+                    status = SLA_SUCCESS;
+                    break;
+                }
+                if (!(rzn > 0.0) || !isfinite(rzn)) {
+                    status = SLA_BREAKDOWN;
+                    break;
+                }
+                const double beta = rzn / rho;
+                rho = rzn;
+                for (int i = tid; i < ns; i += LIST_T)
+                    p[i] = (V)__fma_rn(beta, (double)p[i], (double)z[i]);
+                __syncthreads();
+            }
+        }
+        __syncthreads();
+        for (int i = tid; i < ns; i += LIST_T)
+            X[o0 + i] = x[i];
+        if (Gout) {
+            // dL/dA_ij = -lambda_i x_j on the system's pattern (lambda = this solve's x)
+            const int64_t k0 = rp[o0], k1 = rp[o0 + ns];
+            const int lane = tid & (S - 1), grp = tid / S;
+            for (int i = grp; i < ns; i += LIST_T / S) {
+                const double li = (double)x[i];
+                for (int64_t k = rp[o0 + i] + lane; k < rp[o0 + i + 1]; k += S)
+                    Gout[k] = (V)(-li * (double)xf[ci[k] - o0]);
+            }
+            (void)k0;
+            (void)k1;
+        }
+        if (tid == 0) {
+            info[s].iters = it;
+            info[s].relres = relres;
+            info[s].status = status;
+            info[s].reserved = 0;
+        }
+        __syncthreads();
+    }
+}
+
+template <typename V, int S>
+static sla_status list_launch(const sla_csr *A, const V *dinv, const void *B, void *X, const void *Xf,
+                              void *G, double tol, long long maxit, sla_pcg_info *d_info,
+                              cudaStream_t s)
+{
+    const size_t shm = (size_t)7 * (size_t)A->max_sys_n * sizeof(V);
+    auto kern = k_list_pcg<V, S>;
+    SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm));
+    int per_sm = 0;
+    SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, LIST_T, shm));
+    if (per_sm < 1)
+        return fail(SLA_ERR_UNSUPPORTED, "list solve: a system's vectors do not fit in shared memory");
+    const int grid = std::min<int64_t>(A->batch, (int64_t)per_sm * A->num_sms);
+    kern<<<grid, LIST_T, shm, s>>>(A->rp, A->ci, (const V *)A->val, A->d_sys_off, A->batch,
+                                   (const V *)B, (V *)X, dinv, (const V *)Xf, (V *)G, tol, maxit,
+                                   d_info);
+    SLA_CUDA_TRY(cudaGetLastError());
+    return SLA_SUCCESS;
+}
+
+template <typename V>
+static sla_status list_v(const sla_csr *A, const V *dinv, const void *B, void *X, const void *Xf,
+                         void *G, double tol, long long maxit, sla_pcg_info *d_info, cudaStream_t s)
+{
+    const double mean = A->n > 0 ? (double)A->nnz / (double)A->n : 0.0;
+    if (mean <= 6.0)
+        return list_launch<V, 4>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
+    if (mean <= 24.0)
+        return list_launch<V, 8>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
+    if (mean <= 64.0)
+        return list_launch<V, 16>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
+    return list_launch<V, 32>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
+}
+
+// Forward (Xf == nullptr) or adjoint (Xf = forward solution, B = dL/dx, X = dL/db,
+// G = dL/dA or nullptr) over every system of a list handle.
+sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B, void *X,
+                          const void *Xf, void *G, const sla_pcg_opts *opts, sla_pcg_info *info,
+                          cudaStream_t s)
+{
+    if (M && M->kind != 1)
+        return fail(SLA_ERR_UNSUPPORTED, "list solves support the Jacobi preconditioner or none");
+    if ((size_t)7 * A->max_sys_n * (A->dtype == SLA_F32 ? 4 : 8) > 200 * 1024)
+        return fail(SLA_ERR_UNSUPPORTED, "list solve: largest system exceeds the shared-memory size");
+    const double tol = (opts && opts->rtol > 0) ? opts->rtol : (A->dtype == SLA_F32 ? 1e-6 : 1e-10);
+    const long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 0;
+    sla_pcg_info *d_info = nullptr;
+    SLA_CUDA_TRY(cudaMallocAsync((void **)&d_info, sizeof(sla_pcg_info) * (size_t)A->batch, s));
+    sla_status st;
+    if (A->dtype == SLA_F32)
+        st = list_v<float>(A, M ? (const float *)M->d_dinv : nullptr, B, X, Xf, G, tol, maxit, d_info, s);
+    else
+        st = list_v<double>(A, M ? (const double *)M->d_dinv : nullptr, B, X, Xf, G, tol, maxit, d_info, s);
+    if (st == SLA_SUCCESS) {
+        cudaError_t e = cudaMemcpyAsync(info, d_info, sizeof(sla_pcg_info) * (size_t)A->batch,
+                                        cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess)
+            e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess)
+            st = cuda_fail(e, "list solve result copy");
+    }
+    cudaFreeAsync(d_info, s);
+    if (st != SLA_SUCCESS)
+        return st;
+    sla_status worst = SLA_SUCCESS;
+    for (int i = 0; i < A->batch; ++i)
+        worst = std::max(worst, (sla_status)info[i].status);
+    return worst;
+}
+
+}  // namespace sla

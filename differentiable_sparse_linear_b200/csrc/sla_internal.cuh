@@ -1,0 +1,167 @@
+// Internal declarations of libsla: handles, device solver state, launch helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <map>
+#include <string>
+#include <vector>
+
+#include "sla.h"
+
+namespace sla {
+
+// ------------------------------------------------------------------ error reporting
+void set_error(const std::string &msg);
+sla_status fail(sla_status code, const std::string &msg);
+sla_status cuda_fail(cudaError_t e, const char *what);
+
+#define SLA_CUDA_TRY(expr)                                                   \
+    do {                                                                     \
+        cudaError_t _e = (expr);                                             \
+        if (_e != cudaSuccess) return ::sla::cuda_fail(_e, #expr);           \
+    } while (0)
+
+#define SLA_TRY(expr)                                                        \
+    do {                                                                     \
+        sla_status _s = (expr);                                              \
+        if (_s != SLA_SUCCESS) return _s;                                    \
+    } while (0)
+
+// ------------------------------------------------------------------ limits
+constexpr int KMAX = 16;            // right-hand sides handled by one solve
+constexpr int NPMAX = 2;            // dot products one kernel reduces per right-hand side
+
+// ------------------------------------------------------------------ device solver state
+// One per solve plan.  Scalars of the recurrence (fp64), per right-hand side, plus the
+// loop control the device reads: `active` per RHS, `all_done`, and the last-block ticket.
+struct PcgState {
+    double rho[KMAX];
+    double alpha[KMAX];
+    double beta[KMAX];
+    double bnorm[KMAX];
+    double relres[KMAX];
+    long long iters[KMAX];
+    int status[KMAX];
+    int active[KMAX];
+    int all_done;
+    int phase0;             // 1 while the initial (k = 0) pass runs
+    unsigned int ticket;    // completed-block counter of the running reduction kernel
+    int k;                  // number of RHS slots in use (<= KMAX)
+    double tol;
+    long long maxit;
+    double eps;             // SPAI shift
+    unsigned long long cond_handle;   // cudaGraphConditionalHandle of the solve loop
+    int has_cond;
+    int profile;            // 1: kernels run for timing only; finalisation is skipped
+};
+
+// ------------------------------------------------------------------ tiles
+// Row partition for the load-balanced SpMV: tile t holds rows [tile_row[t], tile_row[t+1]).
+// A tile holds at most D "items" (rows + stored entries) unless it is one single row
+// longer than that (a "long row" tile, reduced by the whole block).
+struct TilePart {
+    int D = 0;
+    int n_tiles = 0;
+    int32_t *d_tile_row = nullptr;
+};
+
+// Read-only view of a CSR matrix passed to kernels.
+template <typename V>
+struct MatView {
+    const int32_t *rp;
+    const int32_t *ci;
+    const V *val;
+    const int32_t *tile_row;
+    int n_tiles;
+    int64_t n;
+};
+
+struct Plan;
+
+}  // namespace sla
+
+// ------------------------------------------------------------------ public handle types
+struct sla_csr {
+    int64_t n = 0, nnz = 0;
+    sla_dtype dtype = SLA_F64;
+    uint32_t flags = 0;
+    const int32_t *rp = nullptr;
+    const int32_t *ci = nullptr;
+    const void *val = nullptr;
+    // owned arrays (used by the internal G^T handle)
+    int32_t *own_rp = nullptr, *own_ci = nullptr;
+    void *own_val = nullptr;
+    // list of systems (block diagonal)
+    int32_t batch = 1;
+    std::vector<int64_t> sys_off;          // host, batch+1
+    int64_t *d_sys_off = nullptr;          // device copy
+    int64_t max_sys_n = 0;
+    int64_t max_sys_nnz = 0;
+    // host copy of row_ptr, for partition building
+    std::vector<int32_t> h_rp;
+    std::map<int, sla::TilePart> tiles;    // by item budget D
+    int device = 0;
+    int num_sms = 148;
+    std::vector<sla::Plan *> plans;
+    int64_t max_row_len = 0;
+};
+
+struct sla_precond {
+    int kind = 0;                          // 1 Jacobi, 2 SPAI
+    const sla_csr *A = nullptr;
+    const sla_csr *G = nullptr;            // borrowed (SPAI)
+    sla_csr *GT = nullptr;                 // owned explicit transpose (SPAI)
+    double eps = 0.0;
+    void *d_dinv = nullptr;                // Jacobi: 1 / A_ii in A's dtype
+    int32_t *d_perm = nullptr;             // SPAI: position in G of each G^T entry
+};
+
+namespace sla {
+
+// Solve plan: workspace + captured graph for one (A, M, K) combination.
+struct Plan {
+    const sla_precond *M = nullptr;
+    int K = 1;
+    int kind = 0;                          // 0 none, 1 Jacobi, 2 SPAI
+    void *ws = nullptr;                    // one device allocation
+    size_t ws_bytes = 0;
+    void *x = nullptr, *ra = nullptr, *rb = nullptr, *pa = nullptr, *pb = nullptr;
+    void *q = nullptr, *z = nullptr, *y = nullptr;
+    double *partials = nullptr;
+    PcgState *st = nullptr;
+    PcgState *h_st = nullptr;              // pinned host mirror for the final read
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    cudaStream_t cs = nullptr, cs2 = nullptr;
+    int grid_tiles_A = 0, grid_tiles_G = 0, grid_tiles_GT = 0, grid_vec = 0;
+    unsigned long long cond = 0;           // conditional handle of the loop node
+};
+
+// ------------------------------------------------------------------ internal entry points
+sla_status ensure_tiles(sla_csr *A, int D, cudaStream_t s, const TilePart **out);
+size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K);
+sla_status get_plan(sla_csr *A, const sla_precond *M, int K, Plan **out);
+void destroy_plan(Plan *p);
+
+// launchers implemented in the .cu files
+sla_status launch_spmv(const sla_csr *A, int K, const void *x, void *y, cudaStream_t s);
+sla_status launch_pattern_grad(const sla_csr *A, int K, const void *lam, const void *x, void *g,
+                               cudaStream_t s);
+sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s);
+sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv, int *d_err, cudaStream_t s);
+sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t *d_perm,
+                                    cudaStream_t s);
+sla_status capture_plan_graph(sla_csr *A, Plan *p);
+// Solve with the plan; with grad_out set, also form dL/dA = -X (x) grad_x on A's pattern
+// (X = lambda) before the single final synchronisation.
+sla_status run_plan(sla_csr *A, Plan *p, int nrhs, const void *B, void *X,
+                    const sla_pcg_opts *opts, sla_pcg_info *info, const void *grad_x,
+                    void *grad_out, cudaStream_t s);
+sla_status kernel_times(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s);
+sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B, void *X,
+                          const void *Xfwd, void *G, const sla_pcg_opts *opts, sla_pcg_info *info,
+                          cudaStream_t s);
+
+}  // namespace sla

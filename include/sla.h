@@ -1,0 +1,211 @@
+/*
+ * sla.h -- C ABI of the B200 (sm_100a) sparse SPD solver library `libsla`.
+ *
+ * The library solves A x = b for a sparse symmetric positive definite A stored in CSR by
+ * the preconditioned conjugate-gradient method, and provides the adjoint (backward) pass:
+ *
+ *   forward   x = A^-1 b                                   (PCG, Jacobi or SPAI preconditioner)
+ *   backward  A^T lambda = dL/dx,  dL/db = lambda,  dL/dA_ij = -lambda_i x_j on A's pattern
+ *
+ * Sources (page title, section):
+ *   [TS]   "torch-sla: Differentiable Sparse Linear Algebra with Adjoint Solvers and Sparse
+ *          Tensor Parallelism for PyTorch": Methodology §1 (the .solve / .matvec API; the
+ *          Jacobi-preconditioned native iterative backend; SparseTensor = one matrix or a
+ *          batch sharing one pattern, SparseTensorList = a batch with distinct patterns),
+ *          Methodology §2 "Linear Systems" (the adjoint), Complexity (O(1) graph nodes,
+ *          O(n + nnz) memory, independent of the iteration count).
+ *   [SPAI] "Learning Sparse Approximate Inverse Preconditioners for Conjugate Gradient
+ *          Solvers on GPUs": Approach (M^-1 = G G^T + eps I, G on A's pattern, two SpMVs
+ *          per CG step) and the epsilon ablation (default eps = 3e-3).
+ *
+ * Conventions common to every call
+ *   - Pointers prefixed d_ are DEVICE pointers on the current CUDA device; h_ are HOST
+ *     pointers.  Indices are int32 (row_ptr, col); values are fp32 or fp64 (sla_dtype).
+ *     Vectors have the matrix's value type: fp32 matrices use fp32 vectors with all dot
+ *     products, norms and the scalars alpha, beta, rho in fp64.
+ *   - Multi-right-hand-side blocks are [n][nrhs] row-major ("interleaved"): entry (i, c)
+ *     is at i * nrhs + c.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All
+ *     device work is enqueued on it.  Calls that return solver results (sla_pcg_*)
+ *     synchronise that stream once, at the end, to fill the info structs; no call
+ *     synchronises per iteration.
+ *   - Ownership: the caller owns every d_ buffer and keeps the arrays passed to
+ *     sla_csr_create alive and unchanged (pattern) for the handle's lifetime; values may be
+ *     changed in place between calls (then call sla_precond_refresh).  The library owns its
+ *     handles, workspaces, the explicit G^T, Jacobi's D^-1 and the captured CUDA graphs; the
+ *     matching _destroy call frees them.
+ *   - Errors: every call returns an sla_status.  Negative values are errors and leave
+ *     outputs unspecified; sla_last_error() gives a thread-local message.  Solver outcomes
+ *     SLA_NOT_CONVERGED and SLA_BREAKDOWN are positive: the outputs hold the last iterate.
+ *   - Handles are not thread-safe: one host thread at a time per handle.
+ */
+#ifndef SLA_H
+#define SLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SLA_API __attribute__((visibility("default")))
+#else
+#define SLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t sla_status;
+#define SLA_SUCCESS 0
+#define SLA_NOT_CONVERGED 1       /* maxit reached; x holds the last iterate           */
+#define SLA_BREAKDOWN 2           /* p.q <= 0, r.z <= 0 or a non-finite value: A or M   */
+                                  /* is not SPD (or the input holds NaN/Inf)            */
+#define SLA_ERR_INVALID_ARG (-1)  /* null pointer, bad size, dtype or handle mismatch   */
+#define SLA_ERR_INVALID_CSR (-2)  /* SLA_VALIDATE found a malformed pattern             */
+#define SLA_ERR_CUDA (-3)         /* a CUDA runtime call failed                         */
+#define SLA_ERR_OOM (-4)          /* device or host allocation failed                   */
+#define SLA_ERR_UNSUPPORTED (-5)  /* valid request outside what this build implements   */
+
+typedef enum { SLA_F32 = 0, SLA_F64 = 1 } sla_dtype;
+
+/* Flags for sla_csr_create*. */
+#define SLA_SPD 1u        /* caller asserts A is symmetric positive definite (needed by PCG) */
+#define SLA_VALIDATE 2u   /* check the pattern on the device: row_ptr[0] = 0, row_ptr non-  */
+                          /* decreasing, row_ptr[n] = nnz, columns in range, strictly        */
+                          /* ascending in each row (so duplicates are rejected, not summed)  */
+
+typedef struct sla_csr sla_csr;
+typedef struct sla_precond sla_precond;
+
+/* Solver options.  Zero-initialised fields take the defaults given. */
+typedef struct {
+    double rtol;        /* stop when ||r_k||_2 / ||b||_2 <= rtol on the recursive residual;
+                           0 -> 1e-10 for fp64, 1e-6 for fp32                              */
+    int64_t maxit;      /* iteration cap per right-hand side; 0 -> 10 * n (n of the system) */
+    int32_t reserved0;
+    int32_t reserved1;
+} sla_pcg_opts;
+
+/* Per right-hand side (or per system of a list) solver outcome. */
+typedef struct {
+    int64_t iters;      /* number of products q = A p taken (0 when b = 0)                   */
+    double relres;      /* ||r||/||b|| of the recursive residual at exit (0 when b = 0)      */
+    int32_t status;     /* SLA_SUCCESS, SLA_NOT_CONVERGED or SLA_BREAKDOWN                   */
+    int32_t reserved;
+} sla_pcg_info;
+
+/* ---------------------------------------------------------------- library */
+SLA_API const char *sla_version(void);
+SLA_API const char *sla_status_string(sla_status s);
+/* Message of the last failing call on this host thread ("" if none). */
+SLA_API const char *sla_last_error(void);
+
+/* ---------------------------------------------------------------- matrices */
+/* One square CSR matrix ([TS] Methodology §1, SparseTensor).
+ * n_rows == n_cols is required (the solver works on square SPD systems); nnz = row_ptr[n].
+ * d_row_ptr (n+1), d_col (nnz), d_val (nnz, `dtype`) are borrowed, not copied.
+ * Set-up work (load-balanced tile partition of the rows, optional validation) runs on
+ * `stream` and is synchronised before return.  Returns SLA_ERR_INVALID_CSR on a pattern
+ * that fails SLA_VALIDATE. */
+SLA_API sla_status sla_csr_create(sla_csr **out, int64_t n_rows, int64_t n_cols, int64_t nnz,
+                          const int32_t *d_row_ptr, const int32_t *d_col, const void *d_val,
+                          sla_dtype dtype, uint32_t flags, void *stream);
+
+/* A batch of independent systems with distinct patterns ([TS] Methodology §1,
+ * SparseTensorList), stored as ONE block-diagonal CSR of n_total rows: system s owns rows
+ * and columns [h_sys_row_off[s], h_sys_row_off[s+1]); h_sys_row_off (host, batch+1 entries,
+ * h_sys_row_off[0] = 0, last = n_total) is copied.  Column indices are global and must lie in
+ * the owning system's range (checked by SLA_VALIDATE).  sla_spmv works on the whole block
+ * matrix; sla_pcg_solve_batched / sla_pcg_adjoint_batched solve every system on its own,
+ * each with its own stopping test and info entry. */
+SLA_API sla_status sla_csr_create_list(sla_csr **out, int32_t batch, const int64_t *h_sys_row_off,
+                               int64_t nnz_total, const int32_t *d_row_ptr, const int32_t *d_col,
+                               const void *d_val, sla_dtype dtype, uint32_t flags, void *stream);
+
+SLA_API sla_status sla_csr_destroy(sla_csr *A);
+
+/* n_rows, nnz and batch (1 for a single matrix) of a handle; any output may be NULL. */
+SLA_API sla_status sla_csr_shape(const sla_csr *A, int64_t *n_rows, int64_t *nnz, int32_t *batch);
+
+/* y = A x ([TS] Methodology §1, .matvec).  d_x, d_y: n vectors of A's dtype, must not
+ * overlap.  Accumulates each row in fp64 and rounds once to the value type. */
+SLA_API sla_status sla_spmv(const sla_csr *A, const void *d_x, void *d_y, void *stream);
+
+/* Y = A X for nrhs right-hand sides in [n][nrhs] layout (1 <= nrhs <= 16). */
+SLA_API sla_status sla_spmv_multi(const sla_csr *A, int32_t nrhs, const void *d_X, void *d_Y, void *stream);
+
+/* ---------------------------------------------------------------- preconditioners */
+/* Jacobi: M^-1 = D^-1, D = diag(A) ([TS] Methodology §1, the native backend's
+ * preconditioner).  Every row must store a positive diagonal entry, else
+ * SLA_ERR_INVALID_ARG.  The preconditioner belongs to A and must be used with A only. */
+SLA_API sla_status sla_precond_jacobi(sla_precond **out, const sla_csr *A, void *stream);
+
+/* SPAI: M^-1 = G G^T + eps I ([SPAI] Approach).  G is a square CSR of A's size (it normally
+ * carries A's lower-triangular pattern; any pattern is accepted), borrowed like A; the
+ * library forms and owns G^T explicitly so each apply is two plain SpMVs.  For a list
+ * handle A, G must be block-diagonal with the same blocks. */
+SLA_API sla_status sla_precond_spai(sla_precond **out, const sla_csr *A, const sla_csr *G, double eps,
+                            void *stream);
+
+/* Recompute what the preconditioner derives from A's or G's values (D^-1, G^T values)
+ * after the caller changed them in place. */
+SLA_API sla_status sla_precond_refresh(sla_precond *M, void *stream);
+
+SLA_API sla_status sla_precond_destroy(sla_precond *M);
+
+/* ---------------------------------------------------------------- solves */
+/* x = A^-1 b by PCG from x0 = 0 ([TS] Methodology §1 .solve; [SPAI] Approach).
+ * M may be NULL (plain CG).  d_b, d_x: n vectors; may not overlap.  On SLA_SUCCESS,
+ * ||r||/||b|| <= rtol for the recursive residual r.  b = 0 gives x = 0 and iters = 0.
+ * info may be NULL.  Workspace is O(n) and does not grow with the iteration count. */
+SLA_API sla_status sla_pcg_solve(const sla_csr *A, const sla_precond *M, const void *d_b, void *d_x,
+                         const sla_pcg_opts *opts, sla_pcg_info *info, void *stream);
+
+/* Adjoint of x = A^-1 b ([TS] Methodology §2, Linear Systems): solves A^T lambda = dL/dx
+ * with the same PCG and preconditioner (A is SPD, so A^T = A), writes dL/db = lambda (n)
+ * and dL/dA_k = -lambda_row(k) * x_col(k) for every stored entry k (nnz, aligned with A's
+ * values).  d_x is the forward solution.  d_dLdA may be NULL to skip the gradient. */
+SLA_API sla_status sla_pcg_adjoint(const sla_csr *A, const sla_precond *M, const void *d_x,
+                           const void *d_dLdx, void *d_dLdb, void *d_dLdA,
+                           const sla_pcg_opts *opts, sla_pcg_info *info, void *stream);
+
+/* Batched solve.  For a single matrix: nrhs (1..16) right-hand sides in [n][nrhs] layout
+ * sharing A, each with its own stopping test; h_info has nrhs entries.  For a list handle:
+ * nrhs must be 1, d_B/d_X are the concatenated n_total vectors and h_info has `batch`
+ * entries. */
+SLA_API sla_status sla_pcg_solve_batched(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                 const void *d_B, void *d_X, const sla_pcg_opts *opts,
+                                 sla_pcg_info *h_info, void *stream);
+
+/* Batched adjoint.  Single matrix: Lambda (= dL/dB) per RHS, dL/dA summed over the RHS
+ * (sum_c -lambda_c,i x_c,j).  List handle: per system, concatenated (each system's block
+ * of dL/dA is its own gradient). */
+SLA_API sla_status sla_pcg_adjoint_batched(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                   const void *d_X, const void *d_dLdX, void *d_dLdB,
+                                   void *d_dLdA, const sla_pcg_opts *opts, sla_pcg_info *h_info,
+                                   void *stream);
+
+/* dL/dA_k = -sum_c lambda_c,row(k) * x_c,col(k) on A's pattern, for nrhs vectors in
+ * [n][nrhs] layout ([TS] Methodology §2; with lambda = x = v it is the Hellmann-Feynman
+ * eigenvalue gradient of the same section up to sign). */
+SLA_API sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *d_lam, const void *d_x,
+                            void *d_g, void *stream);
+
+/* Per-kernel device time of one PCG iteration (metrics).  On the workspace of the
+ * (A, M, nrhs) solver -- normally right after a solve, so it holds that solve's vectors --
+ * launches the iteration's kernels `reps` times in loop order, each bracketed by CUDA
+ * events on `stream`, with the scalar updates switched off, and writes the mean ms per
+ * launch to h_ms[0..2]: [0] p-update + q = A p, [1] the x/r update (Jacobi: with z = D^-1 r;
+ * SPAI: with y = G^T r), [2] z = G y + eps r (SPAI; 0 otherwise).  The workspace contents
+ * are unspecified afterwards (the next solve re-initialises them).  Synchronises `stream`. */
+SLA_API sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                        int32_t reps, double *h_ms, void *stream);
+
+/* Device bytes the solver workspace takes for (A, M, nrhs); it depends on n and nnz only,
+ * never on the iteration count ([TS] Complexity). */
+SLA_API size_t sla_workspace_bytes(const sla_csr *A, const sla_precond *M, int32_t nrhs);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLA_H */
