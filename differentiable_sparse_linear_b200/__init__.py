@@ -90,10 +90,11 @@ def _infos(arr) -> list[PcgInfo]:
     return [PcgInfo(int(a.iters), float(a.relres), int(a.status)) for a in arr]
 
 
-def _opts(rtol: float, maxit: int) -> _lib.sla_pcg_opts:
+def _opts(rtol: float, maxit: int, vector_f64: bool = False) -> _lib.sla_pcg_opts:
     o = _lib.sla_pcg_opts()
     o.rtol = float(rtol)
     o.maxit = int(maxit)
+    o.vector_f64 = 1 if vector_f64 else 0
     return o
 
 
@@ -167,6 +168,12 @@ def _mh(M: Optional[Preconditioner]):
     return None if M is None else M.handle
 
 
+def _check_vec(A: Matrix, v: torch.Tensor, vector_f64: bool):
+    want = torch.float64 if (vector_f64 and A.dtype == torch.float32) else A.dtype
+    if v.dtype != want:
+        raise ValueError(f"vectors must be {want} here (matrix {A.dtype}, vector_f64={vector_f64})")
+
+
 def sla_csr_create(row_ptr: torch.Tensor, col: torch.Tensor, val: torch.Tensor, *,
                    validate: bool = True, spd: bool = True, stream=None) -> Matrix:
     """sla_csr_create: one square CSR matrix (n = row_ptr.numel() - 1)."""
@@ -221,22 +228,26 @@ def sla_precond_spai(A: Matrix, G: Matrix, eps: float = 3e-3, stream=None) -> Pr
 
 def sla_pcg_solve(A: Matrix, M: Optional[Preconditioner], b: torch.Tensor,
                   x: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
-                  stream=None) -> tuple[torch.Tensor, PcgInfo]:
+                  vector_f64: bool = False, stream=None) -> tuple[torch.Tensor, PcgInfo]:
+    """x = A^-1 b.  vector_f64 with an fp32 matrix: b and x are fp64 (mixed precision)."""
+    _check_vec(A, b, vector_f64)
     x = torch.empty_like(b) if x is None else x
     info = _lib.sla_pcg_info()
-    opts = _opts(rtol, maxit)
+    opts = _opts(rtol, maxit, vector_f64)
     _check(lib().sla_pcg_solve(A.handle, _mh(M), _ptr(b), _ptr(x), C.byref(opts), C.byref(info),
                                _stream(stream)), "sla_pcg_solve")
     return x, _infos([info])[0]
 
 
 def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLdx: torch.Tensor, *,
-                    want_dA: bool = True, rtol: float = 0.0, maxit: int = 0, stream=None):
+                    want_dA: bool = True, rtol: float = 0.0, maxit: int = 0, vector_f64: bool = False,
+                    stream=None):
     """Returns (dL/db, dL/dA on A's pattern or None, info)."""
+    _check_vec(A, dLdx, vector_f64)
     dLdb = torch.empty_like(dLdx)
     dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdx.device) if want_dA else None
     info = _lib.sla_pcg_info()
-    opts = _opts(rtol, maxit)
+    opts = _opts(rtol, maxit, vector_f64)
     _check(lib().sla_pcg_adjoint(A.handle, _mh(M), _ptr(x), _ptr(dLdx), _ptr(dLdb), _ptr(dLdA),
                                  C.byref(opts), C.byref(info), _stream(stream)), "sla_pcg_adjoint")
     return dLdb, dLdA, _infos([info])[0]
@@ -244,26 +255,29 @@ def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLd
 
 def sla_pcg_solve_batched(A: Matrix, M: Optional[Preconditioner], B: torch.Tensor,
                           X: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
-                          stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
+                          vector_f64: bool = False, stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
     """Shared matrix: B is [n, nrhs].  List handle: B is the concatenated [n_total] vector."""
+    _check_vec(A, B, vector_f64)
     nrhs = 1 if (B.dim() == 1 or A.batch > 1) else B.shape[1]
     count = A.batch if A.batch > 1 else nrhs
     X = torch.empty_like(B) if X is None else X
     infos = (_lib.sla_pcg_info * count)()
-    opts = _opts(rtol, maxit)
+    opts = _opts(rtol, maxit, vector_f64)
     _check(lib().sla_pcg_solve_batched(A.handle, _mh(M), nrhs, _ptr(B), _ptr(X), C.byref(opts),
                                        infos, _stream(stream)), "sla_pcg_solve_batched")
     return X, _infos(infos)
 
 
 def sla_pcg_adjoint_batched(A: Matrix, M: Optional[Preconditioner], X: torch.Tensor, dLdX: torch.Tensor,
-                            *, want_dA: bool = True, rtol: float = 0.0, maxit: int = 0, stream=None):
+                            *, want_dA: bool = True, rtol: float = 0.0, maxit: int = 0,
+                            vector_f64: bool = False, stream=None):
+    _check_vec(A, dLdX, vector_f64)
     nrhs = 1 if (dLdX.dim() == 1 or A.batch > 1) else dLdX.shape[1]
     count = A.batch if A.batch > 1 else nrhs
     dLdB = torch.empty_like(dLdX)
     dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdX.device) if want_dA else None
     infos = (_lib.sla_pcg_info * count)()
-    opts = _opts(rtol, maxit)
+    opts = _opts(rtol, maxit, vector_f64)
     _check(lib().sla_pcg_adjoint_batched(A.handle, _mh(M), nrhs, _ptr(X), _ptr(dLdX), _ptr(dLdB),
                                          _ptr(dLdA), C.byref(opts), infos, _stream(stream)),
            "sla_pcg_adjoint_batched")
@@ -280,25 +294,26 @@ def sla_pattern_grad(A: Matrix, lam: torch.Tensor, x: torch.Tensor, g: Optional[
 
 
 def sla_pcg_kernel_times(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1, reps: int = 20,
-                         stream=None) -> list[float]:
+                         vector_f64: bool = False, stream=None) -> list[float]:
     """Mean ms per launch of the iteration's kernels: [q = A p, x/r update, z = G y + eps r]."""
     out = (C.c_double * 3)()
-    _check(lib().sla_pcg_kernel_times(A.handle, _mh(M), nrhs, reps, out, _stream(stream)),
-           "sla_pcg_kernel_times")
+    _check(lib().sla_pcg_kernel_times(A.handle, _mh(M), nrhs, 1 if vector_f64 else 0, reps, out,
+                                      _stream(stream)), "sla_pcg_kernel_times")
     return list(out)
 
 
-def sla_workspace_bytes(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1) -> int:
-    return int(lib().sla_workspace_bytes(A.handle, _mh(M), nrhs))
+def sla_workspace_bytes(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1,
+                        vector_f64: bool = False) -> int:
+    return int(lib().sla_workspace_bytes(A.handle, _mh(M), nrhs, 1 if vector_f64 else 0))
 
 
 class _Solve(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, val, b, A, M, rtol, maxit):
-        x, info = sla_pcg_solve(A, M, b, rtol=rtol, maxit=maxit)
+    def forward(ctx, val, b, A, M, rtol, maxit, vector_f64):
+        x, info = sla_pcg_solve(A, M, b, rtol=rtol, maxit=maxit, vector_f64=vector_f64)
         if info.status == SLA_BREAKDOWN:
             raise SlaError(SLA_BREAKDOWN, "solve")
-        ctx.A, ctx.M, ctx.rtol, ctx.maxit = A, M, rtol, maxit
+        ctx.A, ctx.M, ctx.rtol, ctx.maxit, ctx.vf64 = A, M, rtol, maxit, vector_f64
         ctx.info = info
         ctx.save_for_backward(x)
         return x
@@ -308,15 +323,15 @@ class _Solve(torch.autograd.Function):
         (x,) = ctx.saved_tensors
         need_A = ctx.needs_input_grad[0]
         dLdb, dLdA, info = sla_pcg_adjoint(ctx.A, ctx.M, x, gx.contiguous(), want_dA=need_A,
-                                           rtol=ctx.rtol, maxit=ctx.maxit)
-        return dLdA, dLdb, None, None, None, None
+                                           rtol=ctx.rtol, maxit=ctx.maxit, vector_f64=ctx.vf64)
+        return dLdA, dLdb, None, None, None, None, None
 
 
 def solve(A: Matrix, b: torch.Tensor, M: Optional[Preconditioner] = None, *, rtol: float = 0.0,
-          maxit: int = 0) -> torch.Tensor:
+          maxit: int = 0, vector_f64: bool = False) -> torch.Tensor:
     """x = A^-1 b, differentiable in A's values (A.val) and in b.
 
     Gradients flow to ``A.val`` if it requires grad; the backward pass is one adjoint PCG
     solve and one pattern-gradient pass, independent of the forward iteration count.
     """
-    return _Solve.apply(A.val, b, A, M, rtol, maxit)
+    return _Solve.apply(A.val, b, A, M, rtol, maxit, vector_f64)

@@ -22,8 +22,8 @@ SLA_VALIDATE = 2
 
 
 class sla_pcg_opts(C.Structure):
-    _fields_ = [("rtol", C.c_double), ("maxit", C.c_int64), ("reserved0", C.c_int32),
-                ("reserved1", C.c_int32)]
+    _fields_ = [("rtol", C.c_double), ("maxit", C.c_int64), ("vector_f64", C.c_int32),
+                ("reserved", C.c_int32)]
 
 
 class sla_pcg_info(C.Structure):
@@ -59,8 +59,8 @@ SIGNATURES = {
     "sla_pcg_adjoint_batched": (_st, [_vp, _vp, C.c_int32, _vp, _vp, _vp, _vp,
                                       C.POINTER(sla_pcg_opts), C.POINTER(sla_pcg_info), _vp]),
     "sla_pattern_grad": (_st, [_vp, C.c_int32, _vp, _vp, _vp, _vp]),
-    "sla_pcg_kernel_times": (_st, [_vp, _vp, C.c_int32, C.c_int32, C.POINTER(C.c_double), _vp]),
-    "sla_workspace_bytes": (C.c_size_t, [_vp, _vp, C.c_int32]),
+    "sla_pcg_kernel_times": (_st, [_vp, _vp, C.c_int32, C.c_int32, C.c_int32, C.POINTER(C.c_double), _vp]),
+    "sla_workspace_bytes": (C.c_size_t, [_vp, _vp, C.c_int32, C.c_int32]),
 }
 
 _lib = None

@@ -33,55 +33,63 @@ sla_status cuda_fail(cudaError_t e, const char *what)
 
 static size_t vbytes(sla_dtype d) { return d == SLA_F32 ? 4 : 8; }
 
-// Rows grouped into tiles of at most D items (rows + entries); a row with more than D-1
-// entries forms a tile of its own.
-sla_status ensure_tiles(sla_csr *A, int D, cudaStream_t s, const TilePart **out)
+// Rows grouped into tiles of at most D items (rows + entries) and at most RMAX rows; a row
+// with D or more entries forms a tile of its own.  desc[t] = {first row, first entry}.
+sla_status ensure_tiles(sla_csr *A, int D, int RMAX, cudaStream_t s, const TilePart **out)
 {
-    auto it = A->tiles.find(D);
+    const int key = D * 65536 + RMAX;
+    auto it = A->tiles.find(key);
     if (it != A->tiles.end()) {
         *out = &it->second;
         return SLA_SUCCESS;
     }
     std::vector<int32_t> t;
-    t.reserve((size_t)(A->n + A->nnz) / (size_t)D + 16);
+    t.reserve((size_t)(A->n + A->nnz) / (size_t)D + (size_t)A->n / (size_t)RMAX + 16);
     t.push_back(0);
-    int64_t items = 0;
+    int64_t items = 0, rows = 0;
     for (int64_t r = 0; r < A->n; ++r) {
         const int64_t len = (int64_t)A->h_rp[r + 1] - A->h_rp[r];
         if (len + 1 > D) {
             if (items > 0) {
                 t.push_back((int32_t)r);
-                items = 0;
+                items = rows = 0;
             }
             t.push_back((int32_t)(r + 1));
             continue;
         }
-        if (items + len + 1 > D) {
+        if (items + len + 1 > D || rows + 1 > RMAX) {
             t.push_back((int32_t)r);
-            items = 0;
+            items = rows = 0;
         }
         items += len + 1;
+        rows += 1;
     }
     if (items > 0)
         t.push_back((int32_t)A->n);
+    std::vector<int2> desc(t.size());
+    for (size_t i = 0; i < t.size(); ++i)
+        desc[i] = make_int2(t[i], A->h_rp[(size_t)t[i]]);
     TilePart tp;
     tp.D = D;
+    tp.RMAX = RMAX;
     tp.n_tiles = (int)t.size() - 1;
-    SLA_CUDA_TRY(cudaMalloc((void **)&tp.d_tile_row, t.size() * sizeof(int32_t)));
-    SLA_CUDA_TRY(cudaMemcpyAsync(tp.d_tile_row, t.data(), t.size() * sizeof(int32_t),
+    SLA_CUDA_TRY(cudaMalloc((void **)&tp.d_desc, desc.size() * sizeof(int2)));
+    SLA_CUDA_TRY(cudaMemcpyAsync(tp.d_desc, desc.data(), desc.size() * sizeof(int2),
                                  cudaMemcpyHostToDevice, s));
     SLA_CUDA_TRY(cudaStreamSynchronize(s));
-    auto ins = A->tiles.emplace(D, tp);
+    auto ins = A->tiles.emplace(key, tp);
     *out = &ins.first->second;
     return SLA_SUCCESS;
 }
 
 static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K)
+static size_t vec_bytes(const sla_csr *A, int vec64) { return vec64 ? 8 : vbytes(A->dtype); }
+
+size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K, int vec64)
 {
     (void)M;
-    const size_t vec = align256((size_t)A->n * (size_t)K * vbytes(A->dtype));
+    const size_t vec = align256((size_t)A->n * (size_t)K * vec_bytes(A, vec64));
     const size_t parts = align256((size_t)A->num_sms * 32 * 2 * KMAX * sizeof(double));
     return 8 * vec + parts + align256(sizeof(PcgState));
 }
@@ -105,18 +113,20 @@ void destroy_plan(Plan *p)
     delete p;
 }
 
-sla_status get_plan(sla_csr *A, const sla_precond *M, int K, Plan **out)
+sla_status get_plan(sla_csr *A, const sla_precond *M, int K, int vec64, Plan **out)
 {
+    vec64 = (vec64 && A->dtype == SLA_F32) ? 1 : 0;
     for (Plan *p : A->plans)
-        if (p->M == M && p->K == K) {
+        if (p->M == M && p->K == K && p->vec64 == vec64) {
             *out = p;
             return SLA_SUCCESS;
         }
     Plan *p = new Plan();
     p->M = M;
     p->K = K;
+    p->vec64 = vec64;
     p->kind = M ? M->kind : 0;
-    p->ws_bytes = plan_bytes(A, M, K);
+    p->ws_bytes = plan_bytes(A, M, K, vec64);
     auto cleanup = [&](sla_status st) {
         destroy_plan(p);
         return st;
@@ -127,7 +137,7 @@ sla_status get_plan(sla_csr *A, const sla_precond *M, int K, Plan **out)
     e = cudaMallocHost((void **)&p->h_st, sizeof(PcgState));
     if (e != cudaSuccess)
         return cleanup(cuda_fail(e, "pinned solver state"));
-    const size_t vec = align256((size_t)A->n * (size_t)K * vbytes(A->dtype));
+    const size_t vec = align256((size_t)A->n * (size_t)K * vec_bytes(A, vec64));
     char *b = (char *)p->ws;
     void **vs[8] = {&p->x, &p->ra, &p->rb, &p->pa, &p->pb, &p->q, &p->z, &p->y};
     for (int i = 0; i < 8; ++i) {
@@ -154,6 +164,8 @@ static sla_status current_device(sla_csr *A)
 {
     SLA_CUDA_TRY(cudaGetDevice(&A->device));
     SLA_CUDA_TRY(cudaDeviceGetAttribute(&A->num_sms, cudaDevAttrMultiProcessorCount, A->device));
+    SLA_CUDA_TRY(cudaMalloc((void **)&A->d_err, sizeof(int)));
+    SLA_CUDA_TRY(cudaMemset(A->d_err, 0, sizeof(int)));
     return SLA_SUCCESS;
 }
 
@@ -200,15 +212,45 @@ static sla_status setup_pattern(sla_csr *A, uint32_t flags, cudaStream_t s)
     return SLA_SUCCESS;
 }
 
+static void drop_plans_of(sla_csr *A, const sla_precond *M)
+{
+    std::vector<Plan *> keep;
+    for (Plan *p : A->plans) {
+        if (p->M == M)
+            destroy_plan(p);
+        else
+            keep.push_back(p);
+    }
+    A->plans.swap(keep);
+}
+
+static void unlink(std::vector<sla_precond *> &v, const sla_precond *M)
+{
+    v.erase(std::remove(v.begin(), v.end(), M), v.end());
+}
+
 static void free_csr(sla_csr *A)
 {
     if (!A)
         return;
+    // detach the preconditioners that refer to A: their plans live in their matrix and
+    // may reference A's arrays (as A or as G), so they go first
+    for (sla_precond *M : A->dependents) {
+        if (M->A && M->A != A)
+            drop_plans_of(const_cast<sla_csr *>(M->A), M);
+        if (M->A == A)
+            M->A = nullptr;
+        if (M->G == A)
+            M->G = nullptr;   // a SPAI preconditioner without G refuses further use
+    }
+    A->dependents.clear();
     for (Plan *p : A->plans)
         destroy_plan(p);
     A->plans.clear();
     for (auto &kv : A->tiles)
-        cudaFree(kv.second.d_tile_row);
+        cudaFree(kv.second.d_desc);
+    if (A->d_err)
+        cudaFree(A->d_err);
     if (A->d_sys_off)
         cudaFree(A->d_sys_off);
     if (A->own_rp)
@@ -383,7 +425,7 @@ static sla_status jacobi_setup(sla_precond *M, cudaStream_t s)
     int *d_err = nullptr;
     SLA_CUDA_TRY(cudaMallocAsync((void **)&d_err, sizeof(int), s));
     SLA_CUDA_TRY(cudaMemsetAsync(d_err, 0, sizeof(int), s));
-    sla_status st = launch_jacobi_dinv(A, M->d_dinv, d_err, s);
+    sla_status st = launch_jacobi_dinv(A, M->d_dinv64, M->d_dinv, d_err, s);
     int h_err = 0;
     if (st == SLA_SUCCESS) {
         cudaError_t e = cudaMemcpyAsync(&h_err, d_err, sizeof(int), cudaMemcpyDeviceToHost, s);
@@ -409,17 +451,24 @@ sla_status sla_precond_jacobi(sla_precond **out, const sla_csr *A, void *stream)
     sla_precond *M = new sla_precond();
     M->kind = 1;
     M->A = A;
-    cudaError_t e = cudaMalloc(&M->d_dinv, (size_t)std::max<int64_t>(A->n, 1) * vbytes(A->dtype));
+    const size_t nb = (size_t)std::max<int64_t>(A->n, 1);
+    cudaError_t e = cudaMalloc(&M->d_dinv64, nb * sizeof(double));
+    if (e == cudaSuccess && A->dtype == SLA_F32)
+        e = cudaMalloc(&M->d_dinv, nb * sizeof(float));
     if (e != cudaSuccess) {
+        cudaFree(M->d_dinv64);
         delete M;
         return cuda_fail(e, "Jacobi D^-1");
     }
     sla_status st = jacobi_setup(M, s);
     if (st != SLA_SUCCESS) {
-        cudaFree(M->d_dinv);
+        cudaFree(M->d_dinv64);
+        if (M->d_dinv)
+            cudaFree(M->d_dinv);
         delete M;
         return st;
     }
+    const_cast<sla_csr *>(A)->dependents.push_back(M);
     *out = M;
     return SLA_SUCCESS;
 }
@@ -491,17 +540,15 @@ static void free_precond(sla_precond *M)
         return;
     if (M->A) {
         sla_csr *A = const_cast<sla_csr *>(M->A);
-        std::vector<Plan *> keep;
-        for (Plan *p : A->plans) {
-            if (p->M == M)
-                destroy_plan(p);
-            else
-                keep.push_back(p);
-        }
-        A->plans.swap(keep);
+        drop_plans_of(A, M);
+        unlink(A->dependents, M);
     }
+    if (M->G)
+        unlink(const_cast<sla_csr *>(M->G)->dependents, M);
     if (M->d_dinv)
         cudaFree(M->d_dinv);
+    if (M->d_dinv64)
+        cudaFree(M->d_dinv64);
     if (M->d_perm)
         cudaFree(M->d_perm);
     if (M->GT)
@@ -527,9 +574,13 @@ sla_status sla_precond_spai(sla_precond **out, const sla_csr *A, const sla_csr *
     sla_status st = spai_transpose(M, (cudaStream_t)stream);
     if (st != SLA_SUCCESS) {
         M->A = nullptr;
+        M->G = nullptr;
         free_precond(M);
         return st;
     }
+    const_cast<sla_csr *>(A)->dependents.push_back(M);
+    if (G != A)
+        const_cast<sla_csr *>(G)->dependents.push_back(M);
     *out = M;
     return SLA_SUCCESS;
 }
@@ -539,6 +590,8 @@ sla_status sla_precond_refresh(sla_precond *M, void *stream)
     if (!M)
         return fail(SLA_ERR_INVALID_ARG, "NULL preconditioner");
     cudaStream_t s = (cudaStream_t)stream;
+    if (!M->A || (M->kind == 2 && !M->G))
+        return fail(SLA_ERR_INVALID_ARG, "a handle this preconditioner was built from was destroyed");
     if (M->kind == 1)
         return jacobi_setup(M, s);
     SLA_TRY(refresh_transpose_values(M->G, M->GT, M->d_perm, s));
@@ -559,6 +612,8 @@ static sla_status check_solve(const sla_csr *A, const sla_precond *M)
         return fail(SLA_ERR_INVALID_ARG, "NULL matrix handle");
     if (M && M->A != A)
         return fail(SLA_ERR_INVALID_ARG, "the preconditioner was built for another matrix handle");
+    if (M && M->kind == 2 && !M->G)
+        return fail(SLA_ERR_INVALID_ARG, "the SPAI factor G of this preconditioner was destroyed");
     return SLA_SUCCESS;
 }
 
@@ -579,7 +634,7 @@ sla_status sla_pcg_solve(const sla_csr *A, const sla_precond *M, const void *d_b
         return SLA_SUCCESS;
     }
     Plan *p = nullptr;
-    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, 1, &p));
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, 1, opts ? opts->vector_f64 : 0, &p));
     return run_plan(const_cast<sla_csr *>(A), p, 1, d_b, d_x, opts, info, nullptr, nullptr,
                     (cudaStream_t)stream);
 }
@@ -596,7 +651,7 @@ sla_status sla_pcg_adjoint(const sla_csr *A, const sla_precond *M, const void *d
     if (A->n == 0)
         return SLA_SUCCESS;
     Plan *p = nullptr;
-    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, 1, &p));
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, 1, opts ? opts->vector_f64 : 0, &p));
     return run_plan(const_cast<sla_csr *>(A), p, 1, d_dLdx, d_dLdb, opts, info, d_x, d_dLdA,
                     (cudaStream_t)stream);
 }
@@ -627,7 +682,7 @@ sla_status sla_pcg_solve_batched(const sla_csr *A, const sla_precond *M, int32_t
     while (K < nrhs)
         K <<= 1;
     Plan *p = nullptr;
-    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, &p));
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, opts ? opts->vector_f64 : 0, &p));
     return run_plan(const_cast<sla_csr *>(A), p, nrhs, d_B, d_X, opts, h_info, nullptr, nullptr,
                     s);
 }
@@ -656,7 +711,7 @@ sla_status sla_pcg_adjoint_batched(const sla_csr *A, const sla_precond *M, int32
     while (K < nrhs)
         K <<= 1;
     Plan *p = nullptr;
-    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, &p));
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, opts ? opts->vector_f64 : 0, &p));
     return run_plan(const_cast<sla_csr *>(A), p, nrhs, d_dLdX, d_dLdB, opts, h_info, d_X, d_dLdA,
                     s);
 }
@@ -672,11 +727,11 @@ sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *d_lam, c
         return fail(SLA_ERR_INVALID_ARG, "NULL vector");
     if (A->nnz == 0)
         return SLA_SUCCESS;
-    return launch_pattern_grad(A, nrhs, d_lam, d_x, d_g, (cudaStream_t)stream);
+    return launch_pattern_grad(A, nrhs, 0, d_lam, d_x, d_g, (cudaStream_t)stream);
 }
 
-sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t nrhs, int32_t reps,
-                                double *h_ms, void *stream)
+sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                int32_t vector_f64, int32_t reps, double *h_ms, void *stream)
 {
     SLA_TRY(check_solve(A, M));
     if (!h_ms || reps < 1)
@@ -691,18 +746,18 @@ sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t 
     while (K < nrhs)
         K <<= 1;
     Plan *p = nullptr;
-    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, &p));
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, vector_f64, &p));
     return kernel_times(const_cast<sla_csr *>(A), p, nrhs, reps, h_ms, (cudaStream_t)stream);
 }
 
-size_t sla_workspace_bytes(const sla_csr *A, const sla_precond *M, int32_t nrhs)
+size_t sla_workspace_bytes(const sla_csr *A, const sla_precond *M, int32_t nrhs, int32_t vector_f64)
 {
     if (!A || nrhs < 1 || nrhs > KMAX)
         return 0;
     int K = 1;
     while (K < nrhs)
         K <<= 1;
-    return plan_bytes(A, M, K);
+    return plan_bytes(A, M, K, (vector_f64 && A->dtype == SLA_F32) ? 1 : 0);
 }
 
 }  // extern "C"

@@ -168,15 +168,12 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
             X[o0 + i] = x[i];
         if (Gout) {
             // dL/dA_ij = -lambda_i x_j on the system's pattern (lambda = this solve's x)
-            const int64_t k0 = rp[o0], k1 = rp[o0 + ns];
             const int lane = tid & (S - 1), grp = tid / S;
             for (int i = grp; i < ns; i += LIST_T / S) {
                 const double li = (double)x[i];
                 for (int64_t k = rp[o0 + i] + lane; k < rp[o0 + i + 1]; k += S)
                     Gout[k] = (V)(-li * (double)xf[ci[k] - o0]);
             }
-            (void)k0;
-            (void)k1;
         }
         if (tid == 0) {
             info[s].iters = it;
@@ -240,7 +237,7 @@ sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B,
     if (A->dtype == SLA_F32)
         st = list_v<float>(A, M ? (const float *)M->d_dinv : nullptr, B, X, Xf, G, tol, maxit, d_info, s);
     else
-        st = list_v<double>(A, M ? (const double *)M->d_dinv : nullptr, B, X, Xf, G, tol, maxit, d_info, s);
+        st = list_v<double>(A, M ? (const double *)M->d_dinv64 : nullptr, B, X, Xf, G, tol, maxit, d_info, s);
     if (st == SLA_SUCCESS) {
         cudaError_t e = cudaMemcpyAsync(info, d_info, sizeof(sla_pcg_info) * (size_t)A->batch,
                                         cudaMemcpyDeviceToHost, s);

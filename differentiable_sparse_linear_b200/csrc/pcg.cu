@@ -21,6 +21,9 @@
 // Each kernel's last block reduces the dot products (fp64, fixed order) and updates the
 // scalars in PcgState: alpha after Q, the stopping test after U, beta after U_J / Z.
 // When every right-hand side has stopped it clears the graph's loop condition.
+//
+// Matrix values (VM) and vectors (VV) may differ: fp32 values with fp64 vectors is the
+// mixed-precision mode.  Products and sums are always formed in fp64.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -128,10 +131,12 @@ __device__ void finalize_beta(PcgState *st, const double *rz)
 // y = A x for K right-hand sides with leading dimension ld (columns c >= nc are zero).
 template <typename V, int K>
 struct OpSpmv {
-    static constexpr int NP = 0, NS = 0;
+    using VV = V;
+    static constexpr int NP = 0, NS = 0, NV = 0;
     const V *x;
     V *y;
     int ld, nc;
+    __device__ const V *row_vec(int) const { return nullptr; }
     __device__ bool skip() const { return false; }
     __device__ void stage(double *) const {}
     __device__ __forceinline__ double operand(int64_t j, int c, const double *) const
@@ -139,8 +144,8 @@ struct OpSpmv {
         return c < nc ? (double)__ldg(&x[j * ld + c]) : 0.0;
     }
     template <int N>
-    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N],
-                                         const double *) const
+    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N], const double *,
+                                         const RowVecs<V, K, NV> &) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c)
@@ -153,33 +158,31 @@ struct OpSpmv {
 // Q: p_new = z + beta p_old, q = A p_new, partial p_new.q
 template <typename V, int K>
 struct OpQ {
-    static constexpr int NP = 1, NS = K;
+    using VV = V;
+    static constexpr int NP = 1, NS = K, NV = 2;
     const V *z;
     const V *p_old;
     V *p_new;
     V *q;
     PcgState *st;
+    __device__ const V *row_vec(int v) const { return v == 0 ? p_old : z; }
     __device__ bool skip() const { return *(volatile int *)&st->all_done; }
     __device__ void stage(double *s) const
     {
         for (int c = 0; c < K; ++c)
             s[c] = st->beta[c];
     }
-    __device__ __forceinline__ V pnew(int64_t j, int c, const double *s) const
-    {
-        return (V)__fma_rn(s[c], (double)p_old[j * K + c], (double)z[j * K + c]);
-    }
     __device__ __forceinline__ double operand(int64_t j, int c, const double *s) const
     {
-        return (double)pnew(j, c, s);
+        return (double)(V)__fma_rn(s[c], (double)p_old[j * K + c], (double)z[j * K + c]);
     }
     template <int N>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s) const
+                                         const double *s, const RowVecs<V, K, NV> &rv) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c) {
-            const V pn = pnew(i, c, s);
+            const V pn = (V)__fma_rn(s[c], (double)rv.get(0, i, c), (double)rv.get(1, i, c));
             const V qv = (V)acc[c];
             p_new[i * K + c] = pn;
             q[i * K + c] = qv;
@@ -192,14 +195,17 @@ struct OpQ {
 // U_S: r_new = r_old - alpha q, x += alpha p, y = G^T r_new, partial r_new.r_new
 template <typename V, int K>
 struct OpUS {
-    static constexpr int NP = 1, NS = 2 * K;
+    using VV = V;
+    static constexpr int NP = 1, NS = 2 * K, NV = 4;
     const V *r_old;
     const V *q;
     const V *p;
+    const V *x_in;
     V *r_new;
     V *x;
     V *y;
     PcgState *st;
+    __device__ const V *row_vec(int v) const { return v == 0 ? r_old : v == 1 ? q : v == 2 ? p : x_in; }
     __device__ bool skip() const { return *(volatile int *)&st->all_done; }
     __device__ void stage(double *s) const
     {
@@ -208,25 +214,24 @@ struct OpUS {
             s[K + c] = st->active[c] ? 1.0 : 0.0;
         }
     }
-    __device__ __forceinline__ V rnew(int64_t j, int c, const double *s) const
+    __device__ __forceinline__ V rnew(V ro, V qv, int c, const double *s) const
     {
-        const V ro = r_old[j * K + c];
-        return s[K + c] != 0.0 ? (V)__fma_rn(-s[c], (double)q[j * K + c], (double)ro) : ro;
+        return s[K + c] != 0.0 ? (V)__fma_rn(-s[c], (double)qv, (double)ro) : ro;
     }
     __device__ __forceinline__ double operand(int64_t j, int c, const double *s) const
     {
-        return (double)rnew(j, c, s);
+        return (double)rnew(r_old[j * K + c], q[j * K + c], c, s);
     }
     template <int N>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s) const
+                                         const double *s, const RowVecs<V, K, NV> &rv) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c) {
-            const V rn = rnew(i, c, s);
+            const V rn = rnew(rv.get(0, i, c), rv.get(1, i, c), c, s);
             r_new[i * K + c] = rn;
             if (s[K + c] != 0.0)
-                x[i * K + c] = (V)__fma_rn(s[c], (double)p[i * K + c], (double)x[i * K + c]);
+                x[i * K + c] = (V)__fma_rn(s[c], (double)rv.get(2, i, c), (double)rv.get(3, i, c));
             y[i * K + c] = (V)acc[c];
             part[c] += (double)rn * (double)rn;
         }
@@ -243,11 +248,13 @@ struct OpUS {
 // Z: z = G y + eps r, partial r.z
 template <typename V, int K>
 struct OpZ {
-    static constexpr int NP = 1, NS = 1;
+    using VV = V;
+    static constexpr int NP = 1, NS = 1, NV = 1;
     const V *y;
     const V *r;
     V *z;
     PcgState *st;
+    __device__ const V *row_vec(int) const { return r; }
     __device__ bool skip() const { return *(volatile int *)&st->all_done; }
     __device__ void stage(double *s) const { s[0] = st->eps; }
     __device__ __forceinline__ double operand(int64_t j, int c, const double *) const
@@ -256,14 +263,14 @@ struct OpZ {
     }
     template <int N>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s) const
+                                         const double *s, const RowVecs<V, K, NV> &rv) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c) {
-            const double rv = (double)r[i * K + c];
-            const V zv = (V)__fma_rn(s[0], rv, acc[c]);
+            const double rv_ = (double)rv.get(0, i, c);
+            const V zv = (V)__fma_rn(s[0], rv_, acc[c]);
             z[i * K + c] = zv;
-            part[c] += rv * (double)zv;
+            part[c] += rv_ * (double)zv;
         }
     }
     __device__ void finalize(const double *sums) const { finalize_beta(st, sums); }
@@ -292,6 +299,8 @@ k_update_jacobi(int64_t n, V *x, V *r, const V *p, const V *q, V *z, const V *di
     __shared__ double s_a[K];
     __shared__ double s_on[K];
     __shared__ double s_red[(VEC_T / 32) * 2 * K];
+    __shared__ double s_sum[2 * K];
+    __shared__ int s_flag;
     if (*(volatile int *)&st->all_done)
         return;
     if (threadIdx.x < K) {
@@ -323,7 +332,8 @@ k_update_jacobi(int64_t n, V *x, V *r, const V *p, const V *q, V *z, const V *di
         }
     }
     UJFinal fin{st, K};
-    grid_reduce_finalize<VEC_T, 2 * K>(part, partials, st, fin, s_red);
+    auto sync = [] { __syncthreads(); };
+    grid_reduce_finalize<VEC_T, 2 * K>(part, partials, st, fin, s_red, &s_flag, s_sum, (int)threadIdx.x, sync);
 }
 
 // Reset the state and load the right-hand sides: r = b (padded to K columns), x = p = q = 0.
@@ -365,6 +375,7 @@ __global__ void k_init(int64_t n, int nrhs, const V *B, V *x, V *r, V *p, V *q, 
         st->cond_handle = cond;
         st->has_cond = has_cond;
         st->profile = 0;
+        st->error = 0;
     }
 }
 
@@ -391,6 +402,14 @@ __global__ void k_copy_out(int64_t n, int nrhs, const V *x, V *X)
     }
 }
 
+template <typename V>
+__global__ void k_fill(int64_t n, V *a, V v)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        a[i] = v;
+}
+
 // ------------------------------------------------------------------ pattern gradient
 // g_k = -sum_c lam[row(k)*nrhs + c] * x[col(k)*nrhs + c] over the tiles of A: the tile's
 // row ends are staged in shared memory and each entry finds its row by binary search, so
@@ -398,17 +417,17 @@ __global__ void k_copy_out(int64_t n, int nrhs, const V *x, V *X)
 constexpr int GRAD_T = 256;
 constexpr int GRAD_D = 2048;
 
-template <typename V>
+template <typename VM, typename VV>
 __global__ void __launch_bounds__(GRAD_T)
-k_pattern_grad(const MatView<V> m, int nrhs, const V *lam, const V *x, V *g)
+k_pattern_grad(const MatView<VM> m, int nrhs, const VV *lam, const VV *x, VM *g)
 {
     __shared__ int32_t s_rp[GRAD_D];
     for (int t = blockIdx.x; t < m.n_tiles; t += gridDim.x) {
-        const int r0 = m.tile_row[t];
-        const int r1 = m.tile_row[t + 1];
+        const int r0 = m.desc[t].x;
+        const int r1 = m.desc[t + 1].x;
         const int nr = r1 - r0;
-        const int64_t k0 = m.rp[r0];
-        const int nk = (int)(m.rp[r1] - k0);
+        const int64_t k0 = (int64_t)(uint32_t)m.desc[t].y;
+        const int nk = (int)((int64_t)(uint32_t)m.desc[t + 1].y - k0);
         const bool longrow = nr + nk > GRAD_D;
         if (!longrow)
             for (int r = threadIdx.x; r < nr; r += GRAD_T)
@@ -432,7 +451,7 @@ k_pattern_grad(const MatView<V> m, int nrhs, const V *lam, const V *x, V *g)
             double s = 0.0;
             for (int c = 0; c < nrhs; ++c)
                 s = __fma_rn((double)lam[i * nrhs + c], (double)x[j * nrhs + c], s);
-            g[k0 + e] = (V)(-s);
+            g[k0 + e] = (VM)(-s);
         }
         __syncthreads();
     }
@@ -470,10 +489,11 @@ __global__ void k_validate(int64_t n, const int32_t *rp, const int32_t *ci, cons
     }
 }
 
-// D^-1 of A in A's value type; a missing or non-positive diagonal sets *err.
-template <typename V>
-__global__ void k_jacobi_dinv(int64_t n, const int32_t *rp, const int32_t *ci, const V *val,
-                              V *dinv, int *err)
+// D^-1 of A in fp64 and, for fp32 matrices, in fp32; a missing or non-positive diagonal
+// sets *err.
+template <typename VM>
+__global__ void k_jacobi_dinv(int64_t n, const int32_t *rp, const int32_t *ci, const VM *val,
+                              double *dinv64, float *dinv32, int *err)
 {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
@@ -481,12 +501,12 @@ __global__ void k_jacobi_dinv(int64_t n, const int32_t *rp, const int32_t *ci, c
         for (int64_t k = rp[i]; k < rp[i + 1]; ++k)
             if (ci[k] == i)
                 d = (double)val[k];
-        if (!(d > 0.0)) {
+        const double inv = d > 0.0 ? 1.0 / d : 0.0;
+        if (!(d > 0.0))
             atomicOr(err, 1);
-            dinv[i] = (V)0;
-        } else {
-            dinv[i] = (V)(1.0 / d);
-        }
+        dinv64[i] = inv;
+        if (dinv32)
+            dinv32[i] = (float)inv;
     }
 }
 
@@ -508,30 +528,48 @@ static MatView<V> view(const sla_csr *A, const TilePart *tp)
     m.rp = A->rp;
     m.ci = A->ci;
     m.val = (const V *)A->val;
-    m.tile_row = tp->d_tile_row;
+    m.desc = tp->d_desc;
     m.n_tiles = tp->n_tiles;
     m.n = A->n;
+    m.nnz = A->nnz;
     return m;
 }
 
-template <int K, typename V, class Op>
-static int tile_grid(const sla_csr *A, const TilePart *tp)
-{
-    int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_tile<K, V, Op>, TileCfg<K>::T, 0);
-    per_sm = std::max(per_sm, 1);
-    return std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
-}
+template <int K, typename VM, class Op>
+struct TileLaunch {
+    using L = StageLayout<K, VM, typename Op::VV, Op::NV>;
+    static constexpr int THREADS = TileCfg<K>::TC + 32;
+    static constexpr size_t SMEM = TileCfg<K>::NST * L::BYTES;
+
+    static sla_status setup(const sla_csr *A, const TilePart *tp, int *grid)
+    {
+        auto kern = k_tile<K, VM, Op>;
+        SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM));
+        int per_sm = 0;
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, SMEM));
+        per_sm = std::max(per_sm, 1);
+        *grid = std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
+        return SLA_SUCCESS;
+    }
+    static void launch(cudaStream_t s, int grid, const MatView<VM> &m, const Op &op, double *part,
+                       PcgState *st, int *err)
+    {
+        k_tile<K, VM, Op><<<grid, THREADS, SMEM, s>>>(m, op, part, st, err);
+    }
+};
 
 template <typename V, int K>
 static sla_status spmv_k(const sla_csr *A, int nc, const void *x, void *y, cudaStream_t s)
 {
     const TilePart *tp;
-    SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), TileCfg<K>::D, s, &tp));
-    OpSpmv<V, K> op{(const V *)x, (V *)y, nc, nc};
-    const int grid = tile_grid<K, V, OpSpmv<V, K>>(A, tp);
-    if (tp->n_tiles > 0)
-        k_tile<K, V, OpSpmv<V, K>><<<grid, TileCfg<K>::T, 0, s>>>(view<V>(A, tp), op, nullptr, nullptr);
+    SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), TileCfg<K>::D, TileCfg<K>::RMAX, s, &tp));
+    if (tp->n_tiles == 0)
+        return SLA_SUCCESS;
+    using Op = OpSpmv<V, K>;
+    Op op{(const V *)x, (V *)y, nc, nc};
+    int grid = 0;
+    SLA_TRY((TileLaunch<K, V, Op>::setup(A, tp, &grid)));
+    TileLaunch<K, V, Op>::launch(s, grid, view<V>(A, tp), op, nullptr, nullptr, A->d_err);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
 }
@@ -562,28 +600,29 @@ sla_status launch_spmv(const sla_csr *A, int K, const void *x, void *y, cudaStre
     return A->dtype == SLA_F32 ? spmv_v<float>(A, K, x, y, s) : spmv_v<double>(A, K, x, y, s);
 }
 
-template <typename V>
+template <typename VM, typename VV>
 static sla_status grad_v(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g,
                          cudaStream_t s)
 {
     const TilePart *tp;
-    SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), GRAD_D, s, &tp));
+    SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), GRAD_D, GRAD_D, s, &tp));
     if (tp->n_tiles == 0)
         return SLA_SUCCESS;
     int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_pattern_grad<V>, GRAD_T, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_pattern_grad<VM, VV>, GRAD_T, 0);
     const int grid = std::max(1, std::min(tp->n_tiles, std::max(per_sm, 1) * A->num_sms));
-    k_pattern_grad<V><<<grid, GRAD_T, 0, s>>>(view<V>(A, tp), nrhs, (const V *)lam, (const V *)x,
-                                              (V *)g);
+    k_pattern_grad<VM, VV><<<grid, GRAD_T, 0, s>>>(view<VM>(A, tp), nrhs, (const VV *)lam,
+                                                   (const VV *)x, (VM *)g);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
 }
 
-sla_status launch_pattern_grad(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g,
-                               cudaStream_t s)
+sla_status launch_pattern_grad(const sla_csr *A, int nrhs, int vec64, const void *lam, const void *x,
+                               void *g, cudaStream_t s)
 {
-    return A->dtype == SLA_F32 ? grad_v<float>(A, nrhs, lam, x, g, s)
-                               : grad_v<double>(A, nrhs, lam, x, g, s);
+    if (A->dtype == SLA_F64)
+        return grad_v<double, double>(A, nrhs, lam, x, g, s);
+    return vec64 ? grad_v<float, double>(A, nrhs, lam, x, g, s) : grad_v<float, float>(A, nrhs, lam, x, g, s);
 }
 
 sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s)
@@ -595,22 +634,21 @@ sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s)
     return SLA_SUCCESS;
 }
 
-sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv, int *d_err, cudaStream_t s)
+sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv64, void *dinv32, int *d_err, cudaStream_t s)
 {
     if (A->n == 0)
         return SLA_SUCCESS;
     if (A->dtype == SLA_F32)
         k_jacobi_dinv<float><<<vec_grid(A), 256, 0, s>>>(A->n, A->rp, A->ci, (const float *)A->val,
-                                                         (float *)dinv, d_err);
+                                                         (double *)dinv64, (float *)dinv32, d_err);
     else
         k_jacobi_dinv<double><<<vec_grid(A), 256, 0, s>>>(A->n, A->rp, A->ci, (const double *)A->val,
-                                                          (double *)dinv, d_err);
+                                                          (double *)dinv64, nullptr, d_err);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
 }
 
-sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t *perm,
-                                    cudaStream_t s)
+sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t *perm, cudaStream_t s)
 {
     if (G->nnz == 0)
         return SLA_SUCCESS;
@@ -626,14 +664,18 @@ sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t
 
 // ------------------------------------------------------------------ solve plans
 // The kernels of one PCG iteration for a plan, with their grids and operands bound.
-template <typename V, int K>
+template <typename VM, typename VV, int K>
 struct PlanKernels {
+    using LQ = TileLaunch<K, VM, OpQ<VV, K>>;
+    using LUS = TileLaunch<K, VM, OpUS<VV, K>>;
+    using LZ = TileLaunch<K, VM, OpZ<VV, K>>;
     int64_t n = 0;
-    V *x, *ra, *rb, *pa, *pb, *q, *z, *y;
-    const V *dinv = nullptr;
+    VV *x, *ra, *rb, *pa, *pb, *q, *z, *y;
+    const VV *dinv = nullptr;
     PcgState *st;
     double *part;
-    MatView<V> mA{}, mG{}, mGT{};
+    int *err;
+    MatView<VM> mA{}, mG{}, mGT{};
     int gA = 0, gG = 0, gGT = 0, gv = 0;
 
     sla_status bind(sla_csr *A, Plan *p, cudaStream_t s)
@@ -641,26 +683,27 @@ struct PlanKernels {
         const sla_precond *M = p->M;
         n = A->n;
         const TilePart *tpA;
-        SLA_TRY(ensure_tiles(A, TileCfg<K>::D, s, &tpA));
-        x = (V *)p->x; ra = (V *)p->ra; rb = (V *)p->rb; pa = (V *)p->pa; pb = (V *)p->pb;
-        q = (V *)p->q; z = (V *)p->z; y = (V *)p->y;
+        SLA_TRY(ensure_tiles(A, TileCfg<K>::D, TileCfg<K>::RMAX, s, &tpA));
+        x = (VV *)p->x; ra = (VV *)p->ra; rb = (VV *)p->rb; pa = (VV *)p->pa; pb = (VV *)p->pb;
+        q = (VV *)p->q; z = (VV *)p->z; y = (VV *)p->y;
         st = p->st;
         part = p->partials;
-        mA = view<V>(A, tpA);
-        gA = tile_grid<K, V, OpQ<V, K>>(A, tpA);
+        err = &p->st->error;
+        mA = view<VM>(A, tpA);
+        SLA_TRY(LQ::setup(A, tpA, &gA));
         gv = vec_grid(A);
         if (p->kind == 1)
-            dinv = (const V *)M->d_dinv;
+            dinv = (const VV *)(sizeof(VV) == 8 ? M->d_dinv64 : M->d_dinv);
         else if (p->kind == 0)
-            dinv = (const V *)p->y;  // ones (y is unused without SPAI)
+            dinv = (const VV *)p->y;  // ones (y is unused without SPAI)
         if (p->kind == 2) {
             const TilePart *tpG, *tpGT;
-            SLA_TRY(ensure_tiles(const_cast<sla_csr *>(M->G), TileCfg<K>::D, s, &tpG));
-            SLA_TRY(ensure_tiles(M->GT, TileCfg<K>::D, s, &tpGT));
-            mG = view<V>(M->G, tpG);
-            mGT = view<V>(M->GT, tpGT);
-            gG = tile_grid<K, V, OpZ<V, K>>(M->G, tpG);
-            gGT = tile_grid<K, V, OpUS<V, K>>(M->GT, tpGT);
+            SLA_TRY(ensure_tiles(const_cast<sla_csr *>(M->G), TileCfg<K>::D, TileCfg<K>::RMAX, s, &tpG));
+            SLA_TRY(ensure_tiles(M->GT, TileCfg<K>::D, TileCfg<K>::RMAX, s, &tpGT));
+            mG = view<VM>(M->G, tpG);
+            mGT = view<VM>(M->GT, tpGT);
+            SLA_TRY(LZ::setup(M->G, tpG, &gG));
+            SLA_TRY(LUS::setup(M->GT, tpGT, &gGT));
         }
         p->grid_tiles_A = gA;
         p->grid_tiles_G = gG;
@@ -668,34 +711,31 @@ struct PlanKernels {
         p->grid_vec = gv;
         return SLA_SUCCESS;
     }
-    void Q(cudaStream_t s, const V *pold, V *pnew) const
+    void Q(cudaStream_t s, const VV *pold, VV *pnew) const
     {
-        OpQ<V, K> op{z, pold, pnew, q, st};
-        k_tile<K, V, OpQ<V, K>><<<gA, TileCfg<K>::T, 0, s>>>(mA, op, part, st);
+        LQ::launch(s, gA, mA, OpQ<VV, K>{z, pold, pnew, q, st}, part, st, err);
     }
-    void UJ(cudaStream_t s, const V *pcur) const
+    void UJ(cudaStream_t s, const VV *pcur) const
     {
-        k_update_jacobi<V, K><<<gv, VEC_T, 0, s>>>(n, x, ra, pcur, q, z, dinv, part, st);
+        k_update_jacobi<VV, K><<<gv, VEC_T, 0, s>>>(n, x, ra, pcur, q, z, dinv, part, st);
     }
-    void US(cudaStream_t s, const V *rold, V *rnew, const V *pcur) const
+    void US(cudaStream_t s, const VV *rold, VV *rnew, const VV *pcur) const
     {
-        OpUS<V, K> op{rold, q, pcur, rnew, x, y, st};
-        k_tile<K, V, OpUS<V, K>><<<gGT, TileCfg<K>::T, 0, s>>>(mGT, op, part, st);
+        LUS::launch(s, gGT, mGT, OpUS<VV, K>{rold, q, pcur, x, rnew, x, y, st}, part, st, err);
     }
-    void Z(cudaStream_t s, const V *rcur) const
+    void Z(cudaStream_t s, const VV *rcur) const
     {
-        OpZ<V, K> op{y, rcur, z, st};
-        k_tile<K, V, OpZ<V, K>><<<gG, TileCfg<K>::T, 0, s>>>(mG, op, part, st);
+        LZ::launch(s, gG, mG, OpZ<VV, K>{y, rcur, z, st}, part, st, err);
     }
 };
 
-template <typename V, int K>
+template <typename VM, typename VV, int K>
 static sla_status capture_k(sla_csr *A, Plan *p)
 {
-    PlanKernels<V, K> kr;
+    PlanKernels<VM, VV, K> kr;
     SLA_TRY(kr.bind(A, p, p->cs));
     SLA_CUDA_TRY(cudaStreamSynchronize(p->cs));
-    V *ra = kr.ra, *rb = kr.rb, *pa = kr.pa, *pb = kr.pb;
+    VV *ra = kr.ra, *rb = kr.rb, *pa = kr.pa, *pb = kr.pb;
 
     cudaGraph_t g = nullptr;
     SLA_CUDA_TRY(cudaGraphCreate(&g, 0));
@@ -759,10 +799,10 @@ static sla_status capture_k(sla_csr *A, Plan *p)
 
 // Mean device time of each kernel of one iteration, each launch bracketed by events in
 // the order the loop runs them (so each sees the cache state of the real iteration).
-template <typename V, int K>
+template <typename VM, typename VV, int K>
 static sla_status times_k(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s)
 {
-    PlanKernels<V, K> kr;
+    PlanKernels<VM, VV, K> kr;
     SLA_TRY(kr.bind(A, p, s));
     k_profile_mode<<<1, 1, 0, s>>>(p->st, nrhs);
     SLA_CUDA_TRY(cudaGetLastError());
@@ -803,102 +843,91 @@ static sla_status times_k(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms,
     return st;
 }
 
-template <typename V>
-static sla_status capture_v(sla_csr *A, Plan *p)
-{
-    switch (p->K) {
-    case 1: return capture_k<V, 1>(A, p);
-    case 2: return capture_k<V, 2>(A, p);
-    case 4: return capture_k<V, 4>(A, p);
-    case 8: return capture_k<V, 8>(A, p);
-    case 16: return capture_k<V, 16>(A, p);
-    default: return fail(SLA_ERR_INVALID_ARG, "unsupported right-hand-side count");
-    }
-}
-
-sla_status capture_plan_graph(sla_csr *A, Plan *p)
-{
-    return A->dtype == SLA_F32 ? capture_v<float>(A, p) : capture_v<double>(A, p);
-}
-
-template <typename V>
-static sla_status times_v(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s)
-{
-    switch (p->K) {
-    case 1: return times_k<V, 1>(A, p, nrhs, reps, h_ms, s);
-    case 2: return times_k<V, 2>(A, p, nrhs, reps, h_ms, s);
-    case 4: return times_k<V, 4>(A, p, nrhs, reps, h_ms, s);
-    case 8: return times_k<V, 8>(A, p, nrhs, reps, h_ms, s);
-    case 16: return times_k<V, 16>(A, p, nrhs, reps, h_ms, s);
-    default: return fail(SLA_ERR_INVALID_ARG, "unsupported right-hand-side count");
-    }
-}
-
-sla_status kernel_times(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s)
-{
-    return A->dtype == SLA_F32 ? times_v<float>(A, p, nrhs, reps, h_ms, s)
-                               : times_v<double>(A, p, nrhs, reps, h_ms, s);
-}
-
-template <typename V>
-__global__ void k_fill(int64_t n, V *a, V v)
-{
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
-        a[i] = v;
-}
-
-template <typename V, int K>
-static sla_status run_k(sla_csr *A, Plan *p, int nrhs, const void *B, void *X,
-                        double tol, long long maxit, cudaStream_t s)
+template <typename VM, typename VV, int K>
+static sla_status run_k(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,
+                        long long maxit, cudaStream_t s)
 {
     const int64_t n = A->n;
     const int gv = vec_grid(A);
-    V *y = (V *)p->y;
+    VV *y = (VV *)p->y;
     if (p->kind == 0) {
         // without a preconditioner the Jacobi kernel runs with D^-1 = 1 (held in y)
-        k_fill<V><<<gv, 256, 0, s>>>(n, y, (V)1);
+        k_fill<VV><<<gv, 256, 0, s>>>(n, y, (VV)1);
         y = nullptr;
     }
-    k_init<V, K><<<gv, 256, 0, s>>>(n, nrhs, (const V *)B, (V *)p->x, (V *)p->ra, (V *)p->pa,
-                                    (V *)p->q, (V *)p->z, p->kind == 2 ? y : nullptr, p->st, tol,
-                                    maxit, p->M ? p->M->eps : 0.0, p->cond, 1);
+    k_init<VV, K><<<gv, 256, 0, s>>>(n, nrhs, (const VV *)B, (VV *)p->x, (VV *)p->ra, (VV *)p->pa,
+                                     (VV *)p->q, (VV *)p->z, p->kind == 2 ? y : nullptr, p->st, tol,
+                                     maxit, p->M ? p->M->eps : 0.0, p->cond, 1);
     SLA_CUDA_TRY(cudaGetLastError());
     SLA_CUDA_TRY(cudaGraphLaunch(p->exec, s));
-    k_copy_out<V, K><<<gv, 256, 0, s>>>(n, nrhs, (const V *)p->x, (V *)X);
+    k_copy_out<VV, K><<<gv, 256, 0, s>>>(n, nrhs, (const VV *)p->x, (VV *)X);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
 }
 
-template <typename V>
-static sla_status run_v(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,
-                        long long maxit, cudaStream_t s)
-{
-    switch (p->K) {
-    case 1: return run_k<V, 1>(A, p, nrhs, B, X, tol, maxit, s);
-    case 2: return run_k<V, 2>(A, p, nrhs, B, X, tol, maxit, s);
-    case 4: return run_k<V, 4>(A, p, nrhs, B, X, tol, maxit, s);
-    case 8: return run_k<V, 8>(A, p, nrhs, B, X, tol, maxit, s);
-    case 16: return run_k<V, 16>(A, p, nrhs, B, X, tol, maxit, s);
-    default: return fail(SLA_ERR_INVALID_ARG, "unsupported right-hand-side count");
+// ------------------------------------------------------------------ dispatch
+#define SLA_DISPATCH_K(K_, FN, ...)                                                    \
+    switch (K_) {                                                                      \
+    case 1: return FN<VM, VV, 1>(__VA_ARGS__);                                         \
+    case 2: return FN<VM, VV, 2>(__VA_ARGS__);                                         \
+    case 4: return FN<VM, VV, 4>(__VA_ARGS__);                                         \
+    case 8: return FN<VM, VV, 8>(__VA_ARGS__);                                         \
+    case 16: return FN<VM, VV, 16>(__VA_ARGS__);                                       \
+    default: return fail(SLA_ERR_INVALID_ARG, "unsupported right-hand-side count");    \
     }
+
+template <typename VM, typename VV>
+static sla_status capture_mv(sla_csr *A, Plan *p) { SLA_DISPATCH_K(p->K, capture_k, A, p) }
+template <typename VM, typename VV>
+static sla_status times_mv(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s)
+{
+    SLA_DISPATCH_K(p->K, times_k, A, p, nrhs, reps, h_ms, s)
+}
+template <typename VM, typename VV>
+static sla_status run_mv(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,
+                         long long maxit, cudaStream_t s)
+{
+    SLA_DISPATCH_K(p->K, run_k, A, p, nrhs, B, X, tol, maxit, s)
+}
+
+sla_status capture_plan_graph(sla_csr *A, Plan *p)
+{
+    if (A->dtype == SLA_F64)
+        return capture_mv<double, double>(A, p);
+    return p->vec64 ? capture_mv<float, double>(A, p) : capture_mv<float, float>(A, p);
+}
+
+sla_status kernel_times(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s)
+{
+    if (A->dtype == SLA_F64)
+        return times_mv<double, double>(A, p, nrhs, reps, h_ms, s);
+    return p->vec64 ? times_mv<float, double>(A, p, nrhs, reps, h_ms, s)
+                    : times_mv<float, float>(A, p, nrhs, reps, h_ms, s);
 }
 
 sla_status run_plan(sla_csr *A, Plan *p, int nrhs, const void *B, void *X,
                     const sla_pcg_opts *opts, sla_pcg_info *info, const void *grad_x,
                     void *grad_out, cudaStream_t s)
 {
-    double tol = (opts && opts->rtol > 0) ? opts->rtol : (A->dtype == SLA_F32 ? 1e-6 : 1e-10);
+    const bool f64 = A->dtype == SLA_F64 || p->vec64;
+    double tol = (opts && opts->rtol > 0) ? opts->rtol : (f64 ? 1e-10 : 1e-6);
     long long n_sys = A->batch > 1 ? A->max_sys_n : A->n;
     long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 10 * std::max<long long>(n_sys, 1);
-    sla_status st = A->dtype == SLA_F32 ? run_v<float>(A, p, nrhs, B, X, tol, maxit, s)
-                                        : run_v<double>(A, p, nrhs, B, X, tol, maxit, s);
+    sla_status st;
+    if (A->dtype == SLA_F64)
+        st = run_mv<double, double>(A, p, nrhs, B, X, tol, maxit, s);
+    else if (p->vec64)
+        st = run_mv<float, double>(A, p, nrhs, B, X, tol, maxit, s);
+    else
+        st = run_mv<float, float>(A, p, nrhs, B, X, tol, maxit, s);
     if (st != SLA_SUCCESS)
         return st;
     if (grad_out)
-        SLA_TRY(launch_pattern_grad(A, nrhs, X, grad_x, grad_out, s));
+        SLA_TRY(launch_pattern_grad(A, nrhs, p->vec64, X, grad_x, grad_out, s));
     SLA_CUDA_TRY(cudaMemcpyAsync(p->h_st, p->st, sizeof(PcgState), cudaMemcpyDeviceToHost, s));
     SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    if (p->h_st->error)
+        return fail(SLA_ERR_CUDA, "a pipeline wait inside a solver kernel ran out of time; results are invalid");
     sla_status worst = SLA_SUCCESS;
     for (int c = 0; c < nrhs; ++c) {
         if (info) {

@@ -55,16 +55,20 @@ struct PcgState {
     unsigned long long cond_handle;   // cudaGraphConditionalHandle of the solve loop
     int has_cond;
     int profile;            // 1: kernels run for timing only; finalisation is skipped
+    int error;              // nonzero: a pipeline wait ran out of time (results invalid)
+    int vec64;              // vectors are fp64 (matrix may be fp32)
 };
 
 // ------------------------------------------------------------------ tiles
-// Row partition for the load-balanced SpMV: tile t holds rows [tile_row[t], tile_row[t+1]).
-// A tile holds at most D "items" (rows + stored entries) unless it is one single row
-// longer than that (a "long row" tile, reduced by the whole block).
+// Row partition for the load-balanced SpMV: tile t holds rows [desc[t].x, desc[t+1].x) and
+// entries [desc[t].y, desc[t+1].y).  A tile holds at most D "items" (rows + stored entries)
+// and at most RMAX rows, unless it is one single row with D or more entries (a "long row"
+// tile, streamed in chunks and reduced by the whole block).
 struct TilePart {
     int D = 0;
+    int RMAX = 0;
     int n_tiles = 0;
-    int32_t *d_tile_row = nullptr;
+    int2 *d_desc = nullptr;
 };
 
 // Read-only view of a CSR matrix passed to kernels.
@@ -73,9 +77,10 @@ struct MatView {
     const int32_t *rp;
     const int32_t *ci;
     const V *val;
-    const int32_t *tile_row;
+    const int2 *desc;
     int n_tiles;
     int64_t n;
+    int64_t nnz;
 };
 
 struct Plan;
@@ -106,6 +111,10 @@ struct sla_csr {
     int num_sms = 148;
     std::vector<sla::Plan *> plans;
     int64_t max_row_len = 0;
+    int *d_err = nullptr;                  // pipeline error word of kernels without a plan
+    // preconditioners built on this handle (as A or as G); they are detached when it is
+    // destroyed, whatever the order the caller destroys handles in
+    std::vector<sla_precond *> dependents;
 };
 
 struct sla_precond {
@@ -114,7 +123,8 @@ struct sla_precond {
     const sla_csr *G = nullptr;            // borrowed (SPAI)
     sla_csr *GT = nullptr;                 // owned explicit transpose (SPAI)
     double eps = 0.0;
-    void *d_dinv = nullptr;                // Jacobi: 1 / A_ii in A's dtype
+    void *d_dinv = nullptr;                // Jacobi: 1 / A_ii in fp32 (fp32 matrices only)
+    void *d_dinv64 = nullptr;              // Jacobi: 1 / A_ii in fp64
     int32_t *d_perm = nullptr;             // SPAI: position in G of each G^T entry
 };
 
@@ -124,6 +134,7 @@ namespace sla {
 struct Plan {
     const sla_precond *M = nullptr;
     int K = 1;
+    int vec64 = 0;                         // fp64 vectors with an fp32 matrix
     int kind = 0;                          // 0 none, 1 Jacobi, 2 SPAI
     void *ws = nullptr;                    // one device allocation
     size_t ws_bytes = 0;
@@ -140,17 +151,17 @@ struct Plan {
 };
 
 // ------------------------------------------------------------------ internal entry points
-sla_status ensure_tiles(sla_csr *A, int D, cudaStream_t s, const TilePart **out);
-size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K);
-sla_status get_plan(sla_csr *A, const sla_precond *M, int K, Plan **out);
+sla_status ensure_tiles(sla_csr *A, int D, int RMAX, cudaStream_t s, const TilePart **out);
+size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K, int vec64);
+sla_status get_plan(sla_csr *A, const sla_precond *M, int K, int vec64, Plan **out);
 void destroy_plan(Plan *p);
 
 // launchers implemented in the .cu files
 sla_status launch_spmv(const sla_csr *A, int K, const void *x, void *y, cudaStream_t s);
-sla_status launch_pattern_grad(const sla_csr *A, int K, const void *lam, const void *x, void *g,
-                               cudaStream_t s);
+sla_status launch_pattern_grad(const sla_csr *A, int K, int vec64, const void *lam, const void *x,
+                               void *g, cudaStream_t s);
 sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s);
-sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv, int *d_err, cudaStream_t s);
+sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv64, void *dinv32, int *d_err, cudaStream_t s);
 sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t *d_perm,
                                     cudaStream_t s);
 sla_status capture_plan_graph(sla_csr *A, Plan *p);

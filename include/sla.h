@@ -82,8 +82,11 @@ typedef struct {
     double rtol;        /* stop when ||r_k||_2 / ||b||_2 <= rtol on the recursive residual;
                            0 -> 1e-10 for fp64, 1e-6 for fp32                              */
     int64_t maxit;      /* iteration cap per right-hand side; 0 -> 10 * n (n of the system) */
-    int32_t reserved0;
-    int32_t reserved1;
+    int32_t vector_f64; /* nonzero with an fp32 matrix: mixed precision -- b, x, the adjoint's
+                           dL/dx and dL/db and all solver vectors are fp64 (dL/dA stays fp32);
+                           the default tolerance is then 1e-10.  Ignored for fp64 matrices
+                           and for list handles. */
+    int32_t reserved;
 } sla_pcg_opts;
 
 /* Per right-hand side (or per system of a list) solver outcome. */
@@ -192,18 +195,19 @@ SLA_API sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *
                             void *d_g, void *stream);
 
 /* Per-kernel device time of one PCG iteration (metrics).  On the workspace of the
- * (A, M, nrhs) solver -- normally right after a solve, so it holds that solve's vectors --
+ * (A, M, nrhs, vector_f64) solver -- normally right after a solve, so it holds that solve's vectors --
  * launches the iteration's kernels `reps` times in loop order, each bracketed by CUDA
  * events on `stream`, with the scalar updates switched off, and writes the mean ms per
  * launch to h_ms[0..2]: [0] p-update + q = A p, [1] the x/r update (Jacobi: with z = D^-1 r;
  * SPAI: with y = G^T r), [2] z = G y + eps r (SPAI; 0 otherwise).  The workspace contents
  * are unspecified afterwards (the next solve re-initialises them).  Synchronises `stream`. */
 SLA_API sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t nrhs,
-                                        int32_t reps, double *h_ms, void *stream);
+                                        int32_t vector_f64, int32_t reps, double *h_ms, void *stream);
 
-/* Device bytes the solver workspace takes for (A, M, nrhs); it depends on n and nnz only,
+/* Device bytes the solver workspace takes for (A, M, nrhs, vector_f64); it depends on n and nnz only,
  * never on the iteration count ([TS] Complexity). */
-SLA_API size_t sla_workspace_bytes(const sla_csr *A, const sla_precond *M, int32_t nrhs);
+SLA_API size_t sla_workspace_bytes(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                   int32_t vector_f64);
 
 #ifdef __cplusplus
 }

@@ -18,6 +18,7 @@ def tol_key(dtype):
 
 
 def dev(a, dtype=None):
+    """Host array -> CUDA tensor (optionally cast first)."""
     t = torch.from_numpy(np.ascontiguousarray(a if dtype is None else a.astype(dtype)))
     return t.cuda()
 
