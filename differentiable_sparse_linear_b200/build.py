@@ -12,6 +12,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -44,7 +45,7 @@ def build(verbose: bool = False, force: bool = False, extra: tuple[str, ...] = (
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_t = max(_newest_header(), os.path.getmtime(__file__))
     objs = []
-    rebuilt = False
+    jobs = []
     for src in srcs:
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
@@ -54,8 +55,16 @@ def build(verbose: bool = False, force: bool = False, extra: tuple[str, ...] = (
         if verbose:
             cmd += ["-Xptxas", "-v"]
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
-        rebuilt = True
+        jobs.append(cmd)
+    for stale in glob.glob(os.path.join(BUILD, "*.o")):
+        if stale not in objs:
+            os.remove(stale)
+    with ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
+        for r in list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), jobs)):
+            sys.stderr.write(r.stderr)
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args, r.stdout, r.stderr)
+    rebuilt = bool(jobs)
     if rebuilt or force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
         tmp = LIB + f".tmp{os.getpid()}"
         cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]

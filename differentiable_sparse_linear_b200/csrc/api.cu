@@ -302,6 +302,9 @@ sla_status sla_csr_create(sla_csr **out, int64_t n_rows, int64_t n_cols, int64_t
         return fail(SLA_ERR_INVALID_ARG, "dtype must be SLA_F32 or SLA_F64");
     if (!d_row_ptr || (nnz > 0 && (!d_col || !d_val)))
         return fail(SLA_ERR_INVALID_ARG, "NULL row_ptr, col or val");
+    // the SpMV pipeline streams these arrays with 16-byte-aligned bulk copies
+    if (((uintptr_t)d_row_ptr & 15) || ((uintptr_t)d_col & 15) || ((uintptr_t)d_val & 15))
+        return fail(SLA_ERR_INVALID_ARG, "row_ptr, col and val must be 16-byte aligned device pointers");
     cudaStream_t s = (cudaStream_t)stream;
     sla_csr *A = new sla_csr();
     A->n = n_rows;

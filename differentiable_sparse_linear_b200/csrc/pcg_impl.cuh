@@ -1,29 +1,8 @@
-// PCG forward/adjoint on one B200: fused SpMV + vector-update kernels, device-side
-// convergence, and the whole loop as one CUDA graph with a conditional WHILE node.
-//
-// Method ("torch-sla: Differentiable Sparse Linear Algebra with Adjoint Solvers and Sparse
-// Tensor Parallelism for PyTorch", Methodology §1 native Jacobi-preconditioned CG and §2
-// adjoint; "Learning Sparse Approximate Inverse Preconditioners for Conjugate Gradient
-// Solvers on GPUs", Approach: M^-1 = G G^T + eps I):
-//
-//   r = b, z = M^-1 r, p = z, rho = r.z
-//   loop: q = A p; alpha = rho/(p.q); x += alpha p; r -= alpha q; stop if ||r||/||b|| <= tol
-//         z = M^-1 r; rho' = r.z; beta = rho'/rho; p = z + beta p; rho = rho'
-//
-// Kernel schedule of one iteration (each kernel streams one CSR matrix at most):
-//   Q   : p_new = z + beta p_old (own rows) and q = A p_new, p_new.q      [A]
-//         (the gathered operand z_j + beta p_old_j is formed on the fly, so p is never
-//          written and re-read in a separate pass; p is double-buffered)
-//   Jacobi  U_J : x += alpha p; r -= alpha q; z = D^-1 r; r.r and r.z    [elementwise]
-//   SPAI    U_S : r_new = r_old - alpha q (own rows and gathered), x += alpha p,
-//                 y = G^T r_new, r_new.r_new                             [G^T]
-//           Z   : z = G y + eps r_new, r_new.z                           [G]
-// Each kernel's last block reduces the dot products (fp64, fixed order) and updates the
-// scalars in PcgState: alpha after Q, the stopping test after U, beta after U_J / Z.
-// When every right-hand side has stopped it clears the graph's loop condition.
-//
-// Matrix values (VM) and vectors (VV) may differ: fp32 values with fp64 vectors is the
-// mixed-precision mode.  Products and sums are always formed in fp64.
+// Templates of the PCG solver kernels, shared by the per-precision translation units
+// (pcg_ff.cu: fp32 values and vectors; pcg_dd.cu: fp64; pcg_fd.cu: fp32 values, fp64
+// vectors).  See pcg_dispatch.cu for the method and the kernel schedule.
+#pragma once
+
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -31,14 +10,15 @@
 #include <cstring>
 
 #include "sla_internal.cuh"
+#include "row_engine.cuh"
 #include "tile_engine.cuh"
 
 namespace sla {
 
 // ------------------------------------------------------------------ scalar finalisation
-__device__ __forceinline__ bool finite_d(double a) { return isfinite(a); }
+static __device__ __forceinline__ bool finite_d(double a) { return isfinite(a); }
 
-__device__ void signal_if_done(PcgState *st)
+static __device__ __noinline__ void signal_if_done(PcgState *st)
 {
     int any = 0;
     for (int c = 0; c < st->k; ++c)
@@ -51,7 +31,7 @@ __device__ void signal_if_done(PcgState *st)
 }
 
 // After q = A p: alpha = rho / (p.q); p.q <= 0 or non-finite is a breakdown.
-__device__ void finalize_alpha(PcgState *st, const double *pq)
+static __device__ __noinline__ void finalize_alpha(PcgState *st, const double *pq)
 {
     if (st->profile)
         return;
@@ -70,7 +50,7 @@ __device__ void finalize_alpha(PcgState *st, const double *pq)
 }
 
 // After the x/r update: stopping test on ||r||/||b|| (initial pass: record ||b||).
-__device__ void finalize_residual(PcgState *st, const double *rr)
+static __device__ __noinline__ void finalize_residual(PcgState *st, const double *rr)
 {
     if (st->profile)
         return;
@@ -107,7 +87,7 @@ __device__ void finalize_residual(PcgState *st, const double *rr)
 }
 
 // After z = M^-1 r: rho' = r.z, beta = rho'/rho (0 on the initial pass).
-__device__ void finalize_beta(PcgState *st, const double *rz)
+static __device__ __noinline__ void finalize_beta(PcgState *st, const double *rz)
 {
     if (st->profile)
         return;
@@ -139,13 +119,13 @@ struct OpSpmv {
     __device__ const V *row_vec(int) const { return nullptr; }
     __device__ bool skip() const { return false; }
     __device__ void stage(double *) const {}
-    __device__ __forceinline__ double operand(int64_t j, int c, const double *) const
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
     {
-        return c < nc ? (double)__ldg(&x[j * ld + c]) : 0.0;
+        return c < nc ? __ldg(&x[j * ld + c]) : (V)0;
     }
-    template <int N>
+    template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N], const double *,
-                                         const RowVecs<V, K, NV> &) const
+                                         const RV &) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c)
@@ -172,13 +152,13 @@ struct OpQ {
         for (int c = 0; c < K; ++c)
             s[c] = st->beta[c];
     }
-    __device__ __forceinline__ double operand(int64_t j, int c, const double *s) const
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
     {
-        return (double)(V)__fma_rn(s[c], (double)p_old[j * K + c], (double)z[j * K + c]);
+        return (V)__fma_rn(s[c], (double)p_old[j * K + c], (double)z[j * K + c]);
     }
-    template <int N>
+    template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s, const RowVecs<V, K, NV> &rv) const
+                                         const double *s, const RV &rv) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c) {
@@ -218,13 +198,13 @@ struct OpUS {
     {
         return s[K + c] != 0.0 ? (V)__fma_rn(-s[c], (double)qv, (double)ro) : ro;
     }
-    __device__ __forceinline__ double operand(int64_t j, int c, const double *s) const
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
     {
-        return (double)rnew(r_old[j * K + c], q[j * K + c], c, s);
+        return rnew(r_old[j * K + c], q[j * K + c], c, s);
     }
-    template <int N>
+    template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s, const RowVecs<V, K, NV> &rv) const
+                                         const double *s, const RV &rv) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c) {
@@ -257,13 +237,13 @@ struct OpZ {
     __device__ const V *row_vec(int) const { return r; }
     __device__ bool skip() const { return *(volatile int *)&st->all_done; }
     __device__ void stage(double *s) const { s[0] = st->eps; }
-    __device__ __forceinline__ double operand(int64_t j, int c, const double *) const
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
     {
-        return (double)y[j * K + c];
+        return y[j * K + c];
     }
-    template <int N>
+    template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s, const RowVecs<V, K, NV> &rv) const
+                                         const double *s, const RV &rv) const
     {
 #pragma unroll
         for (int c = 0; c < K; ++c) {
@@ -381,7 +361,7 @@ __global__ void k_init(int64_t n, int nrhs, const V *B, V *x, V *r, V *p, V *q, 
 
 // Timing mode: every RHS active, finalisation off, so each kernel can be launched alone
 // any number of times on the workspace the last solve left.
-__global__ void k_profile_mode(PcgState *st, int nrhs)
+static __global__ void k_profile_mode(PcgState *st, int nrhs)
 {
     for (int c = 0; c < KMAX; ++c)
         st->active[c] = c < nrhs ? 1 : 0;
@@ -458,37 +438,6 @@ k_pattern_grad(const MatView<VM> m, int nrhs, const VV *lam, const VV *x, VM *g)
 }
 
 // ------------------------------------------------------------------ set-up kernels
-// Pattern check of every row: columns inside [lo, hi) of the row's system, strictly ascending.
-__global__ void k_validate(int64_t n, const int32_t *rp, const int32_t *ci, const int64_t *sys_off,
-                           int batch, int *err)
-{
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-        int64_t lo = 0, hi = n;
-        if (sys_off) {
-            int a = 0, b = batch - 1;
-            while (a < b) {  // last system whose start <= i
-                const int mid = (a + b + 1) >> 1;
-                if (sys_off[mid] <= i)
-                    a = mid;
-                else
-                    b = mid - 1;
-            }
-            lo = sys_off[a];
-            hi = sys_off[a + 1];
-        }
-        int prev = -1;
-        for (int64_t k = rp[i]; k < rp[i + 1]; ++k) {
-            const int j = ci[k];
-            if (j < lo || j >= hi || j <= prev) {
-                atomicOr(err, 1);
-                break;
-            }
-            prev = j;
-        }
-    }
-}
-
 // D^-1 of A in fp64 and, for fp32 matrices, in fp32; a missing or non-positive diagonal
 // sets *err.
 template <typename VM>
@@ -535,69 +484,88 @@ static MatView<V> view(const sla_csr *A, const TilePart *tp)
     return m;
 }
 
+// Launch configuration of one fused SpMV operation: the short-row engine when every row
+// holds at most 16 entries, the load-balanced tile engine otherwise.
+constexpr int ROWS_MAXL = 16;
+
 template <int K, typename VM, class Op>
 struct TileLaunch {
     using L = StageLayout<K, VM, typename Op::VV, Op::NV>;
     static constexpr int THREADS = TileCfg<K>::TC + 32;
     static constexpr size_t SMEM = TileCfg<K>::NST * L::BYTES;
+    int grid = 0;
+    int maxl = 0;                 // 0: tile engine; else the short-row engine's MAXL
+    MatView<VM> m{};
 
-    static sla_status setup(const sla_csr *A, const TilePart *tp, int *grid)
+    template <int MAXL>
+    sla_status setup_rows(const sla_csr *A)
     {
+        auto kern = k_rows<K, VM, MAXL, Op>;
+        int per_sm = 0;
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ROW_T, 0));
+        per_sm = std::max(per_sm, 1);
+        const int64_t need = (A->n + ROW_T - 1) / ROW_T;
+        grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)per_sm * A->num_sms));
+        maxl = MAXL;
+        return SLA_SUCCESS;
+    }
+
+    sla_status setup(const sla_csr *A, cudaStream_t s)
+    {
+        if (A->max_row_len <= ROWS_MAXL) {
+            // the row engine needs no tiles; the view carries the matrix arrays only
+            m.rp = A->rp;
+            m.ci = A->ci;
+            m.val = (const VM *)A->val;
+            m.desc = nullptr;
+            m.n_tiles = 0;
+            m.n = A->n;
+            m.nnz = A->nnz;
+            if (A->max_row_len <= 4)
+                return setup_rows<4>(A);
+            if (A->max_row_len <= 6)
+                return setup_rows<6>(A);
+            if (A->max_row_len <= 8)
+                return setup_rows<8>(A);
+            return setup_rows<16>(A);
+        }
+        const TilePart *tp;
+        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), TileCfg<K>::D, TileCfg<K>::RMAX, s, &tp));
+        m = view<VM>(A, tp);
         auto kern = k_tile<K, VM, Op>;
         SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM));
         int per_sm = 0;
         SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, SMEM));
         per_sm = std::max(per_sm, 1);
-        *grid = std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
+        grid = std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
+        maxl = 0;
         return SLA_SUCCESS;
     }
-    static void launch(cudaStream_t s, int grid, const MatView<VM> &m, const Op &op, double *part,
-                       PcgState *st, int *err)
+    bool empty() const { return maxl == 0 ? m.n_tiles == 0 : m.n == 0; }
+    void launch(cudaStream_t s, const Op &op, double *part, PcgState *st, int *err) const
     {
-        k_tile<K, VM, Op><<<grid, THREADS, SMEM, s>>>(m, op, part, st, err);
+        if (empty())
+            return;
+        switch (maxl) {
+        case 4: k_rows<K, VM, 4, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
+        case 6: k_rows<K, VM, 6, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
+        case 8: k_rows<K, VM, 8, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
+        case 16: k_rows<K, VM, 16, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
+        default: k_tile<K, VM, Op><<<grid, THREADS, SMEM, s>>>(m, op, part, st, err); break;
+        }
     }
 };
 
 template <typename V, int K>
 static sla_status spmv_k(const sla_csr *A, int nc, const void *x, void *y, cudaStream_t s)
 {
-    const TilePart *tp;
-    SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), TileCfg<K>::D, TileCfg<K>::RMAX, s, &tp));
-    if (tp->n_tiles == 0)
-        return SLA_SUCCESS;
     using Op = OpSpmv<V, K>;
     Op op{(const V *)x, (V *)y, nc, nc};
-    int grid = 0;
-    SLA_TRY((TileLaunch<K, V, Op>::setup(A, tp, &grid)));
-    TileLaunch<K, V, Op>::launch(s, grid, view<V>(A, tp), op, nullptr, nullptr, A->d_err);
+    TileLaunch<K, V, Op> L;
+    SLA_TRY(L.setup(A, s));
+    L.launch(s, op, nullptr, nullptr, A->d_err);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
-}
-
-static int pad_k(int nrhs)
-{
-    int K = 1;
-    while (K < nrhs)
-        K <<= 1;
-    return K;
-}
-
-template <typename V>
-static sla_status spmv_v(const sla_csr *A, int nrhs, const void *x, void *y, cudaStream_t s)
-{
-    switch (pad_k(nrhs)) {
-    case 1: return spmv_k<V, 1>(A, nrhs, x, y, s);
-    case 2: return spmv_k<V, 2>(A, nrhs, x, y, s);
-    case 4: return spmv_k<V, 4>(A, nrhs, x, y, s);
-    case 8: return spmv_k<V, 8>(A, nrhs, x, y, s);
-    case 16: return spmv_k<V, 16>(A, nrhs, x, y, s);
-    default: return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
-    }
-}
-
-sla_status launch_spmv(const sla_csr *A, int K, const void *x, void *y, cudaStream_t s)
-{
-    return A->dtype == SLA_F32 ? spmv_v<float>(A, K, x, y, s) : spmv_v<double>(A, K, x, y, s);
 }
 
 template <typename VM, typename VV>
@@ -617,103 +585,50 @@ static sla_status grad_v(const sla_csr *A, int nrhs, const void *lam, const void
     return SLA_SUCCESS;
 }
 
-sla_status launch_pattern_grad(const sla_csr *A, int nrhs, int vec64, const void *lam, const void *x,
-                               void *g, cudaStream_t s)
-{
-    if (A->dtype == SLA_F64)
-        return grad_v<double, double>(A, nrhs, lam, x, g, s);
-    return vec64 ? grad_v<float, double>(A, nrhs, lam, x, g, s) : grad_v<float, float>(A, nrhs, lam, x, g, s);
-}
-
-sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s)
-{
-    if (A->n == 0)
-        return SLA_SUCCESS;
-    k_validate<<<vec_grid(A), 256, 0, s>>>(A->n, A->rp, A->ci, A->d_sys_off, A->batch, d_err);
-    SLA_CUDA_TRY(cudaGetLastError());
-    return SLA_SUCCESS;
-}
-
-sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv64, void *dinv32, int *d_err, cudaStream_t s)
-{
-    if (A->n == 0)
-        return SLA_SUCCESS;
-    if (A->dtype == SLA_F32)
-        k_jacobi_dinv<float><<<vec_grid(A), 256, 0, s>>>(A->n, A->rp, A->ci, (const float *)A->val,
-                                                         (double *)dinv64, (float *)dinv32, d_err);
-    else
-        k_jacobi_dinv<double><<<vec_grid(A), 256, 0, s>>>(A->n, A->rp, A->ci, (const double *)A->val,
-                                                          (double *)dinv64, nullptr, d_err);
-    SLA_CUDA_TRY(cudaGetLastError());
-    return SLA_SUCCESS;
-}
-
-sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t *perm, cudaStream_t s)
-{
-    if (G->nnz == 0)
-        return SLA_SUCCESS;
-    if (G->dtype == SLA_F32)
-        k_gather_values<float><<<vec_grid(G), 256, 0, s>>>(G->nnz, perm, (const float *)G->val,
-                                                           (float *)GT->own_val);
-    else
-        k_gather_values<double><<<vec_grid(G), 256, 0, s>>>(G->nnz, perm, (const double *)G->val,
-                                                            (double *)GT->own_val);
-    SLA_CUDA_TRY(cudaGetLastError());
-    return SLA_SUCCESS;
-}
 
 // ------------------------------------------------------------------ solve plans
 // The kernels of one PCG iteration for a plan, with their grids and operands bound.
 template <typename VM, typename VV, int K>
 struct PlanKernels {
-    using LQ = TileLaunch<K, VM, OpQ<VV, K>>;
-    using LUS = TileLaunch<K, VM, OpUS<VV, K>>;
-    using LZ = TileLaunch<K, VM, OpZ<VV, K>>;
+    TileLaunch<K, VM, OpQ<VV, K>> LQ;
+    TileLaunch<K, VM, OpUS<VV, K>> LUS;
+    TileLaunch<K, VM, OpZ<VV, K>> LZ;
     int64_t n = 0;
     VV *x, *ra, *rb, *pa, *pb, *q, *z, *y;
     const VV *dinv = nullptr;
     PcgState *st;
     double *part;
     int *err;
-    MatView<VM> mA{}, mG{}, mGT{};
-    int gA = 0, gG = 0, gGT = 0, gv = 0;
+    int gv = 0;
 
     sla_status bind(sla_csr *A, Plan *p, cudaStream_t s)
     {
         const sla_precond *M = p->M;
         n = A->n;
-        const TilePart *tpA;
-        SLA_TRY(ensure_tiles(A, TileCfg<K>::D, TileCfg<K>::RMAX, s, &tpA));
         x = (VV *)p->x; ra = (VV *)p->ra; rb = (VV *)p->rb; pa = (VV *)p->pa; pb = (VV *)p->pb;
         q = (VV *)p->q; z = (VV *)p->z; y = (VV *)p->y;
         st = p->st;
         part = p->partials;
         err = &p->st->error;
-        mA = view<VM>(A, tpA);
-        SLA_TRY(LQ::setup(A, tpA, &gA));
+        SLA_TRY(LQ.setup(A, s));
         gv = vec_grid(A);
         if (p->kind == 1)
             dinv = (const VV *)(sizeof(VV) == 8 ? M->d_dinv64 : M->d_dinv);
         else if (p->kind == 0)
             dinv = (const VV *)p->y;  // ones (y is unused without SPAI)
         if (p->kind == 2) {
-            const TilePart *tpG, *tpGT;
-            SLA_TRY(ensure_tiles(const_cast<sla_csr *>(M->G), TileCfg<K>::D, TileCfg<K>::RMAX, s, &tpG));
-            SLA_TRY(ensure_tiles(M->GT, TileCfg<K>::D, TileCfg<K>::RMAX, s, &tpGT));
-            mG = view<VM>(M->G, tpG);
-            mGT = view<VM>(M->GT, tpGT);
-            SLA_TRY(LZ::setup(M->G, tpG, &gG));
-            SLA_TRY(LUS::setup(M->GT, tpGT, &gGT));
+            SLA_TRY(LZ.setup(M->G, s));
+            SLA_TRY(LUS.setup(M->GT, s));
         }
-        p->grid_tiles_A = gA;
-        p->grid_tiles_G = gG;
-        p->grid_tiles_GT = gGT;
+        p->grid_tiles_A = LQ.grid;
+        p->grid_tiles_G = LZ.grid;
+        p->grid_tiles_GT = LUS.grid;
         p->grid_vec = gv;
         return SLA_SUCCESS;
     }
     void Q(cudaStream_t s, const VV *pold, VV *pnew) const
     {
-        LQ::launch(s, gA, mA, OpQ<VV, K>{z, pold, pnew, q, st}, part, st, err);
+        LQ.launch(s, OpQ<VV, K>{z, pold, pnew, q, st}, part, st, err);
     }
     void UJ(cudaStream_t s, const VV *pcur) const
     {
@@ -721,11 +636,11 @@ struct PlanKernels {
     }
     void US(cudaStream_t s, const VV *rold, VV *rnew, const VV *pcur) const
     {
-        LUS::launch(s, gGT, mGT, OpUS<VV, K>{rold, q, pcur, x, rnew, x, y, st}, part, st, err);
+        LUS.launch(s, OpUS<VV, K>{rold, q, pcur, x, rnew, x, y, st}, part, st, err);
     }
     void Z(cudaStream_t s, const VV *rcur) const
     {
-        LZ::launch(s, gG, mG, OpZ<VV, K>{y, rcur, z, st}, part, st, err);
+        LZ.launch(s, OpZ<VV, K>{y, rcur, z, st}, part, st, err);
     }
 };
 
@@ -863,82 +778,6 @@ static sla_status run_k(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, d
     k_copy_out<VV, K><<<gv, 256, 0, s>>>(n, nrhs, (const VV *)p->x, (VV *)X);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
-}
-
-// ------------------------------------------------------------------ dispatch
-#define SLA_DISPATCH_K(K_, FN, ...)                                                    \
-    switch (K_) {                                                                      \
-    case 1: return FN<VM, VV, 1>(__VA_ARGS__);                                         \
-    case 2: return FN<VM, VV, 2>(__VA_ARGS__);                                         \
-    case 4: return FN<VM, VV, 4>(__VA_ARGS__);                                         \
-    case 8: return FN<VM, VV, 8>(__VA_ARGS__);                                         \
-    case 16: return FN<VM, VV, 16>(__VA_ARGS__);                                       \
-    default: return fail(SLA_ERR_INVALID_ARG, "unsupported right-hand-side count");    \
-    }
-
-template <typename VM, typename VV>
-static sla_status capture_mv(sla_csr *A, Plan *p) { SLA_DISPATCH_K(p->K, capture_k, A, p) }
-template <typename VM, typename VV>
-static sla_status times_mv(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s)
-{
-    SLA_DISPATCH_K(p->K, times_k, A, p, nrhs, reps, h_ms, s)
-}
-template <typename VM, typename VV>
-static sla_status run_mv(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,
-                         long long maxit, cudaStream_t s)
-{
-    SLA_DISPATCH_K(p->K, run_k, A, p, nrhs, B, X, tol, maxit, s)
-}
-
-sla_status capture_plan_graph(sla_csr *A, Plan *p)
-{
-    if (A->dtype == SLA_F64)
-        return capture_mv<double, double>(A, p);
-    return p->vec64 ? capture_mv<float, double>(A, p) : capture_mv<float, float>(A, p);
-}
-
-sla_status kernel_times(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s)
-{
-    if (A->dtype == SLA_F64)
-        return times_mv<double, double>(A, p, nrhs, reps, h_ms, s);
-    return p->vec64 ? times_mv<float, double>(A, p, nrhs, reps, h_ms, s)
-                    : times_mv<float, float>(A, p, nrhs, reps, h_ms, s);
-}
-
-sla_status run_plan(sla_csr *A, Plan *p, int nrhs, const void *B, void *X,
-                    const sla_pcg_opts *opts, sla_pcg_info *info, const void *grad_x,
-                    void *grad_out, cudaStream_t s)
-{
-    const bool f64 = A->dtype == SLA_F64 || p->vec64;
-    double tol = (opts && opts->rtol > 0) ? opts->rtol : (f64 ? 1e-10 : 1e-6);
-    long long n_sys = A->batch > 1 ? A->max_sys_n : A->n;
-    long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 10 * std::max<long long>(n_sys, 1);
-    sla_status st;
-    if (A->dtype == SLA_F64)
-        st = run_mv<double, double>(A, p, nrhs, B, X, tol, maxit, s);
-    else if (p->vec64)
-        st = run_mv<float, double>(A, p, nrhs, B, X, tol, maxit, s);
-    else
-        st = run_mv<float, float>(A, p, nrhs, B, X, tol, maxit, s);
-    if (st != SLA_SUCCESS)
-        return st;
-    if (grad_out)
-        SLA_TRY(launch_pattern_grad(A, nrhs, p->vec64, X, grad_x, grad_out, s));
-    SLA_CUDA_TRY(cudaMemcpyAsync(p->h_st, p->st, sizeof(PcgState), cudaMemcpyDeviceToHost, s));
-    SLA_CUDA_TRY(cudaStreamSynchronize(s));
-    if (p->h_st->error)
-        return fail(SLA_ERR_CUDA, "a pipeline wait inside a solver kernel ran out of time; results are invalid");
-    sla_status worst = SLA_SUCCESS;
-    for (int c = 0; c < nrhs; ++c) {
-        if (info) {
-            info[c].iters = p->h_st->iters[c];
-            info[c].relres = p->h_st->relres[c];
-            info[c].status = p->h_st->status[c];
-            info[c].reserved = 0;
-        }
-        worst = std::max(worst, (sla_status)p->h_st->status[c]);
-    }
-    return worst;
 }
 
 }  // namespace sla

@@ -171,6 +171,22 @@ sla_status run_plan(sla_csr *A, Plan *p, int nrhs, const void *B, void *X,
                     const sla_pcg_opts *opts, sla_pcg_info *info, const void *grad_x,
                     void *grad_out, cudaStream_t s);
 sla_status kernel_times(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s);
+
+// per-precision instantiations: ff = fp32 values/vectors, dd = fp64, fd = fp32 values with
+// fp64 vectors
+#define SLA_COMBO_DECL(T)                                                                            \
+    sla_status capture_##T(sla_csr *A, Plan *p);                                                    \
+    sla_status times_##T(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s);     \
+    sla_status run_##T(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,            \
+                       long long maxit, cudaStream_t s);                                            \
+    sla_status grad_##T(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g,         \
+                        cudaStream_t s);
+SLA_COMBO_DECL(ff)
+SLA_COMBO_DECL(dd)
+SLA_COMBO_DECL(fd)
+#undef SLA_COMBO_DECL
+sla_status spmv_ff(const sla_csr *A, int nrhs, const void *x, void *y, cudaStream_t s);
+sla_status spmv_dd(const sla_csr *A, int nrhs, const void *x, void *y, cudaStream_t s);
 sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B, void *X,
                           const void *Xfwd, void *G, const sla_pcg_opts *opts, sla_pcg_info *info,
                           cudaStream_t s);

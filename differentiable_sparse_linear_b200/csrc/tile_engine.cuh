@@ -254,7 +254,7 @@ constexpr int HDR_LONG = 1, HDR_LAST = 2;
 //   static constexpr int NP, NS, NV;               dots per rhs, staged scalars, staged row vectors
 //   const VV *row_vec(int v) const;                base of staged own-row vector v (K-interleaved)
 //   bool skip() const;  void stage(double *s) const;
-//   double operand(int64_t j, int c, const double *s) const;          gathered value
+//   VV operand(int64_t j, int c, const double *s) const;              gathered value
 //   template <int N> void emit(int64_t i, const double (&acc)[K], double (&part)[N],
 //                              const double *s, const RowVecs<VV,K,NV> &rv) const;
 //   void finalize(const double *sums) const;       sums[p*K + c]
@@ -401,13 +401,26 @@ k_tile(const MatView<VM> m, const Op op, double *partials, PcgState *st, int *er
             const VM *vv = s_val + (kb - sv.ab);
 
             if (is_long) {
-                // chunk of one long row: thread-strided partial sums, kept across chunks
-                for (int e = tid; e < nk; e += TC) {
-                    const double a = (double)vv[e];
-                    const int64_t j = cc[e];
+                // chunk of one long row: thread-strided partial sums, kept across chunks;
+                // all of this thread's operand loads are issued before the first use
+                constexpr int GL = (D + TC - 1) / TC;
+                double ov[GL][K];
+#pragma unroll
+                for (int u = 0; u < GL; ++u) {
+                    const int e = tid + u * TC;
 #pragma unroll
                     for (int c = 0; c < K; ++c)
-                        lacc[c] = fma(a, op.operand(j, c, s_scal), lacc[c]);
+                        ov[u][c] = e < nk ? (double)op.operand(cc[e], c, s_scal) : 0.0;
+                }
+#pragma unroll
+                for (int u = 0; u < GL; ++u) {
+                    const int e = tid + u * TC;
+                    if (e < nk) {
+                        const double a = (double)vv[e];
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            lacc[c] = fma(a, ov[u][c], lacc[c]);
+                    }
                 }
                 if (flags & HDR_LAST) {
 #pragma unroll
@@ -431,11 +444,20 @@ k_tile(const MatView<VM> m, const Op op, double *partials, PcgState *st, int *er
                 // row ends relative to the tile's first entry: rend(x) = end of row x
                 const int32_t *rpp = s_rp + (r0 - sr.ab);
                 const int32_t kb32 = (int32_t)kb;
-                // 1. products (independent gathers)
-                for (int f = tid; f < nk * K; f += TC) {
+                // 1. products: every operand load of this thread in flight at once
+                constexpr int GU = (D * K + TC - 1) / TC;
+                double ov[GU];
+#pragma unroll
+                for (int u = 0; u < GU; ++u) {
+                    const int f = tid + u * TC;
                     const int e = f / K;
-                    const int c = f - e * K;
-                    s_prod[f] = (double)vv[e] * op.operand(cc[e], c, s_scal);
+                    ov[u] = f < nk * K ? (double)op.operand(cc[e], f - e * K, s_scal) : 0.0;
+                }
+#pragma unroll
+                for (int u = 0; u < GU; ++u) {
+                    const int f = tid + u * TC;
+                    if (f < nk * K)
+                        s_prod[f] = (double)vv[f / K] * ov[u];
                 }
                 sync();
                 // 2. merge-path split: largest x (rows finished) with rend(x-1) <= d0 - x
