@@ -101,6 +101,13 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def wait_first_sample(self, limit_s: float = 10.0):
+        """nvidia-smi's start-up takes driver locks; begin timing only once it samples."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < limit_s:
+            time.sleep(0.05)
+        time.sleep(0.25)
+
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
@@ -313,7 +320,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if rank == 0:
         clocks.start()
-        time.sleep(0.3)
+        clocks.wait_first_sample()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     total_iters = 0

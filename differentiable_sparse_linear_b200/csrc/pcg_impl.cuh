@@ -491,21 +491,28 @@ constexpr int ROWS_MAXL = 16;
 template <int K, typename VM, class Op>
 struct TileLaunch {
     using L = StageLayout<K, VM, typename Op::VV, Op::NV>;
+    using LR = RowTmaLayout<K, VM>;
     static constexpr int THREADS = TileCfg<K>::TC + 32;
     static constexpr size_t SMEM = TileCfg<K>::NST * L::BYTES;
+    static constexpr int RTHREADS = RowTmaCfg<K>::TC + 32;
+    static constexpr size_t RSMEM = RowTmaCfg<K>::NST * LR::BYTES;
     int grid = 0;
     int maxl = 0;                 // 0: tile engine; else the short-row engine's MAXL
     MatView<VM> m{};
 
     template <int MAXL>
-    sla_status setup_rows(const sla_csr *A)
+    sla_status setup_rows(const sla_csr *A, cudaStream_t s)
     {
-        auto kern = k_rows<K, VM, MAXL, Op>;
+        const TilePart *tp;
+        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), RowTmaCfg<K>::D,
+                             RowTmaCfg<K>::TC * RowTmaCfg<K>::RPT, s, &tp));
+        m = view<VM>(A, tp);
+        auto kern = k_rows_tma<K, VM, MAXL, Op>;
+        SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RSMEM));
         int per_sm = 0;
-        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ROW_T, 0));
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, RTHREADS, RSMEM));
         per_sm = std::max(per_sm, 1);
-        const int64_t need = (A->n + ROW_T - 1) / ROW_T;
-        grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)per_sm * A->num_sms));
+        grid = std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
         maxl = MAXL;
         return SLA_SUCCESS;
     }
@@ -513,21 +520,13 @@ struct TileLaunch {
     sla_status setup(const sla_csr *A, cudaStream_t s)
     {
         if (A->max_row_len <= ROWS_MAXL) {
-            // the row engine needs no tiles; the view carries the matrix arrays only
-            m.rp = A->rp;
-            m.ci = A->ci;
-            m.val = (const VM *)A->val;
-            m.desc = nullptr;
-            m.n_tiles = 0;
-            m.n = A->n;
-            m.nnz = A->nnz;
             if (A->max_row_len <= 4)
-                return setup_rows<4>(A);
+                return setup_rows<4>(A, s);
             if (A->max_row_len <= 6)
-                return setup_rows<6>(A);
+                return setup_rows<6>(A, s);
             if (A->max_row_len <= 8)
-                return setup_rows<8>(A);
-            return setup_rows<16>(A);
+                return setup_rows<8>(A, s);
+            return setup_rows<16>(A, s);
         }
         const TilePart *tp;
         SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), TileCfg<K>::D, TileCfg<K>::RMAX, s, &tp));
@@ -541,16 +540,15 @@ struct TileLaunch {
         maxl = 0;
         return SLA_SUCCESS;
     }
-    bool empty() const { return maxl == 0 ? m.n_tiles == 0 : m.n == 0; }
     void launch(cudaStream_t s, const Op &op, double *part, PcgState *st, int *err) const
     {
-        if (empty())
+        if (m.n_tiles == 0)
             return;
         switch (maxl) {
-        case 4: k_rows<K, VM, 4, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
-        case 6: k_rows<K, VM, 6, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
-        case 8: k_rows<K, VM, 8, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
-        case 16: k_rows<K, VM, 16, Op><<<grid, ROW_T, 0, s>>>(m, op, part, st); break;
+        case 4: k_rows_tma<K, VM, 4, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
+        case 6: k_rows_tma<K, VM, 6, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
+        case 8: k_rows_tma<K, VM, 8, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
+        case 16: k_rows_tma<K, VM, 16, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
         default: k_tile<K, VM, Op><<<grid, THREADS, SMEM, s>>>(m, op, part, st, err); break;
         }
     }
