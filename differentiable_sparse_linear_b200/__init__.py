@@ -28,6 +28,7 @@ __all__ = [
     "sla_version", "sla_csr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
+    "sla_pcg_solve_batched_noalloc",
     "sla_workspace_bytes", "sla_pcg_kernel_times", "solve",
 ]
 
@@ -265,6 +266,19 @@ def sla_pcg_solve_batched(A: Matrix, M: Optional[Preconditioner], B: torch.Tenso
     opts = _opts(rtol, maxit, vector_f64)
     _check(lib().sla_pcg_solve_batched(A.handle, _mh(M), nrhs, _ptr(B), _ptr(X), C.byref(opts),
                                        infos, _stream(stream)), "sla_pcg_solve_batched")
+    return X, _infos(infos)
+
+
+def sla_pcg_solve_batched_noalloc(A: Matrix, M: Optional[Preconditioner], B: torch.Tensor,
+                                  X: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
+                                  stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
+    """List-handle solve that allocates no device memory inside the call (X must be given
+    by callers that cannot allocate either; here it is created when omitted)."""
+    X = torch.empty_like(B) if X is None else X
+    infos = (_lib.sla_pcg_info * A.batch)()
+    opts = _opts(rtol, maxit)
+    _check(lib().sla_pcg_solve_batched_noalloc(A.handle, _mh(M), _ptr(B), _ptr(X), C.byref(opts), infos,
+                                               _stream(stream)), "sla_pcg_solve_batched_noalloc")
     return X, _infos(infos)
 
 

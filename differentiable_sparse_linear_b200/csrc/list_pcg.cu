@@ -256,3 +256,25 @@ sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B,
 }
 
 }  // namespace sla
+
+namespace sla {
+
+// The list kernel with a caller-provided device array for the per-system results (no
+// allocation here); the caller copies the results back and synchronises.
+sla_status launch_list_kernel(const sla_csr *A, const sla_precond *M, const void *B, void *X,
+                              const sla_pcg_opts *opts, sla_pcg_info *d_info, cudaStream_t s)
+{
+    if (M && M->kind != 1)
+        return fail(SLA_ERR_UNSUPPORTED, "list solves support the Jacobi preconditioner or none");
+    if ((size_t)7 * A->max_sys_n * (A->dtype == SLA_F32 ? 4 : 8) > 200 * 1024)
+        return fail(SLA_ERR_UNSUPPORTED, "list solve: largest system exceeds the shared-memory size");
+    const double tol = (opts && opts->rtol > 0) ? opts->rtol : (A->dtype == SLA_F32 ? 1e-6 : 1e-10);
+    const long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 0;
+    if (A->dtype == SLA_F32)
+        return list_v<float>(A, M ? (const float *)M->d_dinv : nullptr, B, X, nullptr, nullptr, tol, maxit,
+                             d_info, s);
+    return list_v<double>(A, M ? (const double *)M->d_dinv64 : nullptr, B, X, nullptr, nullptr, tol, maxit,
+                          d_info, s);
+}
+
+}  // namespace sla

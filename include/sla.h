@@ -195,6 +195,23 @@ SLA_API sla_status sla_pcg_adjoint_batched(const sla_csr *A, const sla_precond *
 SLA_API sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *d_lam, const void *d_x,
                             void *d_g, void *stream);
 
+/* The list solve of sla_pcg_solve_batched (list handle, nrhs = 1, Jacobi or no
+ * preconditioner) for callers that cannot allocate device memory while they solve --
+ * code under a memory pool or budget that owns the device's memory, hosts that forbid
+ * allocation after start-up, or code that must avoid the synchronisation an allocation or
+ * free can bring.  This call allocates nothing: the per-system results pass through a
+ * fixed array in the library's own device memory (1.5 MiB, held by every GPU that loads
+ * the library until the process exits), and at most 65536 systems are accepted per call
+ * (SLA_ERR_INVALID_ARG beyond that).  The first call on a device looks up that array's
+ * device address, so make it before any stream capture.  All calls on a device share the
+ * array: calls that overlap on the GPU race on it.  The matrix and preconditioner handles
+ * are created beforehand with the usual calls.  There is no counterpart on the pages this
+ * library follows: it is an interface variant, not a different method. */
+SLA_API sla_status sla_pcg_solve_batched_noalloc(const sla_csr *A, const sla_precond *M,
+                                                 const void *d_B, void *d_X,
+                                                 const sla_pcg_opts *opts, sla_pcg_info *h_info,
+                                                 void *stream);
+
 /* Per-kernel device time of one PCG iteration (metrics).  On the workspace of the
  * (A, M, nrhs, vector_f64) solver -- normally right after a solve, so it holds that solve's vectors --
  * launches the iteration's kernels `reps` times in loop order, each bracketed by CUDA
