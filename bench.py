@@ -155,13 +155,16 @@ def measured_peaks() -> tuple[float, str]:
         return 6650.0, "fallback"
 
 
+KERNEL_SOURCES = ("row_engine.cuh", "tile_engine.cuh", "pcg_impl.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the sources that define the SpMV/PCG kernels (ncu traffic is tied to it)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differentiable_sparse_linear_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(f.read())
+    for fn in KERNEL_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
