@@ -24,7 +24,7 @@ LIB = os.path.join(LIBDIR, "libsla.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-           "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]
+           "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills", "-Werror", "cross-execution-space-call"]
 
 
 def nvcc() -> str:

@@ -82,6 +82,98 @@ sla_status ensure_tiles(sla_csr *A, int D, int RMAX, cudaStream_t s, const TileP
     return SLA_SUCCESS;
 }
 
+// Operand windows: for each tile, the rows of the gathered vectors its columns (and its own
+// rows) touch, as at most WSEG 4-row-aligned ranges totalling at most wmax rows; tiles that
+// do not fit get nseg = 0 (global gathers).  Gaps of up to 32 rows are bridged.
+sla_status ensure_windows(sla_csr *A, const TilePart *tp_c, int wmax, cudaStream_t s)
+{
+    TilePart *tp = const_cast<TilePart *>(tp_c);
+    if (tp->win_rows == wmax)
+        return SLA_SUCCESS;
+    if (A->h_ci.size() != (size_t)A->nnz) {
+        A->h_ci.resize((size_t)A->nnz);
+        if (A->nnz > 0) {
+            SLA_CUDA_TRY(cudaMemcpyAsync(A->h_ci.data(), A->ci, (size_t)A->nnz * sizeof(int32_t),
+                                         cudaMemcpyDeviceToHost, s));
+            SLA_CUDA_TRY(cudaStreamSynchronize(s));
+        }
+    }
+    std::vector<int2> desc((size_t)tp->n_tiles + 1);
+    if (tp->n_tiles > 0)
+        SLA_CUDA_TRY(cudaMemcpy(desc.data(), tp->d_desc, desc.size() * sizeof(int2), cudaMemcpyDeviceToHost));
+    std::vector<WinDesc> win((size_t)std::max(tp->n_tiles, 1));
+    const int64_t GAP = 32;
+    for (int t = 0; t < tp->n_tiles; ++t) {
+        WinDesc w{};
+        int64_t lo[8], hi[8];   // closed ranges
+        int ns = 0;
+        bool ok = wmax > 0;
+        auto add = [&](int64_t j) {
+            for (int i = 0; i < ns; ++i)
+                if (j >= lo[i] - GAP && j <= hi[i] + GAP) {
+                    lo[i] = std::min(lo[i], j);
+                    hi[i] = std::max(hi[i], j);
+                    return;
+                }
+            if (ns == 8) {
+                ok = false;
+                return;
+            }
+            lo[ns] = hi[ns] = j;
+            ++ns;
+        };
+        const int r0 = desc[t].x, r1 = desc[t + 1].x;
+        if (r1 > r0) {
+            add(r0);
+            add(r1 - 1);
+        }
+        for (int64_t k = (uint32_t)desc[t].y; ok && k < (int64_t)(uint32_t)desc[t + 1].y; ++k)
+            add(A->h_ci[(size_t)k]);
+        // sort, align to 4 rows, merge
+        int64_t L[8], H[8];
+        int m = 0;
+        if (ok) {
+            for (int i = 0; i < ns; ++i) {
+                int b = i;
+                for (int jdx = i + 1; jdx < ns; ++jdx)
+                    if (lo[jdx] < lo[b])
+                        b = jdx;
+                std::swap(lo[i], lo[b]);
+                std::swap(hi[i], hi[b]);
+            }
+            for (int i = 0; i < ns; ++i) {
+                const int64_t a = lo[i] & ~(int64_t)3, e = (hi[i] + 1 + 3) & ~(int64_t)3;
+                if (m > 0 && a <= H[m - 1] + GAP)
+                    H[m - 1] = std::max(H[m - 1], e);
+                else {
+                    L[m] = a;
+                    H[m] = e;
+                    ++m;
+                }
+            }
+            int64_t total = 0;
+            for (int i = 0; i < m; ++i)
+                total += H[i] - L[i];
+            if (m > WSEG || total > wmax || (m > 0 && H[m - 1] > A->n))
+                ok = false;
+        }
+        if (ok) {
+            w.nseg = m;
+            for (int i = 0; i < m; ++i) {
+                w.a[i] = (int)L[i];
+                w.l[i] = (int)(H[i] - L[i]);
+            }
+        }
+        win[(size_t)t] = w;
+    }
+    if (!tp->d_win)
+        SLA_CUDA_TRY(cudaMalloc((void **)&tp->d_win, win.size() * sizeof(WinDesc)));
+    SLA_CUDA_TRY(cudaMemcpyAsync(tp->d_win, win.data(), win.size() * sizeof(WinDesc), cudaMemcpyHostToDevice, s));
+    SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    tp->win_rows = wmax;
+    return SLA_SUCCESS;
+}
+
 static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 static size_t vec_bytes(const sla_csr *A, int vec64) { return vec64 ? 8 : vbytes(A->dtype); }
@@ -247,8 +339,11 @@ static void free_csr(sla_csr *A)
     for (Plan *p : A->plans)
         destroy_plan(p);
     A->plans.clear();
-    for (auto &kv : A->tiles)
+    for (auto &kv : A->tiles) {
         cudaFree(kv.second.d_desc);
+        if (kv.second.d_win)
+            cudaFree(kv.second.d_win);
+    }
     if (A->d_err)
         cudaFree(A->d_err);
     if (A->d_sys_off)

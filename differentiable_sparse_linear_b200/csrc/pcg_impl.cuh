@@ -113,12 +113,20 @@ template <typename V, int K>
 struct OpSpmv {
     using VV = V;
     static constexpr int NP = 0, NS = 0, NV = 0;
+    static constexpr int NG = 1;
     const V *x;
     V *y;
     int ld, nc;
     __device__ const V *row_vec(int) const { return nullptr; }
+    __host__ __device__ const V *gvec(int) const { return x; }
+    __host__ __device__ int gstride() const { return ld; }
+    static __device__ constexpr int rv_src(int) { return -1; }
     __device__ bool skip() const { return false; }
     __device__ void stage(double *) const {}
+    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *) const
+    {
+        return c < nc ? g[0] : (V)0;
+    }
     __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
     {
         return c < nc ? __ldg(&x[j * ld + c]) : (V)0;
@@ -145,12 +153,20 @@ struct OpQ {
     V *p_new;
     V *q;
     PcgState *st;
+    static constexpr int NG = 2;
     __device__ const V *row_vec(int v) const { return v == 0 ? p_old : z; }
+    __host__ __device__ const V *gvec(int g) const { return g == 0 ? p_old : z; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int v) { return v; }
     __device__ bool skip() const { return *(volatile int *)&st->all_done; }
     __device__ void stage(double *s) const
     {
         for (int c = 0; c < K; ++c)
             s[c] = st->beta[c];
+    }
+    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *s) const
+    {
+        return (V)__fma_rn(s[c], (double)g[0], (double)g[1]);
     }
     __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
     {
@@ -185,7 +201,11 @@ struct OpUS {
     V *x;
     V *y;
     PcgState *st;
+    static constexpr int NG = 2;
     __device__ const V *row_vec(int v) const { return v == 0 ? r_old : v == 1 ? q : v == 2 ? p : x_in; }
+    __host__ __device__ const V *gvec(int g) const { return g == 0 ? r_old : q; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int v) { return v < 2 ? v : -1; }
     __device__ bool skip() const { return *(volatile int *)&st->all_done; }
     __device__ void stage(double *s) const
     {
@@ -197,6 +217,10 @@ struct OpUS {
     __device__ __forceinline__ V rnew(V ro, V qv, int c, const double *s) const
     {
         return s[K + c] != 0.0 ? (V)__fma_rn(-s[c], (double)qv, (double)ro) : ro;
+    }
+    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *s) const
+    {
+        return rnew(g[0], g[1], c, s);
     }
     __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
     {
@@ -234,9 +258,14 @@ struct OpZ {
     const V *r;
     V *z;
     PcgState *st;
+    static constexpr int NG = 1;
     __device__ const V *row_vec(int) const { return r; }
+    __host__ __device__ const V *gvec(int) const { return y; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int) { return -1; }
     __device__ bool skip() const { return *(volatile int *)&st->all_done; }
     __device__ void stage(double *s) const { s[0] = st->eps; }
+    __device__ __forceinline__ V combine(const V (&g)[NG], int, const double *) const { return g[0]; }
     __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
     {
         return y[j * K + c];
@@ -491,7 +520,7 @@ constexpr int ROWS_MAXL = 16;
 template <int K, typename VM, class Op>
 struct TileLaunch {
     using L = StageLayout<K, VM, typename Op::VV, Op::NV>;
-    using LR = RowTmaLayout<K, VM>;
+    using LR = RowTmaLayout<K, VM, typename Op::VV, Op::NG>;
     static constexpr int THREADS = TileCfg<K>::TC + 32;
     static constexpr size_t SMEM = TileCfg<K>::NST * L::BYTES;
     static constexpr int RTHREADS = RowTmaCfg<K>::TC + 32;
@@ -499,6 +528,7 @@ struct TileLaunch {
     int grid = 0;
     int maxl = 0;                 // 0: tile engine; else the short-row engine's MAXL
     MatView<VM> m{};
+    const WinDesc *win = nullptr; // operand windows (short-row engine, K <= 2)
 
     template <int MAXL>
     sla_status setup_rows(const sla_csr *A, cudaStream_t s)
@@ -507,6 +537,10 @@ struct TileLaunch {
         SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), RowTmaCfg<K>::D,
                              RowTmaCfg<K>::TC * RowTmaCfg<K>::RPT, s, &tp));
         m = view<VM>(A, tp);
+        if (RowTmaCfg<K>::WMAX > 0) {
+            SLA_TRY(ensure_windows(const_cast<sla_csr *>(A), tp, RowTmaCfg<K>::WMAX, s));
+            win = tp->d_win;
+        }
         auto kern = k_rows_tma<K, VM, MAXL, Op>;
         SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RSMEM));
         int per_sm = 0;
@@ -544,11 +578,16 @@ struct TileLaunch {
     {
         if (m.n_tiles == 0)
             return;
+        // windows are bulk-copied from the gathered vectors: they need 16-byte alignment
+        bool aligned = true;
+        for (int g = 0; g < Op::NG; ++g)
+            aligned = aligned && (((uintptr_t)op.gvec(g) & 15) == 0);
+        const WinDesc *w = aligned ? win : nullptr;
         switch (maxl) {
-        case 4: k_rows_tma<K, VM, 4, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
-        case 6: k_rows_tma<K, VM, 6, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
-        case 8: k_rows_tma<K, VM, 8, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
-        case 16: k_rows_tma<K, VM, 16, Op><<<grid, RTHREADS, RSMEM, s>>>(m, op, part, st, err); break;
+        case 4: k_rows_tma<K, VM, 4, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
+        case 6: k_rows_tma<K, VM, 6, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
+        case 8: k_rows_tma<K, VM, 8, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
+        case 16: k_rows_tma<K, VM, 16, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         default: k_tile<K, VM, Op><<<grid, THREADS, SMEM, s>>>(m, op, part, st, err); break;
         }
     }

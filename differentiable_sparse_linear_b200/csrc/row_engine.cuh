@@ -105,25 +105,36 @@ namespace sla {
 // items (rows + entries); rows have at most MAXL entries, so there are no long rows.
 // Consumers release a stage by arriving on its "empty" mbarrier (one arrival per thread),
 // so no block-wide barrier is needed in the steady state.
+//
+// Operand windows (WIN): for a banded matrix the columns a tile touches lie in a few
+// contiguous row ranges of the gathered vectors (for a 2D grid: the rows one grid line
+// above, the tile's own rows, one grid line below).  Those ranges, precomputed per tile on
+// the host (at most WSEG segments, 4-row aligned, at most WMAX rows in all), are bulk-copied
+// into the stage with the matrix arrays, and the consumers read their operands from shared
+// memory.  The gather latency is then hidden by the pipeline like the matrix stream's.  A
+// tile whose columns do not fit keeps global gathers.
 template <int K>
 struct RowTmaCfg;
-template <> struct RowTmaCfg<1> { static constexpr int TC = 256, RPT = 2, D = 3072, NST = 2; };
-template <> struct RowTmaCfg<2> { static constexpr int TC = 256, RPT = 2, D = 3072, NST = 2; };
-template <> struct RowTmaCfg<4> { static constexpr int TC = 256, RPT = 1, D = 2048, NST = 2; };
-template <> struct RowTmaCfg<8> { static constexpr int TC = 256, RPT = 1, D = 2048, NST = 2; };
-template <> struct RowTmaCfg<16> { static constexpr int TC = 128, RPT = 1, D = 1024, NST = 2; };
+template <> struct RowTmaCfg<1> { static constexpr int TC = 256, RPT = 2, D = 2048, NST = 2, WMAX = 2048; };
+template <> struct RowTmaCfg<2> { static constexpr int TC = 256, RPT = 2, D = 2048, NST = 2, WMAX = 1024; };
+template <> struct RowTmaCfg<4> { static constexpr int TC = 256, RPT = 1, D = 2048, NST = 2, WMAX = 0; };
+template <> struct RowTmaCfg<8> { static constexpr int TC = 256, RPT = 1, D = 2048, NST = 2, WMAX = 0; };
+template <> struct RowTmaCfg<16> { static constexpr int TC = 128, RPT = 1, D = 1024, NST = 2, WMAX = 0; };
 
-template <int K, typename VM>
+template <int K, typename VM, typename VV, int NG>
 struct RowTmaLayout {
     static constexpr int D = RowTmaCfg<K>::D;
     static constexpr int RMAX = RowTmaCfg<K>::TC * RowTmaCfg<K>::RPT;
+    static constexpr int WMAX = RowTmaCfg<K>::WMAX;
     static constexpr int PAD = 8;
     static constexpr size_t align16(size_t b) { return (b + 15) & ~(size_t)15; }
-    static constexpr size_t HDR = 32;
+    static constexpr size_t HDR = 128;
     static constexpr size_t COL_OFF = HDR;
     static constexpr size_t VAL_OFF = COL_OFF + align16((D + PAD) * 4);
     static constexpr size_t RP_OFF = VAL_OFF + align16((D + PAD) * sizeof(VM));
-    static constexpr size_t BYTES = align16(RP_OFF + (RMAX + 1 + PAD) * 4);
+    static constexpr size_t WIN_OFF = RP_OFF + align16((RMAX + 1 + PAD) * 4);
+    static constexpr size_t WIN_STRIDE = align16((size_t)WMAX * K * sizeof(VV));
+    static constexpr size_t BYTES = align16(WIN_OFF + (WMAX > 0 ? NG : 0) * WIN_STRIDE);
 };
 
 // Own-row vector values loaded into registers before the row's gathers.
@@ -135,17 +146,20 @@ struct RowVals {
 
 template <int K, typename VM, int MAXL, class Op>
 __global__ void __launch_bounds__(RowTmaCfg<K>::TC + 32)
-k_rows_tma(const MatView<VM> m, const Op op, double *partials, PcgState *st, int *err)
+k_rows_tma(const MatView<VM> m, const WinDesc *win, const Op op, double *partials, PcgState *st,
+           int *err)
 {
     using VV = typename Op::VV;
     using Acc = typename std::conditional<sizeof(VM) == 4 && sizeof(VV) == 4, float, double>::type;
     constexpr int TC = RowTmaCfg<K>::TC;
     constexpr int RPT = RowTmaCfg<K>::RPT;
     constexpr int NST = RowTmaCfg<K>::NST;
+    constexpr int WMAX = RowTmaCfg<K>::WMAX;
     constexpr int NV = Op::NV;
+    constexpr int NG = Op::NG;
     constexpr int NPK = Op::NP * K;
     constexpr int NR = NPK > 0 ? NPK : 1;
-    using L = RowTmaLayout<K, VM>;
+    using L = RowTmaLayout<K, VM, VV, NG>;
 
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ uint64_t full_bar[NST], empty_bar[NST];
@@ -165,6 +179,7 @@ k_rows_tma(const MatView<VM> m, const Op op, double *partials, PcgState *st, int
         op.stage(s_scal);
     }
     __syncthreads();
+    const int gs = op.gstride();
 
     // ---------------------------------------------------------------- producer
     if (threadIdx.x >= TC) {
@@ -174,6 +189,11 @@ k_rows_tma(const MatView<VM> m, const Op op, double *partials, PcgState *st, int
         uint32_t phase = 0;
         for (int t = blockIdx.x; t < m.n_tiles; t += gridDim.x) {
             const int2 d0 = m.desc[t], d1 = m.desc[t + 1];
+            WinDesc wd;
+            if (WMAX > 0 && win)
+                wd = win[t];
+            else
+                wd.nseg = 0;
             const int r0 = d0.x, r1 = d1.x;
             const int64_t kb = (int64_t)(uint32_t)d0.y, ke = (int64_t)(uint32_t)d1.y;
             mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, err);
@@ -190,10 +210,27 @@ k_rows_tma(const MatView<VM> m, const Op op, double *partials, PcgState *st, int
             hdr[5] = (int32_t)(kb - sv.ab);          // ... in val[]
             hdr[6] = (int32_t)(r0 - sr.ab);          // smem index of row_ptr[r0]
             hdr[7] = (sc.tail < ke || sv.tail < ke || sr.tail < (int64_t)r1 + 1) ? 1 : 0;
-            mbar_arrive_expect_tx(&full_bar[stage], sc.bytes() + sv.bytes() + sr.bytes());
+            uint32_t tx = sc.bytes() + sv.bytes() + sr.bytes();
+            if (WMAX > 0) {
+                *(WinDesc *)(sb + 32) = wd;
+                for (int s2 = 0; s2 < wd.nseg; ++s2)
+                    tx += (uint32_t)NG * (uint32_t)wd.l[s2] * (uint32_t)gs * (uint32_t)sizeof(VV);
+            }
+            mbar_arrive_expect_tx(&full_bar[stage], tx);
             span_issue(sc, sb + L::COL_OFF, m.ci, &full_bar[stage]);
             span_issue(sv, sb + L::VAL_OFF, m.val, &full_bar[stage]);
             span_issue(sr, sb + L::RP_OFF, m.rp, &full_bar[stage]);
+            if (WMAX > 0) {
+                int cum = 0;
+                for (int s2 = 0; s2 < wd.nseg; ++s2) {
+                    const uint32_t bytes = (uint32_t)wd.l[s2] * (uint32_t)gs * (uint32_t)sizeof(VV);
+#pragma unroll
+                    for (int g = 0; g < NG; ++g)
+                        bulk_g2s(sb + L::WIN_OFF + g * L::WIN_STRIDE + (size_t)cum * gs * sizeof(VV),
+                                 op.gvec(g) + (int64_t)wd.a[s2] * gs, bytes, &full_bar[stage]);
+                    cum += wd.l[s2];
+                }
+            }
             if (++stage == NST) {
                 stage = 0;
                 phase ^= 1u;
@@ -241,9 +278,107 @@ k_rows_tma(const MatView<VM> m, const Op op, double *partials, PcgState *st, int
         const int32_t *cc = s_col + hdr[4];
         const VM *vv = s_val + hdr[5];
         const int32_t *rpp = s_rp + hdr[6];
+        // window of this tile (nseg == 0: operands come from global memory)
+        int nseg = 0, wa[WSEG], wl[WSEG], wc[WSEG];
+        if (WMAX > 0) {
+            const WinDesc *wd = (const WinDesc *)(sb + 32);
+            nseg = wd->nseg;
+            int cum = 0;
+#pragma unroll
+            for (int s2 = 0; s2 < WSEG; ++s2) {
+                wa[s2] = wd->a[s2];
+                wl[s2] = s2 < nseg ? wd->l[s2] : 0;
+                wc[s2] = cum;
+                cum += wl[s2];
+            }
+        }
+        const VV *swin = (const VV *)(sb + L::WIN_OFF);
+        auto wrow = [&](int j) -> int {   // window row of vector row j, -1 if outside
+            int pos = -1;
+#pragma unroll
+            for (int s2 = 0; s2 < WSEG; ++s2)
+                if ((unsigned)(j - wa[s2]) < (unsigned)wl[s2])
+                    pos = wc[s2] + (j - wa[s2]);
+            return pos;
+        };
 
-        int len[RPT], off[RPT];
         RowVals<VV, K, NV> rvals[RPT];
+        if (WMAX > 0 && nseg > 0) {
+            // windowed tile: operands and own-row values of gathered vectors come from shared
+            // memory, so the row sums are formed while reading; only the other own-row
+            // vectors are loaded from global memory (issued first).
+            const VV *wv[NG];
+#pragma unroll
+            for (int g = 0; g < NG; ++g)
+                wv[g] = swin + (size_t)g * (L::WIN_STRIDE / sizeof(VV));
+#pragma unroll
+            for (int q = 0; q < RPT; ++q) {
+                const int r = tid + q * TC;
+#pragma unroll
+                for (int v = 0; v < NV; ++v)
+                    if (Op::rv_src(v) < 0)
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            rvals[q].v[v][c] = r < nr ? op.row_vec(v)[((int64_t)r0 + r) * K + c] : (VV)0;
+            }
+            double acc[RPT][K];
+#pragma unroll
+            for (int q = 0; q < RPT; ++q) {
+                const int r = tid + q * TC;
+                const bool live = r < nr;
+                const int o = live ? rpp[r] - kb32 : 0;
+                const int n_ = live ? rpp[r + 1] - kb32 - o : 0;
+                const int rw = live ? wrow(r0 + r) : 0;
+#pragma unroll
+                for (int v = 0; v < NV; ++v)
+                    if (Op::rv_src(v) >= 0)
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            rvals[q].v[v][c] = !live ? (VV)0
+                                               : rw >= 0 ? wv[Op::rv_src(v)][(size_t)rw * gs + c]
+                                                         : op.row_vec(v)[((int64_t)r0 + r) * K + c];
+                Acc a[K];
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    a[c] = (Acc)0;
+#pragma unroll
+                for (int u = 0; u < MAXL; ++u) {
+                    if (u < n_) {
+                        const int j = cc[o + u];
+                        const int w = wrow(j);       // always inside: the window was built from these columns
+                        const Acc av = (Acc)vv[o + u];
+#pragma unroll
+                        for (int c = 0; c < K; ++c) {
+                            VV gv[NG];
+#pragma unroll
+                            for (int g = 0; g < NG; ++g)
+                                gv[g] = w >= 0 ? wv[g][(size_t)w * gs + c] : op.gvec(g)[(int64_t)j * gs + c];
+                            a[c] = fma(av, (Acc)op.combine(gv, c, s_scal), a[c]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    acc[q][c] = (double)a[c];
+            }
+            // the stage's shared memory is no longer read: hand it back to the producer
+            fence_proxy_async_smem();
+            mbar_arrive(&empty_bar[stage]);
+            if (++stage == NST) {
+                stage = 0;
+                phase ^= 1u;
+            }
+#pragma unroll
+            for (int q = 0; q < RPT; ++q) {
+                const int r = tid + q * TC;
+                if (r < nr)
+                    op.emit((int64_t)r0 + r, acc[q], part, s_scal, rvals[q]);
+            }
+            continue;
+        }
+
+        // global gathers: every load of this thread in flight at once
+        int len[RPT], off[RPT];
         int cj[RPT][MAXL];
         VM av[RPT][MAXL];
 #pragma unroll

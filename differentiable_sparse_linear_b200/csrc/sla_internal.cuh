@@ -69,6 +69,19 @@ struct TilePart {
     int RMAX = 0;
     int n_tiles = 0;
     int2 *d_desc = nullptr;
+    struct WinDesc *d_win = nullptr;       // operand windows per tile (see ensure_windows)
+    int win_rows = -1;                     // WMAX the windows were built for (-1: not built)
+};
+
+// Operand window of a tile of a banded matrix: the tile's columns (and its own rows) lie in
+// nseg ranges of rows [a[s], a[s] + l[s]) of the gathered vectors, 4-row aligned; nseg = 0
+// means the tile gathers from global memory.
+constexpr int WSEG = 4;
+struct __align__(16) WinDesc {
+    int nseg;
+    int a[WSEG];
+    int l[WSEG];
+    int pad[16 - 1 - 2 * WSEG];
 };
 
 // Read-only view of a CSR matrix passed to kernels.
@@ -106,6 +119,7 @@ struct sla_csr {
     int64_t max_sys_nnz = 0;
     // host copy of row_ptr, for partition building
     std::vector<int32_t> h_rp;
+    std::vector<int32_t> h_ci;             // host copy of col (short-row matrices, for windows)
     std::map<int, sla::TilePart> tiles;    // by item budget D
     int device = 0;
     int num_sms = 148;
@@ -152,6 +166,8 @@ struct Plan {
 
 // ------------------------------------------------------------------ internal entry points
 sla_status ensure_tiles(sla_csr *A, int D, int RMAX, cudaStream_t s, const TilePart **out);
+// Build (once) the operand windows of a tile partition, at most wmax rows per tile.
+sla_status ensure_windows(sla_csr *A, const TilePart *tp, int wmax, cudaStream_t s);
 size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K, int vec64);
 sla_status get_plan(sla_csr *A, const sla_precond *M, int K, int vec64, Plan **out);
 void destroy_plan(Plan *p);
