@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--size", default="full", choices=["full", "small", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-reps", type=int, default=20)
+    ap.add_argument("--engine", default="auto", choices=["auto", "graph", "persistent"])
     return ap.parse_args()
 
 
@@ -155,7 +156,7 @@ def measured_peaks() -> tuple[float, str]:
         return 6650.0, "fallback"
 
 
-KERNEL_SOURCES = ("row_engine.cuh", "tile_engine.cuh", "pcg_impl.cuh")
+KERNEL_SOURCES = ("row_engine.cuh", "tile_engine.cuh", "pcg_ops.cuh", "persist.cuh", "pcg_impl.cuh")
 
 
 def kernel_source_hash() -> str:
@@ -289,25 +290,32 @@ def run_ours(args):
     multi = is_list or nrhs > 1
     body_kernels = 6 if w.precond == "spai" else 4       # two iterations per graph loop body
     prologue = 2 if w.precond == "spai" else 1
+    engines_seen = set()
 
-    def launches(iters: int) -> int:
-        """Kernels one solve launches: init, prologue, loop bodies (two iterations each), copy-out."""
+    def launches(iters: int, engine: str) -> int:
+        """Kernels one solve launches: init, the solve (persistent: one kernel; graph: prologue
+        and loop bodies of two iterations each), copy-out."""
+        if engine == "persistent":
+            return 3
         return 2 + prologue + body_kernels * ((iters + 1) // 2)
 
     def step(bv, wv, x_out):
         if multi:
-            x, inf = sla.sla_pcg_solve_batched(Ad, M, bv, x_out, rtol=w.tol)
-            lam, g, ainf = sla.sla_pcg_adjoint_batched(Ad, M, x, wv, rtol=w.tol)
+            x, inf = sla.sla_pcg_solve_batched(Ad, M, bv, x_out, rtol=w.tol, engine=args.engine)
+            lam, g, ainf = sla.sla_pcg_adjoint_batched(Ad, M, x, wv, rtol=w.tol, engine=args.engine)
+            engines_seen.update(i.engine for i in inf + ainf)
             if is_list:
                 return sum(i.iters for i in inf) + sum(i.iters for i in ainf), 2, x, lam
             it = max(i.iters for i in inf), max(i.iters for i in ainf)
             return (sum(i.iters for i in inf) + sum(i.iters for i in ainf),
-                    launches(it[0]) + launches(it[1]) + 1, x, lam)
-        x, inf = sla.sla_pcg_solve(Ad, M, bv, x_out, rtol=w.tol)
-        lam, g, ainf = sla.sla_pcg_adjoint(Ad, M, x, wv, rtol=w.tol)
+                    launches(it[0], inf[0].engine) + launches(it[1], ainf[0].engine) + 1, x, lam)
+        x, inf = sla.sla_pcg_solve(Ad, M, bv, x_out, rtol=w.tol, engine=args.engine)
+        lam, g, ainf = sla.sla_pcg_adjoint(Ad, M, x, wv, rtol=w.tol, engine=args.engine)
+        engines_seen.update((inf.engine, ainf.engine))
         if inf.status != 0 or ainf.status != 0:
             raise RuntimeError(f"solve did not converge: {inf} {ainf}")
-        return inf.iters + ainf.iters, launches(inf.iters) + launches(ainf.iters) + 1, x, lam
+        return (inf.iters + ainf.iters, launches(inf.iters, inf.engine) + launches(ainf.iters, ainf.engine) + 1,
+                x, lam)
 
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
@@ -391,7 +399,44 @@ def run_ours(args):
     roofline = None
     kernels = {}
     spmv = None
-    if not is_list:
+    if not is_list and engines_seen == {"persistent"}:
+        # the whole solve is one launch of the persistent kernel: time forward solves alone
+        # (L2 flushed before each; the launch brackets also hold the two small set-up and
+        # copy-out kernels) and take the algorithmic bytes of every phase the launch ran
+        kb = kernel_bytes(w)
+        names = list(kb)
+        reps = 3
+        tot = 0.0
+        for r in range(reps + 1):
+            flush.zero_()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record()
+            if multi:
+                sla.sla_pcg_solve_batched(Ad, M, b, X, rtol=w.tol, engine=args.engine)
+            else:
+                sla.sla_pcg_solve(Ad, M, b, X, rtol=w.tol, engine=args.engine)
+            s1.record()
+            torch.cuda.synchronize()
+            if r >= 1:
+                tot += s0.elapsed_time(s1)
+        launch_ms = tot / reps
+        pms, pcnt = sla.sla_pcg_phase_times(Ad, M, nrhs)
+        slot = {"q_spmv": 0, "update_gt_spmv": 1, "z_g_spmv": 2, "update_jacobi": 3}
+        launch_bytes = 0
+        for nm in names:
+            i = slot[nm]
+            launch_bytes += kb[nm] * pcnt[i]
+            kernels[nm] = {"ms": pms[i], "phases": pcnt[i], "bytes": kb[nm],
+                           "gbs": kb[nm] / (pms[i] * 1e6) if pms[i] > 0 else None,
+                           "timing": "in-kernel, grid barrier to grid barrier (block 0)"}
+        ach = launch_bytes / (launch_ms * 1e6)
+        roofline = {"bound": "hbm", "kernel": "k_pcg_persistent", "achieved": ach, "peak": peak, "unit": "GB/s",
+                    "frac": ach / peak, "traffic": profiled_traffic("k_pcg_persistent", w.name),
+                    "peak_source": peak_kind, "algorithmic_bytes": launch_bytes, "ms_per_launch": launch_ms,
+                    "units_per_launch": {nm: pcnt[slot[nm]] for nm in names},
+                    "note": "one launch = one forward solve; bytes = per-phase algorithmic bytes x phases run"}
+    elif not is_list:
         kt = sla.sla_pcg_kernel_times(Ad, M, nrhs, reps=args.kernel_reps)
         names = list(kernel_bytes(w))
         kb = kernel_bytes(w)
@@ -403,6 +448,7 @@ def run_ours(args):
         roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
                     "frac": ach / peak, "traffic": tr, "peak_source": peak_kind,
                     "algorithmic_bytes": kb[dom], "ms_per_launch": kernels[dom]["ms"]}
+    if not is_list:
         # standalone SpMV y = A x, L2 flushed before each launch
         xs = torch.randn(A.n_rows * nrhs, dtype=va.dtype, device=dev).reshape(b.shape)
         ys = torch.empty_like(xs)
@@ -443,7 +489,8 @@ def run_ours(args):
                        "iters_per_step": iters_per_step,
                        "step": "forward PCG solve + adjoint PCG solve + pattern gradient",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed between steps (512 MiB write)", "setup_s": setup_s},
+                       "l2": "flushed between steps (512 MiB write)", "setup_s": setup_s,
+                       "engine": "+".join(sorted(engines_seen))},
             "roofline": roofline, "spmv": spmv, "kernels": kernels,
             "gpu_launches": total_launch, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }

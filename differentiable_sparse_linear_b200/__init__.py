@@ -29,7 +29,8 @@ __all__ = [
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
     "sla_pcg_solve_batched_noalloc",
-    "sla_workspace_bytes", "sla_pcg_kernel_times", "solve",
+    "sla_workspace_bytes", "sla_pcg_kernel_times", "sla_pcg_phase_times", "solve",
+    "ENGINES",
 ]
 
 
@@ -76,11 +77,17 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise ValueError(f"values must be float32 or float64, got {dt}")
 
 
+# solve engines (SLA_ENGINE_*): "auto" takes the persistent engine where it applies
+ENGINES = {"auto": 0, "graph": 1, "persistent": 2}
+_ENGINE_NAMES = {0: "auto", 1: "graph", 2: "persistent", 3: "list"}
+
+
 @dataclass
 class PcgInfo:
     iters: int
     relres: float
     status: int
+    engine: str = "auto"
 
     @property
     def converged(self) -> bool:
@@ -88,14 +95,18 @@ class PcgInfo:
 
 
 def _infos(arr) -> list[PcgInfo]:
-    return [PcgInfo(int(a.iters), float(a.relres), int(a.status)) for a in arr]
+    return [PcgInfo(int(a.iters), float(a.relres), int(a.status), _ENGINE_NAMES.get(int(a.engine), "?"))
+            for a in arr]
 
 
-def _opts(rtol: float, maxit: int, vector_f64: bool = False) -> _lib.sla_pcg_opts:
+def _opts(rtol: float, maxit: int, vector_f64: bool = False, engine: str = "auto") -> _lib.sla_pcg_opts:
+    if engine not in ENGINES:
+        raise ValueError(f"engine must be one of {sorted(ENGINES)}, got {engine!r}")
     o = _lib.sla_pcg_opts()
     o.rtol = float(rtol)
     o.maxit = int(maxit)
     o.vector_f64 = 1 if vector_f64 else 0
+    o.engine = ENGINES[engine]
     return o
 
 
@@ -229,12 +240,12 @@ def sla_precond_spai(A: Matrix, G: Matrix, eps: float = 3e-3, stream=None) -> Pr
 
 def sla_pcg_solve(A: Matrix, M: Optional[Preconditioner], b: torch.Tensor,
                   x: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
-                  vector_f64: bool = False, stream=None) -> tuple[torch.Tensor, PcgInfo]:
+                  vector_f64: bool = False, engine: str = "auto", stream=None) -> tuple[torch.Tensor, PcgInfo]:
     """x = A^-1 b.  vector_f64 with an fp32 matrix: b and x are fp64 (mixed precision)."""
     _check_vec(A, b, vector_f64)
     x = torch.empty_like(b) if x is None else x
     info = _lib.sla_pcg_info()
-    opts = _opts(rtol, maxit, vector_f64)
+    opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_solve(A.handle, _mh(M), _ptr(b), _ptr(x), C.byref(opts), C.byref(info),
                                _stream(stream)), "sla_pcg_solve")
     return x, _infos([info])[0]
@@ -242,13 +253,13 @@ def sla_pcg_solve(A: Matrix, M: Optional[Preconditioner], b: torch.Tensor,
 
 def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLdx: torch.Tensor, *,
                     want_dA: bool = True, rtol: float = 0.0, maxit: int = 0, vector_f64: bool = False,
-                    stream=None):
+                    engine: str = "auto", stream=None):
     """Returns (dL/db, dL/dA on A's pattern or None, info)."""
     _check_vec(A, dLdx, vector_f64)
     dLdb = torch.empty_like(dLdx)
     dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdx.device) if want_dA else None
     info = _lib.sla_pcg_info()
-    opts = _opts(rtol, maxit, vector_f64)
+    opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_adjoint(A.handle, _mh(M), _ptr(x), _ptr(dLdx), _ptr(dLdb), _ptr(dLdA),
                                  C.byref(opts), C.byref(info), _stream(stream)), "sla_pcg_adjoint")
     return dLdb, dLdA, _infos([info])[0]
@@ -256,14 +267,14 @@ def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLd
 
 def sla_pcg_solve_batched(A: Matrix, M: Optional[Preconditioner], B: torch.Tensor,
                           X: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
-                          vector_f64: bool = False, stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
+                          vector_f64: bool = False, engine: str = "auto", stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
     """Shared matrix: B is [n, nrhs].  List handle: B is the concatenated [n_total] vector."""
     _check_vec(A, B, vector_f64)
     nrhs = 1 if (B.dim() == 1 or A.batch > 1) else B.shape[1]
     count = A.batch if A.batch > 1 else nrhs
     X = torch.empty_like(B) if X is None else X
     infos = (_lib.sla_pcg_info * count)()
-    opts = _opts(rtol, maxit, vector_f64)
+    opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_solve_batched(A.handle, _mh(M), nrhs, _ptr(B), _ptr(X), C.byref(opts),
                                        infos, _stream(stream)), "sla_pcg_solve_batched")
     return X, _infos(infos)
@@ -284,14 +295,14 @@ def sla_pcg_solve_batched_noalloc(A: Matrix, M: Optional[Preconditioner], B: tor
 
 def sla_pcg_adjoint_batched(A: Matrix, M: Optional[Preconditioner], X: torch.Tensor, dLdX: torch.Tensor,
                             *, want_dA: bool = True, rtol: float = 0.0, maxit: int = 0,
-                            vector_f64: bool = False, stream=None):
+                            vector_f64: bool = False, engine: str = "auto", stream=None):
     _check_vec(A, dLdX, vector_f64)
     nrhs = 1 if (dLdX.dim() == 1 or A.batch > 1) else dLdX.shape[1]
     count = A.batch if A.batch > 1 else nrhs
     dLdB = torch.empty_like(dLdX)
     dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdX.device) if want_dA else None
     infos = (_lib.sla_pcg_info * count)()
-    opts = _opts(rtol, maxit, vector_f64)
+    opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_adjoint_batched(A.handle, _mh(M), nrhs, _ptr(X), _ptr(dLdX), _ptr(dLdB),
                                          _ptr(dLdA), C.byref(opts), infos, _stream(stream)),
            "sla_pcg_adjoint_batched")
@@ -314,6 +325,17 @@ def sla_pcg_kernel_times(A: Matrix, M: Optional[Preconditioner] = None, nrhs: in
     _check(lib().sla_pcg_kernel_times(A.handle, _mh(M), nrhs, 1 if vector_f64 else 0, reps, out,
                                       _stream(stream)), "sla_pcg_kernel_times")
     return list(out)
+
+
+def sla_pcg_phase_times(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1,
+                        vector_f64: bool = False, stream=None) -> tuple[list[float], list[int]]:
+    """In-kernel mean ms per phase of the last persistent-engine solve, and phase counts:
+    [q = A p, x/r update + y = G^T r, z = G y + eps r, x/r update + z = D^-1 r]."""
+    ms = (C.c_double * 4)()
+    cnt = (C.c_int64 * 4)()
+    _check(lib().sla_pcg_phase_times(A.handle, _mh(M), nrhs, 1 if vector_f64 else 0, ms, cnt,
+                                     _stream(stream)), "sla_pcg_phase_times")
+    return list(ms), [int(c) for c in cnt]
 
 
 def sla_workspace_bytes(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1,

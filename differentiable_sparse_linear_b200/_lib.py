@@ -19,16 +19,20 @@ SLA_F32 = 0
 SLA_F64 = 1
 SLA_SPD = 1
 SLA_VALIDATE = 2
+SLA_ENGINE_AUTO = 0
+SLA_ENGINE_GRAPH = 1
+SLA_ENGINE_PERSISTENT = 2
+SLA_ENGINE_LIST = 3
 
 
 class sla_pcg_opts(C.Structure):
     _fields_ = [("rtol", C.c_double), ("maxit", C.c_int64), ("vector_f64", C.c_int32),
-                ("reserved", C.c_int32)]
+                ("engine", C.c_int32)]
 
 
 class sla_pcg_info(C.Structure):
     _fields_ = [("iters", C.c_int64), ("relres", C.c_double), ("status", C.c_int32),
-                ("reserved", C.c_int32)]
+                ("engine", C.c_int32)]
 
 
 _vp = C.c_void_p
@@ -62,6 +66,8 @@ SIGNATURES = {
     "sla_pcg_solve_batched_noalloc": (_st, [_vp, _vp, _vp, _vp, C.POINTER(sla_pcg_opts),
                                             C.POINTER(sla_pcg_info), _vp]),
     "sla_pcg_kernel_times": (_st, [_vp, _vp, C.c_int32, C.c_int32, C.c_int32, C.POINTER(C.c_double), _vp]),
+    "sla_pcg_phase_times": (_st, [_vp, _vp, C.c_int32, C.c_int32, C.POINTER(C.c_double),
+                                  C.POINTER(C.c_int64), _vp]),
     "sla_workspace_bytes": (C.c_size_t, [_vp, _vp, C.c_int32, C.c_int32]),
 }
 

@@ -848,6 +848,33 @@ sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t 
     return kernel_times(const_cast<sla_csr *>(A), p, nrhs, reps, h_ms, (cudaStream_t)stream);
 }
 
+sla_status sla_pcg_phase_times(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                               int32_t vector_f64, double *h_ms, int64_t *h_count, void *stream)
+{
+    SLA_TRY(check_solve(A, M));
+    if (!h_ms || !h_count)
+        return fail(SLA_ERR_INVALID_ARG, "h_ms and h_count are required");
+    if (A->batch > 1)
+        return fail(SLA_ERR_UNSUPPORTED, "phase timing covers the single-matrix solver");
+    if (nrhs < 1 || nrhs > KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    int K = 1;
+    while (K < nrhs)
+        K <<= 1;
+    Plan *p = nullptr;
+    SLA_TRY(get_plan(const_cast<sla_csr *>(A), M, K, vector_f64, &p));
+    cudaStream_t s = (cudaStream_t)stream;
+    SLA_CUDA_TRY(cudaMemcpyAsync(p->h_st, p->st, sizeof(PcgState), cudaMemcpyDeviceToHost, s));
+    SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    if (!p->h_st->persistent)
+        return fail(SLA_ERR_INVALID_ARG, "the last solve of this solver did not run on the persistent engine");
+    for (int i = 0; i < 4; ++i) {
+        h_count[i] = p->h_st->phase_cnt[i];
+        h_ms[i] = h_count[i] > 0 ? 1e-6 * (double)p->h_st->phase_ns[i] / (double)h_count[i] : 0.0;
+    }
+    return SLA_SUCCESS;
+}
+
 size_t sla_workspace_bytes(const sla_csr *A, const sla_precond *M, int32_t nrhs, int32_t vector_f64)
 {
     if (!A || nrhs < 1 || nrhs > KMAX)

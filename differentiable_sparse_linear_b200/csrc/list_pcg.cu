@@ -179,7 +179,7 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
             info[s].iters = it;
             info[s].relres = relres;
             info[s].status = status;
-            info[s].reserved = 0;
+            info[s].engine = SLA_ENGINE_LIST;
         }
         __syncthreads();
     }

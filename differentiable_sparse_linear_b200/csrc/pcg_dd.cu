@@ -21,9 +21,9 @@ sla_status times_dd(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaS
 }
 
 sla_status run_dd(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol, long long maxit,
-                      cudaStream_t s)
+                      int engine, cudaStream_t s)
 {
-    SLA_DISPATCH_K(p->K, run_k, A, p, nrhs, B, X, tol, maxit, s)
+    SLA_DISPATCH_K(p->K, run_k, A, p, nrhs, B, X, tol, maxit, engine, s)
 }
 
 sla_status grad_dd(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g, cudaStream_t s)

@@ -169,13 +169,16 @@ sla_status run_plan(sla_csr *A, Plan *p, int nrhs, const void *B, void *X,
     double tol = (opts && opts->rtol > 0) ? opts->rtol : (f64 ? 1e-10 : 1e-6);
     long long n_sys = A->batch > 1 ? A->max_sys_n : A->n;
     long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 10 * std::max<long long>(n_sys, 1);
+    const int engine = opts ? opts->engine : SLA_ENGINE_AUTO;
+    if (engine < SLA_ENGINE_AUTO || engine > SLA_ENGINE_PERSISTENT)
+        return fail(SLA_ERR_INVALID_ARG, "unknown solve engine");
     sla_status st;
     if (A->dtype == SLA_F64)
-        st = run_dd(A, p, nrhs, B, X, tol, maxit, s);
+        st = run_dd(A, p, nrhs, B, X, tol, maxit, engine, s);
     else if (p->vec64)
-        st = run_fd(A, p, nrhs, B, X, tol, maxit, s);
+        st = run_fd(A, p, nrhs, B, X, tol, maxit, engine, s);
     else
-        st = run_ff(A, p, nrhs, B, X, tol, maxit, s);
+        st = run_ff(A, p, nrhs, B, X, tol, maxit, engine, s);
     if (st != SLA_SUCCESS)
         return st;
     if (grad_out)
@@ -190,7 +193,7 @@ sla_status run_plan(sla_csr *A, Plan *p, int nrhs, const void *B, void *X,
             info[c].iters = p->h_st->iters[c];
             info[c].relres = p->h_st->relres[c];
             info[c].status = p->h_st->status[c];
-            info[c].reserved = 0;
+            info[c].engine = p->h_st->persistent ? SLA_ENGINE_PERSISTENT : SLA_ENGINE_GRAPH;
         }
         worst = std::max(worst, (sla_status)p->h_st->status[c]);
     }

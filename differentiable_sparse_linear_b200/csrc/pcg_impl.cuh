@@ -10,280 +10,12 @@
 #include <cstring>
 
 #include "sla_internal.cuh"
+#include "pcg_ops.cuh"
+#include "persist.cuh"
 #include "row_engine.cuh"
 #include "tile_engine.cuh"
 
 namespace sla {
-
-// ------------------------------------------------------------------ scalar finalisation
-static __device__ __forceinline__ bool finite_d(double a) { return isfinite(a); }
-
-static __device__ __noinline__ void signal_if_done(PcgState *st)
-{
-    int any = 0;
-    for (int c = 0; c < st->k; ++c)
-        any |= st->active[c];
-    if (!any) {
-        st->all_done = 1;
-        if (st->has_cond)
-            cudaGraphSetConditional((cudaGraphConditionalHandle)st->cond_handle, 0u);
-    }
-}
-
-// After q = A p: alpha = rho / (p.q); p.q <= 0 or non-finite is a breakdown.
-static __device__ __noinline__ void finalize_alpha(PcgState *st, const double *pq)
-{
-    if (st->profile)
-        return;
-    for (int c = 0; c < st->k; ++c) {
-        if (!st->active[c])
-            continue;
-        const double d = pq[c];
-        if (!(d > 0.0) || !finite_d(d)) {
-            st->status[c] = SLA_BREAKDOWN;
-            st->active[c] = 0;
-        } else {
-            st->alpha[c] = st->rho[c] / d;
-        }
-    }
-    signal_if_done(st);
-}
-
-// After the x/r update: stopping test on ||r||/||b|| (initial pass: record ||b||).
-static __device__ __noinline__ void finalize_residual(PcgState *st, const double *rr)
-{
-    if (st->profile)
-        return;
-    for (int c = 0; c < st->k; ++c) {
-        if (!st->active[c])
-            continue;
-        if (st->phase0) {
-            const double bn = sqrt(rr[c]);
-            st->bnorm[c] = bn;
-            st->relres[c] = bn > 0.0 ? 1.0 : 0.0;
-            if (!finite_d(bn)) {
-                st->status[c] = SLA_BREAKDOWN;
-                st->active[c] = 0;
-            } else if (bn == 0.0) {
-                st->status[c] = SLA_SUCCESS;
-                st->active[c] = 0;
-            }
-        } else {
-            st->iters[c] += 1;
-            const double rel = sqrt(rr[c]) / st->bnorm[c];
-            st->relres[c] = rel;
-            if (!finite_d(rel)) {
-                st->status[c] = SLA_BREAKDOWN;
-                st->active[c] = 0;
-            } else if (rel <= st->tol) {
-                st->status[c] = SLA_SUCCESS;
-                st->active[c] = 0;
-            } else if (st->iters[c] >= st->maxit) {
-                st->status[c] = SLA_NOT_CONVERGED;
-                st->active[c] = 0;
-            }
-        }
-    }
-}
-
-// After z = M^-1 r: rho' = r.z, beta = rho'/rho (0 on the initial pass).
-static __device__ __noinline__ void finalize_beta(PcgState *st, const double *rz)
-{
-    if (st->profile)
-        return;
-    for (int c = 0; c < st->k; ++c) {
-        if (!st->active[c])
-            continue;
-        const double v = rz[c];
-        if (!(v > 0.0) || !finite_d(v)) {
-            st->status[c] = SLA_BREAKDOWN;
-            st->active[c] = 0;
-            continue;
-        }
-        st->beta[c] = st->phase0 ? 0.0 : v / st->rho[c];
-        st->rho[c] = v;
-    }
-    st->phase0 = 0;
-    signal_if_done(st);
-}
-
-// ------------------------------------------------------------------ operations
-// y = A x for K right-hand sides with leading dimension ld (columns c >= nc are zero).
-template <typename V, int K>
-struct OpSpmv {
-    using VV = V;
-    static constexpr int NP = 0, NS = 0, NV = 0;
-    static constexpr int NG = 1;
-    const V *x;
-    V *y;
-    int ld, nc;
-    __device__ const V *row_vec(int) const { return nullptr; }
-    __host__ __device__ const V *gvec(int) const { return x; }
-    __host__ __device__ int gstride() const { return ld; }
-    static __device__ constexpr int rv_src(int) { return -1; }
-    __device__ bool skip() const { return false; }
-    __device__ void stage(double *) const {}
-    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *) const
-    {
-        return c < nc ? g[0] : (V)0;
-    }
-    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
-    {
-        return c < nc ? __ldg(&x[j * ld + c]) : (V)0;
-    }
-    template <int N, class RV>
-    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N], const double *,
-                                         const RV &) const
-    {
-#pragma unroll
-        for (int c = 0; c < K; ++c)
-            if (c < nc)
-                y[i * ld + c] = (V)acc[c];
-    }
-    __device__ void finalize(const double *) const {}
-};
-
-// Q: p_new = z + beta p_old, q = A p_new, partial p_new.q
-template <typename V, int K>
-struct OpQ {
-    using VV = V;
-    static constexpr int NP = 1, NS = K, NV = 2;
-    const V *z;
-    const V *p_old;
-    V *p_new;
-    V *q;
-    PcgState *st;
-    static constexpr int NG = 2;
-    __device__ const V *row_vec(int v) const { return v == 0 ? p_old : z; }
-    __host__ __device__ const V *gvec(int g) const { return g == 0 ? p_old : z; }
-    __host__ __device__ int gstride() const { return K; }
-    static __device__ constexpr int rv_src(int v) { return v; }
-    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
-    __device__ void stage(double *s) const
-    {
-        for (int c = 0; c < K; ++c)
-            s[c] = st->beta[c];
-    }
-    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *s) const
-    {
-        return (V)__fma_rn(s[c], (double)g[0], (double)g[1]);
-    }
-    __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
-    {
-        return (V)__fma_rn(s[c], (double)p_old[j * K + c], (double)z[j * K + c]);
-    }
-    template <int N, class RV>
-    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s, const RV &rv) const
-    {
-#pragma unroll
-        for (int c = 0; c < K; ++c) {
-            const V pn = (V)__fma_rn(s[c], (double)rv.get(0, i, c), (double)rv.get(1, i, c));
-            const V qv = (V)acc[c];
-            p_new[i * K + c] = pn;
-            q[i * K + c] = qv;
-            part[c] += (double)pn * (double)qv;
-        }
-    }
-    __device__ void finalize(const double *sums) const { finalize_alpha(st, sums); }
-};
-
-// U_S: r_new = r_old - alpha q, x += alpha p, y = G^T r_new, partial r_new.r_new
-template <typename V, int K>
-struct OpUS {
-    using VV = V;
-    static constexpr int NP = 1, NS = 2 * K, NV = 4;
-    const V *r_old;
-    const V *q;
-    const V *p;
-    const V *x_in;
-    V *r_new;
-    V *x;
-    V *y;
-    PcgState *st;
-    static constexpr int NG = 2;
-    __device__ const V *row_vec(int v) const { return v == 0 ? r_old : v == 1 ? q : v == 2 ? p : x_in; }
-    __host__ __device__ const V *gvec(int g) const { return g == 0 ? r_old : q; }
-    __host__ __device__ int gstride() const { return K; }
-    static __device__ constexpr int rv_src(int v) { return v < 2 ? v : -1; }
-    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
-    __device__ void stage(double *s) const
-    {
-        for (int c = 0; c < K; ++c) {
-            s[c] = st->alpha[c];
-            s[K + c] = st->active[c] ? 1.0 : 0.0;
-        }
-    }
-    __device__ __forceinline__ V rnew(V ro, V qv, int c, const double *s) const
-    {
-        return s[K + c] != 0.0 ? (V)__fma_rn(-s[c], (double)qv, (double)ro) : ro;
-    }
-    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *s) const
-    {
-        return rnew(g[0], g[1], c, s);
-    }
-    __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
-    {
-        return rnew(r_old[j * K + c], q[j * K + c], c, s);
-    }
-    template <int N, class RV>
-    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s, const RV &rv) const
-    {
-#pragma unroll
-        for (int c = 0; c < K; ++c) {
-            const V rn = rnew(rv.get(0, i, c), rv.get(1, i, c), c, s);
-            r_new[i * K + c] = rn;
-            if (s[K + c] != 0.0)
-                x[i * K + c] = (V)__fma_rn(s[c], (double)rv.get(2, i, c), (double)rv.get(3, i, c));
-            y[i * K + c] = (V)acc[c];
-            part[c] += (double)rn * (double)rn;
-        }
-    }
-    __device__ void finalize(const double *sums) const
-    {
-        if (st->profile)
-            return;
-        finalize_residual(st, sums);
-        signal_if_done(st);
-    }
-};
-
-// Z: z = G y + eps r, partial r.z
-template <typename V, int K>
-struct OpZ {
-    using VV = V;
-    static constexpr int NP = 1, NS = 1, NV = 1;
-    const V *y;
-    const V *r;
-    V *z;
-    PcgState *st;
-    static constexpr int NG = 1;
-    __device__ const V *row_vec(int) const { return r; }
-    __host__ __device__ const V *gvec(int) const { return y; }
-    __host__ __device__ int gstride() const { return K; }
-    static __device__ constexpr int rv_src(int) { return -1; }
-    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
-    __device__ void stage(double *s) const { s[0] = st->eps; }
-    __device__ __forceinline__ V combine(const V (&g)[NG], int, const double *) const { return g[0]; }
-    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
-    {
-        return y[j * K + c];
-    }
-    template <int N, class RV>
-    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
-                                         const double *s, const RV &rv) const
-    {
-#pragma unroll
-        for (int c = 0; c < K; ++c) {
-            const double rv_ = (double)rv.get(0, i, c);
-            const V zv = (V)__fma_rn(s[0], rv_, acc[c]);
-            z[i * K + c] = zv;
-            part[c] += rv_ * (double)zv;
-        }
-    }
-    __device__ void finalize(const double *sums) const { finalize_beta(st, sums); }
-};
 
 // ------------------------------------------------------------------ elementwise kernels
 constexpr int VEC_T = 256;
@@ -329,8 +61,8 @@ k_update_jacobi(int64_t n, V *x, V *r, const V *p, const V *q, V *z, const V *di
             const int64_t e = i * K + c;
             double rv = (double)r[e];
             if (s_on[c] != 0.0) {
-                x[e] = (V)__fma_rn(s_a[c], (double)p[e], (double)x[e]);
-                const V rn = (V)__fma_rn(-s_a[c], (double)q[e], rv);
+                x[e] = vfma<V>(s_a[c], p[e], x[e]);
+                const V rn = vfma<V>(-s_a[c], q[e], r[e]);
                 r[e] = rn;
                 rv = (double)rn;
             }
@@ -385,6 +117,12 @@ __global__ void k_init(int64_t n, int nrhs, const V *B, V *x, V *r, V *p, V *q, 
         st->has_cond = has_cond;
         st->profile = 0;
         st->error = 0;
+        st->persistent = 0;
+        st->gbar = 0ull;
+        for (int i = 0; i < 4; ++i) {
+            st->phase_ns[i] = 0ull;
+            st->phase_cnt[i] = 0;
+        }
     }
 }
 
@@ -795,10 +533,103 @@ static sla_status times_k(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms,
     return st;
 }
 
+// ------------------------------------------------------------------ persistent engine
+// Row-length bound (the kernel's MAXL) the persistent engine uses for this plan, 0 when it
+// does not apply: single systems whose matrices (A; with SPAI also G and G^T) have rows of
+// at most 8 entries (16 with K <= 2), K <= 8, cooperative launch available.
+// Instantiated combinations: those whose consumer code fits the register budget (fp64
+// vectors: K <= 4 and rows of at most 8 entries).
+template <typename VV, int K, int MAXL>
+constexpr bool persist_compiled()
+{
+    return K <= 8 && (MAXL == 8 || K <= 2) && (sizeof(VV) == 4 || (K <= 4 && MAXL == 8));
+}
+
+template <typename VV, int K>
+static int persist_maxl(const sla_csr *A, const Plan *p)
+{
+    if (K > 8 || A->batch > 1 || A->n == 0 || A->nnz == 0)
+        return 0;
+    int64_t L = A->max_row_len;
+    if (p->kind == 2) {
+        if (p->M->G->nnz == 0)
+            return 0;
+        L = std::max(L, std::max(p->M->G->max_row_len, p->M->GT->max_row_len));
+    }
+    int coop = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, A->device) != cudaSuccess || !coop)
+        return 0;
+    if (L <= 8)
+        return persist_compiled<VV, K, 8>() ? 8 : 0;
+    if (L <= 16)
+        return persist_compiled<VV, K, 16>() ? 16 : 0;
+    return 0;
+}
+
+template <typename VM, typename VV, int K, int MAXL>
+static sla_status persist_launch(sla_csr *A, Plan *p, cudaStream_t s)
+{
+    using Pk = Persist<VM, VV, K, MAXL>;
+    constexpr int THREADS = Pk::TC + 32;
+    auto kern = k_pcg_persistent<VM, VV, K, MAXL>;
+    PersistArgs<VM, VV> a{};
+    auto mat = [&](const sla_csr *M_, MatView<VM> &mv, const WinDesc *&w) -> sla_status {
+        const TilePart *tp;
+        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(M_), RowTmaCfg<K>::D,
+                             RowTmaCfg<K>::TC * RowTmaCfg<K>::RPT, s, &tp));
+        mv = view<VM>(M_, tp);
+        w = nullptr;
+        if (RowTmaCfg<K>::WMAX > 0) {
+            SLA_TRY(ensure_windows(const_cast<sla_csr *>(M_), tp, RowTmaCfg<K>::WMAX, s));
+            w = tp->d_win;   // workspace vectors are 256-byte aligned, as window copies need
+        }
+        return SLA_SUCCESS;
+    };
+    SLA_TRY(mat(A, a.A, a.winA));
+    a.spai = p->kind == 2 ? 1 : 0;
+    if (a.spai) {
+        SLA_TRY(mat(p->M->G, a.G, a.winG));
+        SLA_TRY(mat(p->M->GT, a.GT, a.winGT));
+    }
+    a.x = (VV *)p->x; a.ra = (VV *)p->ra; a.rb = (VV *)p->rb; a.pa = (VV *)p->pa; a.pb = (VV *)p->pb;
+    a.q = (VV *)p->q; a.z = (VV *)p->z; a.y = (VV *)p->y;
+    if (p->kind == 1)
+        a.dinv = (const VV *)(sizeof(VV) == 8 ? p->M->d_dinv64 : p->M->d_dinv);
+    else if (p->kind == 0)
+        a.dinv = (const VV *)p->y;   // ones (y is unused without SPAI)
+    a.st = p->st;
+    a.partials = p->partials;
+    a.err = &p->st->error;
+    if (p->persist_grid == 0) {
+        SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Pk::SMEM));
+        int per_sm = 0;
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, Pk::SMEM));
+        if (per_sm < 1)
+            return fail(SLA_ERR_UNSUPPORTED, "persistent solver kernel does not fit on an SM");
+        // every block must be resident at once (cooperative launch); the partials buffer
+        // holds 2 slots of 2K doubles per block.  No more blocks than the largest phase
+        // has work units (tiles, or TC-row chunks for the elementwise phase): every block
+        // arrives at every grid barrier, so idle blocks only add to the barrier's cost.
+        const int cap = (int)(((size_t)A->num_sms * 32 * 2 * KMAX) / (2 * 2 * K));
+        int64_t units = (A->n + Pk::TC - 1) / Pk::TC;
+        units = std::max<int64_t>(units, a.A.n_tiles);
+        if (a.spai)
+            units = std::max<int64_t>(units, std::max(a.G.n_tiles, a.GT.n_tiles));
+        p->persist_grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, std::min(per_sm * A->num_sms, cap)));
+    }
+    void *args[] = {(void *)&a};
+    SLA_CUDA_TRY(cudaLaunchCooperativeKernel((const void *)kern, dim3(p->persist_grid), dim3(THREADS), args,
+                                             Pk::SMEM, s));
+    return SLA_SUCCESS;
+}
+
 template <typename VM, typename VV, int K>
 static sla_status run_k(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,
-                        long long maxit, cudaStream_t s)
+                        long long maxit, int engine, cudaStream_t s)
 {
+    const int maxl = engine == SLA_ENGINE_GRAPH ? 0 : persist_maxl<VV, K>(A, p);
+    if (engine == SLA_ENGINE_PERSISTENT && maxl == 0)
+        return fail(SLA_ERR_INVALID_ARG, "the persistent engine does not apply to this system");
     const int64_t n = A->n;
     const int gv = vec_grid(A);
     VV *y = (VV *)p->y;
@@ -811,7 +642,15 @@ static sla_status run_k(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, d
                                      (VV *)p->q, (VV *)p->z, p->kind == 2 ? y : nullptr, p->st, tol,
                                      maxit, p->M ? p->M->eps : 0.0, p->cond, 1);
     SLA_CUDA_TRY(cudaGetLastError());
-    SLA_CUDA_TRY(cudaGraphLaunch(p->exec, s));
+    if (maxl == 8) {
+        if constexpr (persist_compiled<VV, K, 8>())
+            SLA_TRY((persist_launch<VM, VV, K, 8>(A, p, s)));
+    } else if (maxl == 16) {
+        if constexpr (persist_compiled<VV, K, 16>())
+            SLA_TRY((persist_launch<VM, VV, K, 16>(A, p, s)));
+    } else {
+        SLA_CUDA_TRY(cudaGraphLaunch(p->exec, s));
+    }
     k_copy_out<VV, K><<<gv, 256, 0, s>>>(n, nrhs, (const VV *)p->x, (VV *)X);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;

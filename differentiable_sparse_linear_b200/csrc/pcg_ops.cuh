@@ -1,0 +1,300 @@
+// Scalar finalisation of the PCG recurrence and the fused operations (row epilogues) the
+// SpMV engines run: Q (p update, q = A p, p.q), U_S (x/r update, y = G^T r, r.r), Z
+// (z = G y + eps r, r.z) and the plain SpMV.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "sla_internal.cuh"
+
+namespace sla {
+
+// ------------------------------------------------------------------ scalar finalisation
+static __device__ __forceinline__ bool finite_d(double a) { return isfinite(a); }
+
+static __device__ __noinline__ void signal_if_done(PcgState *st)
+{
+    int any = 0;
+    for (int c = 0; c < st->k; ++c)
+        any |= st->active[c];
+    if (!any) {
+        st->all_done = 1;
+        if (st->has_cond)
+            cudaGraphSetConditional((cudaGraphConditionalHandle)st->cond_handle, 0u);
+    }
+}
+
+// After q = A p: alpha = rho / (p.q); p.q <= 0 or non-finite is a breakdown.
+static __device__ __noinline__ void finalize_alpha(PcgState *st, const double *pq)
+{
+    if (st->profile)
+        return;
+    for (int c = 0; c < st->k; ++c) {
+        if (!st->active[c])
+            continue;
+        const double d = pq[c];
+        if (!(d > 0.0) || !finite_d(d)) {
+            st->status[c] = SLA_BREAKDOWN;
+            st->active[c] = 0;
+        } else {
+            st->alpha[c] = st->rho[c] / d;
+        }
+    }
+    signal_if_done(st);
+}
+
+// After the x/r update: stopping test on ||r||/||b|| (initial pass: record ||b||).
+static __device__ __noinline__ void finalize_residual(PcgState *st, const double *rr)
+{
+    if (st->profile)
+        return;
+    for (int c = 0; c < st->k; ++c) {
+        if (!st->active[c])
+            continue;
+        if (st->phase0) {
+            const double bn = sqrt(rr[c]);
+            st->bnorm[c] = bn;
+            st->relres[c] = bn > 0.0 ? 1.0 : 0.0;
+            if (!finite_d(bn)) {
+                st->status[c] = SLA_BREAKDOWN;
+                st->active[c] = 0;
+            } else if (bn == 0.0) {
+                st->status[c] = SLA_SUCCESS;
+                st->active[c] = 0;
+            }
+        } else {
+            st->iters[c] += 1;
+            const double rel = sqrt(rr[c]) / st->bnorm[c];
+            st->relres[c] = rel;
+            if (!finite_d(rel)) {
+                st->status[c] = SLA_BREAKDOWN;
+                st->active[c] = 0;
+            } else if (rel <= st->tol) {
+                st->status[c] = SLA_SUCCESS;
+                st->active[c] = 0;
+            } else if (st->iters[c] >= st->maxit) {
+                st->status[c] = SLA_NOT_CONVERGED;
+                st->active[c] = 0;
+            }
+        }
+    }
+}
+
+// After z = M^-1 r: rho' = r.z, beta = rho'/rho (0 on the initial pass).
+static __device__ __noinline__ void finalize_beta(PcgState *st, const double *rz)
+{
+    if (st->profile)
+        return;
+    for (int c = 0; c < st->k; ++c) {
+        if (!st->active[c])
+            continue;
+        const double v = rz[c];
+        if (!(v > 0.0) || !finite_d(v)) {
+            st->status[c] = SLA_BREAKDOWN;
+            st->active[c] = 0;
+            continue;
+        }
+        st->beta[c] = st->phase0 ? 0.0 : v / st->rho[c];
+        st->rho[c] = v;
+    }
+    st->phase0 = 0;
+    signal_if_done(st);
+}
+
+// ------------------------------------------------------------------ operations
+// a*b + c for vector elements: in fp32 (a rounded once) for fp32 vectors, fp64 otherwise.
+// Every place that forms the same vector value uses it with the same operands, so values
+// recomputed from gathered operands equal the stored ones bit for bit.
+template <typename V>
+__device__ __forceinline__ V vfma(double a, V b, V c);
+template <>
+__device__ __forceinline__ float vfma<float>(double a, float b, float c)
+{
+    return __fmaf_rn((float)a, b, c);
+}
+template <>
+__device__ __forceinline__ double vfma<double>(double a, double b, double c)
+{
+    return __fma_rn(a, b, c);
+}
+
+// y = A x for K right-hand sides with leading dimension ld (columns c >= nc are zero).
+template <typename V, int K>
+struct OpSpmv {
+    using VV = V;
+    static constexpr int NP = 0, NS = 0, NV = 0;
+    static constexpr int NG = 1;
+    const V *x;
+    V *y;
+    int ld, nc;
+    __device__ const V *row_vec(int) const { return nullptr; }
+    __host__ __device__ const V *gvec(int) const { return x; }
+    __host__ __device__ int gstride() const { return ld; }
+    static __device__ constexpr int rv_src(int) { return -1; }
+    __device__ bool skip() const { return false; }
+    __device__ void stage(double *) const {}
+    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *) const
+    {
+        return c < nc ? g[0] : (V)0;
+    }
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
+    {
+        return c < nc ? __ldg(&x[j * ld + c]) : (V)0;
+    }
+    template <int N, class RV>
+    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N], const double *,
+                                         const RV &) const
+    {
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            if (c < nc)
+                y[i * ld + c] = (V)acc[c];
+    }
+    __device__ void finalize(const double *) const {}
+};
+
+// Q: p_new = z + beta p_old, q = A p_new, partial p_new.q
+template <typename V, int K>
+struct OpQ {
+    using VV = V;
+    static constexpr int NP = 1, NS = K, NV = 2;
+    const V *z;
+    const V *p_old;
+    V *p_new;
+    V *q;
+    PcgState *st;
+    static constexpr int NG = 2;
+    __device__ const V *row_vec(int v) const { return v == 0 ? p_old : z; }
+    __host__ __device__ const V *gvec(int g) const { return g == 0 ? p_old : z; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int v) { return v; }
+    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
+    __device__ void stage(double *s) const
+    {
+        for (int c = 0; c < K; ++c)
+            s[c] = st->beta[c];
+    }
+    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *s) const
+    {
+        return vfma<V>(s[c], g[0], g[1]);
+    }
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
+    {
+        return vfma<V>(s[c], p_old[j * K + c], z[j * K + c]);
+    }
+    template <int N, class RV>
+    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
+                                         const double *s, const RV &rv) const
+    {
+#pragma unroll
+        for (int c = 0; c < K; ++c) {
+            const V pn = vfma<V>(s[c], rv.get(0, i, c), rv.get(1, i, c));
+            const V qv = (V)acc[c];
+            p_new[i * K + c] = pn;
+            q[i * K + c] = qv;
+            part[c] += (double)pn * (double)qv;
+        }
+    }
+    __device__ void finalize(const double *sums) const { finalize_alpha(st, sums); }
+};
+
+// U_S: r_new = r_old - alpha q, x += alpha p, y = G^T r_new, partial r_new.r_new
+template <typename V, int K>
+struct OpUS {
+    using VV = V;
+    static constexpr int NP = 1, NS = 2 * K, NV = 4;
+    const V *r_old;
+    const V *q;
+    const V *p;
+    const V *x_in;
+    V *r_new;
+    V *x;
+    V *y;
+    PcgState *st;
+    static constexpr int NG = 2;
+    __device__ const V *row_vec(int v) const { return v == 0 ? r_old : v == 1 ? q : v == 2 ? p : x_in; }
+    __host__ __device__ const V *gvec(int g) const { return g == 0 ? r_old : q; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int v) { return v < 2 ? v : -1; }
+    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
+    __device__ void stage(double *s) const
+    {
+        for (int c = 0; c < K; ++c) {
+            s[c] = st->alpha[c];
+            s[K + c] = st->active[c] ? 1.0 : 0.0;
+        }
+    }
+    __device__ __forceinline__ V rnew(V ro, V qv, int c, const double *s) const
+    {
+        return s[K + c] != 0.0 ? vfma<V>(-s[c], qv, ro) : ro;
+    }
+    __device__ __forceinline__ V combine(const V (&g)[NG], int c, const double *s) const
+    {
+        return rnew(g[0], g[1], c, s);
+    }
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *s) const
+    {
+        return rnew(r_old[j * K + c], q[j * K + c], c, s);
+    }
+    template <int N, class RV>
+    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
+                                         const double *s, const RV &rv) const
+    {
+#pragma unroll
+        for (int c = 0; c < K; ++c) {
+            const V rn = rnew(rv.get(0, i, c), rv.get(1, i, c), c, s);
+            r_new[i * K + c] = rn;
+            if (s[K + c] != 0.0)
+                x[i * K + c] = vfma<V>(s[c], rv.get(2, i, c), rv.get(3, i, c));
+            y[i * K + c] = (V)acc[c];
+            part[c] += (double)rn * (double)rn;
+        }
+    }
+    __device__ void finalize(const double *sums) const
+    {
+        if (st->profile)
+            return;
+        finalize_residual(st, sums);
+        signal_if_done(st);
+    }
+};
+
+// Z: z = G y + eps r, partial r.z
+template <typename V, int K>
+struct OpZ {
+    using VV = V;
+    static constexpr int NP = 1, NS = 1, NV = 1;
+    const V *y;
+    const V *r;
+    V *z;
+    PcgState *st;
+    static constexpr int NG = 1;
+    __device__ const V *row_vec(int) const { return r; }
+    __host__ __device__ const V *gvec(int) const { return y; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int) { return -1; }
+    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
+    __device__ void stage(double *s) const { s[0] = st->eps; }
+    __device__ __forceinline__ V combine(const V (&g)[NG], int, const double *) const { return g[0]; }
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const
+    {
+        return y[j * K + c];
+    }
+    template <int N, class RV>
+    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
+                                         const double *s, const RV &rv) const
+    {
+#pragma unroll
+        for (int c = 0; c < K; ++c) {
+            const V rv_ = rv.get(0, i, c);
+            const V zv = vfma<V>(s[0], rv_, (V)acc[c]);
+            z[i * K + c] = zv;
+            part[c] += (double)rv_ * (double)zv;
+        }
+    }
+    __device__ void finalize(const double *sums) const { finalize_beta(st, sums); }
+};
+
+}  // namespace sla

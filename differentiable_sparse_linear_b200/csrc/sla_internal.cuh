@@ -57,6 +57,10 @@ struct PcgState {
     int profile;            // 1: kernels run for timing only; finalisation is skipped
     int error;              // nonzero: a pipeline wait ran out of time (results invalid)
     int vec64;              // vectors are fp64 (matrix may be fp32)
+    int persistent;         // 1: the last solve ran in the persistent kernel
+    unsigned long long gbar;            // grid-barrier arrivals of the persistent kernel
+    unsigned long long phase_ns[4];     // persistent kernel: device time per phase kind
+    long long phase_cnt[4];             //   (Q, U_S, Z, U_J) and phases run, last solve
 };
 
 // ------------------------------------------------------------------ tiles
@@ -162,6 +166,7 @@ struct Plan {
     cudaStream_t cs = nullptr, cs2 = nullptr;
     int grid_tiles_A = 0, grid_tiles_G = 0, grid_tiles_GT = 0, grid_vec = 0;
     unsigned long long cond = 0;           // conditional handle of the loop node
+    int persist_grid = 0;                  // persistent engine: blocks (0: not set up yet)
 };
 
 // ------------------------------------------------------------------ internal entry points
@@ -194,7 +199,7 @@ sla_status kernel_times(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, c
     sla_status capture_##T(sla_csr *A, Plan *p);                                                    \
     sla_status times_##T(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, cudaStream_t s);     \
     sla_status run_##T(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,            \
-                       long long maxit, cudaStream_t s);                                            \
+                       long long maxit, int engine, cudaStream_t s);                                \
     sla_status grad_##T(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g,         \
                         cudaStream_t s);
 SLA_COMBO_DECL(ff)

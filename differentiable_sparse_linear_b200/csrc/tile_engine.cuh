@@ -102,6 +102,25 @@ __device__ __forceinline__ void mbar_wait_bounded(uint64_t *bar, uint32_t parity
         }
     }
 }
+// Same, and also give up at once when *abort (a block-wide flag) is set; a wait that runs
+// out sets it, so one stalled wait does not leave the block's later waits running out too.
+__device__ __forceinline__ void mbar_wait_bounded(uint64_t *bar, uint32_t parity, int *err,
+                                                  volatile int *abort)
+{
+    if (mbar_try_wait(bar, parity))
+        return;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (abort && *abort)
+            return;
+        if (global_ns() - t0 > WAIT_LIMIT_NS) {
+            atomicOr(err, 2);
+            if (abort)
+                *abort = 1;
+            return;
+        }
+    }
+}
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
 {
     asm volatile(

@@ -86,15 +86,35 @@ typedef struct {
                            dL/dx and dL/db and all solver vectors are fp64 (dL/dA stays fp32);
                            the default tolerance is then 1e-10.  Ignored for fp64 matrices
                            and for list handles. */
-    int32_t reserved;
+    int32_t engine;     /* how the solve loop runs (SLA_ENGINE_*); 0 -> automatic */
 } sla_pcg_opts;
+
+/* Solve engines.  Both run every step of the method on the GPU with the same fused
+ * operations and the same stopping test; the dot products are summed over different
+ * block partitions (each in a fixed order, so each engine is deterministic), so their
+ * iterates agree to rounding, not bit for bit.
+ *   SLA_ENGINE_GRAPH: one kernel per fused operation, the iteration loop a CUDA graph with
+ *     a device-side conditional (while) node -- any row-length mix.
+ *   SLA_ENGINE_PERSISTENT: the whole solve in one cooperative launch; the fused operations
+ *     are phases separated by grid barriers, and the matrix stream of the next phase is
+ *     prefetched while the current one runs.  For single systems whose matrices (A, and G
+ *     and G^T with SPAI) hold at most 8 entries per row, with at most 8 right-hand sides
+ *     (fp64 vectors: at most 4); fp32 vectors with at most 2 right-hand sides also allow
+ *     rows of up to 16 entries.
+ *   SLA_ENGINE_AUTO (0): persistent where it applies, graph otherwise.
+ * Asking for SLA_ENGINE_PERSISTENT where it does not apply fails with SLA_ERR_INVALID_ARG.
+ * List handles always use the one-block-per-system list kernel (SLA_ENGINE_LIST). */
+#define SLA_ENGINE_AUTO 0
+#define SLA_ENGINE_GRAPH 1
+#define SLA_ENGINE_PERSISTENT 2
+#define SLA_ENGINE_LIST 3
 
 /* Per right-hand side (or per system of a list) solver outcome. */
 typedef struct {
     int64_t iters;      /* number of products q = A p taken (0 when b = 0)                   */
     double relres;      /* ||r||/||b|| of the recursive residual at exit (0 when b = 0)      */
     int32_t status;     /* SLA_SUCCESS, SLA_NOT_CONVERGED or SLA_BREAKDOWN                   */
-    int32_t reserved;
+    int32_t engine;     /* the engine that ran the solve (SLA_ENGINE_GRAPH, _PERSISTENT, _LIST) */
 } sla_pcg_info;
 
 /* ---------------------------------------------------------------- library */
@@ -221,6 +241,17 @@ SLA_API sla_status sla_pcg_solve_batched_noalloc(const sla_csr *A, const sla_pre
  * are unspecified afterwards (the next solve re-initialises them).  Synchronises `stream`. */
 SLA_API sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t nrhs,
                                         int32_t vector_f64, int32_t reps, double *h_ms, void *stream);
+
+/* Device time per phase of the last persistent-engine solve of the (A, M, nrhs, vector_f64)
+ * solver, measured inside the kernel by block 0 from one grid barrier to the next (so each
+ * phase's time includes the barrier that ends it).  h_ms[0..3]: mean ms of a
+ * [0] p-update + q = A p, [1] x/r update with y = G^T r (SPAI), [2] z = G y + eps r (SPAI),
+ * [3] x/r update with z = D^-1 r (Jacobi or none); h_count[0..3]: phases of each kind run.
+ * SLA_ERR_INVALID_ARG when that solver's last solve did not run on the persistent engine.
+ * Synchronises `stream`. */
+SLA_API sla_status sla_pcg_phase_times(const sla_csr *A, const sla_precond *M, int32_t nrhs,
+                                       int32_t vector_f64, double *h_ms, int64_t *h_count,
+                                       void *stream);
 
 /* Device bytes the solver workspace takes for (A, M, nrhs, vector_f64); it depends on n and nnz only,
  * never on the iteration count ([TS] Complexity). */

@@ -40,13 +40,17 @@ def _iters_ok(gpu, ora_it, w, vf64):
     return iters_close(gpu, ora_it)
 
 
+@pytest.mark.parametrize("engine", ["auto", "graph"])
 @pytest.mark.parametrize("cfg,size,vf64", SINGLE)
-def test_forward_parity(ora, cfg, size, vf64):
+def test_forward_parity(ora, cfg, size, vf64, engine):
     import differentiable_sparse_linear_b200 as sla
     w = W.workload(cfg, size)
     Ad = matrix(w.A)
     M, _G = precond(w, Ad)
-    x, info = sla.sla_pcg_solve(Ad, M, dev(w.B, _vecs(w, vf64)), rtol=w.tol, vector_f64=vf64)
+    x, info = sla.sla_pcg_solve(Ad, M, dev(w.B, _vecs(w, vf64)), rtol=w.tol, vector_f64=vf64,
+                                engine=engine)
+    if engine == "graph":
+        assert info.engine == "graph"
     ref = ora.pcg(w.A, w.B, **_ora_kw(w))
     assert info.status == 0 and ref.status == 0
     assert _iters_ok(info.iters, ref.iters, w, vf64), (info.iters, ref.iters)
@@ -58,14 +62,16 @@ def test_forward_parity(ora, cfg, size, vf64):
     assert true <= (10 * w.tol if w.dtype == np.float64 else 1e-3)
 
 
+@pytest.mark.parametrize("engine", ["auto", "graph"])
 @pytest.mark.parametrize("cfg,size,vf64", SINGLE)
-def test_adjoint_parity(ora, cfg, size, vf64):
+def test_adjoint_parity(ora, cfg, size, vf64, engine):
     import differentiable_sparse_linear_b200 as sla
     w = W.workload(cfg, size)
     Ad = matrix(w.A)
     M, _G = precond(w, Ad)
-    x, _ = sla.sla_pcg_solve(Ad, M, dev(w.B, _vecs(w, vf64)), rtol=w.tol, vector_f64=vf64)
-    lam, g, info = sla.sla_pcg_adjoint(Ad, M, x, dev(w.W, _vecs(w, vf64)), rtol=w.tol, vector_f64=vf64)
+    x, _ = sla.sla_pcg_solve(Ad, M, dev(w.B, _vecs(w, vf64)), rtol=w.tol, vector_f64=vf64, engine=engine)
+    lam, g, info = sla.sla_pcg_adjoint(Ad, M, x, dev(w.W, _vecs(w, vf64)), rtol=w.tol, vector_f64=vf64,
+                                       engine=engine)
     xo = ora.pcg(w.A, w.B, **_ora_kw(w)).x
     ref = ora.adjoint(w.A, xo, w.W, **_ora_kw(w))
     assert info.status == 0
@@ -78,15 +84,17 @@ def test_adjoint_parity(ora, cfg, size, vf64):
     assert rel(host(g), g2) <= (1e-15 if w.dtype == np.float64 else 1e-7)
 
 
+@pytest.mark.parametrize("engine", ["auto", "graph"])
 @pytest.mark.parametrize("k", [1, 2, 5, 17])
 @pytest.mark.parametrize("cfg,vf64", [(1, False), (2, False), (5, False), (5, True)])
-def test_lockstep_iterates(ora, cfg, vf64, k):
+def test_lockstep_iterates(ora, cfg, vf64, k, engine):
     """Both sides run exactly k iterations; the iterates agree (no stopping-rule effects)."""
     import differentiable_sparse_linear_b200 as sla
     w = W.workload(cfg, "small")
     Ad = matrix(w.A)
     M, _G = precond(w, Ad)
-    x, info = sla.sla_pcg_solve(Ad, M, dev(w.B, _vecs(w, vf64)), rtol=1e-300, maxit=k, vector_f64=vf64)
+    x, info = sla.sla_pcg_solve(Ad, M, dev(w.B, _vecs(w, vf64)), rtol=1e-300, maxit=k, vector_f64=vf64,
+                                engine=engine)
     assert info.status == sla.SLA_NOT_CONVERGED and info.iters == k
     ref = ora.pcg(w.A, w.B, precond=w.precond, G=w.G, eps=w.eps, fixed_iters=k)
     bound = 1e-11 if (w.dtype == np.float64 or vf64) else 1e-5
