@@ -54,24 +54,8 @@ k_update_jacobi(int64_t n, V *x, V *r, const V *p, const V *q, V *z, const V *di
     for (int i = 0; i < 2 * K; ++i)
         part[i] = 0.0;
     const int64_t stride = (int64_t)gridDim.x * VEC_T;
-    for (int64_t i = (int64_t)blockIdx.x * VEC_T + threadIdx.x; i < n; i += stride) {
-        const double di = (double)dinv[i];
-#pragma unroll
-        for (int c = 0; c < K; ++c) {
-            const int64_t e = i * K + c;
-            double rv = (double)r[e];
-            if (s_on[c] != 0.0) {
-                x[e] = vfma<V>(s_a[c], p[e], x[e]);
-                const V rn = vfma<V>(-s_a[c], q[e], r[e]);
-                r[e] = rn;
-                rv = (double)rn;
-            }
-            const V zv = (V)(rv * di);
-            z[e] = zv;
-            part[c] += rv * rv;
-            part[K + c] += rv * (double)zv;
-        }
-    }
+    for (int64_t i = (int64_t)blockIdx.x * VEC_T + threadIdx.x; i < n; i += stride)
+        jacobi_row<V, K>(i, x, r, p, q, z, dinv, s_a, s_on, part);
     UJFinal fin{st, K};
     auto sync = [] { __syncthreads(); };
     grid_reduce_finalize<VEC_T, 2 * K>(part, partials, st, fin, s_red, &s_flag, s_sum, (int)threadIdx.x, sync);

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstring>
 
 #include "sla_internal.cuh"
 
@@ -120,6 +121,68 @@ __device__ __forceinline__ double vfma<double>(double a, double b, double c)
     return __fma_rn(a, b, c);
 }
 
+// A row of K contiguous vector elements (the solver's [n][K] layout) moved with the widest
+// access its size allows, up to 16 bytes; the row must be aligned to that width (the
+// solver's vectors are 256-byte aligned and K is a power of two).  Plain loads: the data
+// may have been written earlier in the same kernel by other blocks.
+template <typename V, int K>
+struct RowIO {
+    static constexpr int BYTES = K * (int)sizeof(V);
+    static constexpr int W = BYTES % 16 == 0 ? 16 : BYTES % 8 == 0 ? 8 : (int)sizeof(V);
+    static constexpr int N = BYTES / W;          // accesses per row
+    static constexpr int E = W / (int)sizeof(V); // elements per access
+    __device__ static __forceinline__ void load(const V *p, V (&v)[K])
+    {
+        if constexpr (W == 16) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const uint4 u = reinterpret_cast<const uint4 *>(p)[i];
+                memcpy(&v[i * E], &u, 16);
+            }
+        } else if constexpr (W == 8 && sizeof(V) == 4) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const uint2 u = reinterpret_cast<const uint2 *>(p)[i];
+                memcpy(&v[i * E], &u, 8);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+                v[c] = p[c];
+        }
+    }
+    __device__ static __forceinline__ void store(V *p, const V (&v)[K])
+    {
+        if constexpr (W == 16) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                uint4 u;
+                memcpy(&u, &v[i * E], 16);
+                reinterpret_cast<uint4 *>(p)[i] = u;
+            }
+        } else if constexpr (W == 8 && sizeof(V) == 4) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                uint2 u;
+                memcpy(&u, &v[i * E], 8);
+                reinterpret_cast<uint2 *>(p)[i] = u;
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+                p[c] = v[c];
+        }
+    }
+};
+
+// Interface of an operation (the row epilogue an SpMV engine runs), for K right-hand sides:
+//   NP dot products per column reduced over the grid, NS staged scalars, NV own-row
+//   vectors the epilogue reads, NG gathered vectors combined into the SpMV operand;
+//   operand(j, c) / operand_row(j, o): the operand at vector row j (global memory);
+//   combine(g, c): the operand from the NG gathered values (shared-memory windows);
+//   load_rv(v, i, o): own-row vector v at row i; emit(i, acc, part, s, rv): the epilogue of
+//   row i with its row sums acc; finalize(sums): the scalar step after the grid reduction.
+
 // y = A x for K right-hand sides with leading dimension ld (columns c >= nc are zero).
 template <typename V, int K>
 struct OpSpmv {
@@ -143,6 +206,19 @@ struct OpSpmv {
     {
         return c < nc ? __ldg(&x[j * ld + c]) : (V)0;
     }
+    // caller vectors: any leading dimension, so element by element
+    __device__ __forceinline__ void operand_row(int64_t j, V (&o)[K], const double *s) const
+    {
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            o[c] = operand(j, c, s);
+    }
+    __device__ __forceinline__ void load_rv(int, int64_t, V (&o)[K]) const
+    {
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            o[c] = (V)0;
+    }
     template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N], const double *,
                                          const RV &) const
@@ -159,6 +235,7 @@ struct OpSpmv {
 template <typename V, int K>
 struct OpQ {
     using VV = V;
+    using IO = RowIO<V, K>;
     static constexpr int NP = 1, NS = K, NV = 2;
     const V *z;
     const V *p_old;
@@ -184,26 +261,42 @@ struct OpQ {
     {
         return vfma<V>(s[c], p_old[j * K + c], z[j * K + c]);
     }
+    __device__ __forceinline__ void operand_row(int64_t j, V (&o)[K], const double *s) const
+    {
+        V p[K], zz[K];
+        IO::load(p_old + j * K, p);
+        IO::load(z + j * K, zz);
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            o[c] = vfma<V>(s[c], p[c], zz[c]);
+    }
+    __device__ __forceinline__ void load_rv(int v, int64_t i, V (&o)[K]) const
+    {
+        IO::load(row_vec(v) + i * K, o);
+    }
     template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
                                          const double *s, const RV &rv) const
     {
+        V pn[K], qv[K];
 #pragma unroll
         for (int c = 0; c < K; ++c) {
-            const V pn = vfma<V>(s[c], rv.get(0, i, c), rv.get(1, i, c));
-            const V qv = (V)acc[c];
-            p_new[i * K + c] = pn;
-            q[i * K + c] = qv;
-            part[c] += (double)pn * (double)qv;
+            pn[c] = vfma<V>(s[c], rv.get(0, i, c), rv.get(1, i, c));
+            qv[c] = (V)acc[c];
+            part[c] += (double)pn[c] * (double)qv[c];
         }
+        IO::store(p_new + i * K, pn);
+        IO::store(q + i * K, qv);
     }
     __device__ void finalize(const double *sums) const { finalize_alpha(st, sums); }
 };
 
-// U_S: r_new = r_old - alpha q, x += alpha p, y = G^T r_new, partial r_new.r_new
+// U_S: r_new = r_old - alpha q, x += alpha p, y = G^T r_new, partial r_new.r_new.  Columns
+// that have stopped keep r and x (x is rewritten with its own value).
 template <typename V, int K>
 struct OpUS {
     using VV = V;
+    using IO = RowIO<V, K>;
     static constexpr int NP = 1, NS = 2 * K, NV = 4;
     const V *r_old;
     const V *q;
@@ -238,19 +331,34 @@ struct OpUS {
     {
         return rnew(r_old[j * K + c], q[j * K + c], c, s);
     }
+    __device__ __forceinline__ void operand_row(int64_t j, V (&o)[K], const double *s) const
+    {
+        V ro[K], qq[K];
+        IO::load(r_old + j * K, ro);
+        IO::load(q + j * K, qq);
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            o[c] = rnew(ro[c], qq[c], c, s);
+    }
+    __device__ __forceinline__ void load_rv(int v, int64_t i, V (&o)[K]) const
+    {
+        IO::load(row_vec(v) + i * K, o);
+    }
     template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
                                          const double *s, const RV &rv) const
     {
+        V rn[K], xn[K], yv[K];
 #pragma unroll
         for (int c = 0; c < K; ++c) {
-            const V rn = rnew(rv.get(0, i, c), rv.get(1, i, c), c, s);
-            r_new[i * K + c] = rn;
-            if (s[K + c] != 0.0)
-                x[i * K + c] = vfma<V>(s[c], rv.get(2, i, c), rv.get(3, i, c));
-            y[i * K + c] = (V)acc[c];
-            part[c] += (double)rn * (double)rn;
+            rn[c] = rnew(rv.get(0, i, c), rv.get(1, i, c), c, s);
+            xn[c] = s[K + c] != 0.0 ? vfma<V>(s[c], rv.get(2, i, c), rv.get(3, i, c)) : rv.get(3, i, c);
+            yv[c] = (V)acc[c];
+            part[c] += (double)rn[c] * (double)rn[c];
         }
+        IO::store(r_new + i * K, rn);
+        IO::store(x + i * K, xn);
+        IO::store(y + i * K, yv);
     }
     __device__ void finalize(const double *sums) const
     {
@@ -265,6 +373,7 @@ struct OpUS {
 template <typename V, int K>
 struct OpZ {
     using VV = V;
+    using IO = RowIO<V, K>;
     static constexpr int NP = 1, NS = 1, NV = 1;
     const V *y;
     const V *r;
@@ -282,19 +391,58 @@ struct OpZ {
     {
         return y[j * K + c];
     }
+    __device__ __forceinline__ void operand_row(int64_t j, V (&o)[K], const double *) const
+    {
+        IO::load(y + j * K, o);
+    }
+    __device__ __forceinline__ void load_rv(int, int64_t i, V (&o)[K]) const
+    {
+        IO::load(r + i * K, o);
+    }
     template <int N, class RV>
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
                                          const double *s, const RV &rv) const
     {
+        V zv[K];
 #pragma unroll
         for (int c = 0; c < K; ++c) {
             const V rv_ = rv.get(0, i, c);
-            const V zv = vfma<V>(s[0], rv_, (V)acc[c]);
-            z[i * K + c] = zv;
-            part[c] += (double)rv_ * (double)zv;
+            zv[c] = vfma<V>(s[0], rv_, (V)acc[c]);
+            part[c] += (double)rv_ * (double)zv[c];
         }
+        IO::store(z + i * K, zv);
     }
     __device__ void finalize(const double *sums) const { finalize_beta(st, sums); }
 };
+
+// U_J on row i: x += alpha p and r -= alpha q in the active columns, z = D^-1 r; adds r.r
+// to part[c] and r.z to part[K + c].  Stopped columns are rewritten with their own values.
+template <typename V, int K>
+__device__ __forceinline__ void jacobi_row(int64_t i, V *x, V *r, const V *p, const V *q, V *z,
+                                           const V *dinv, const double *alpha, const double *on,
+                                           double (&part)[2 * K])
+{
+    using IO = RowIO<V, K>;
+    V xr[K], rr[K], pr[K], qr[K], zr[K];
+    const double di = (double)dinv[i];
+    IO::load(x + i * K, xr);
+    IO::load(r + i * K, rr);
+    IO::load(p + i * K, pr);
+    IO::load(q + i * K, qr);
+#pragma unroll
+    for (int c = 0; c < K; ++c) {
+        if (on[c] != 0.0) {
+            xr[c] = vfma<V>(alpha[c], pr[c], xr[c]);
+            rr[c] = vfma<V>(-alpha[c], qr[c], rr[c]);
+        }
+        const double rv = (double)rr[c];
+        zr[c] = (V)(rv * di);
+        part[c] += rv * rv;
+        part[K + c] += rv * (double)zr[c];
+    }
+    IO::store(x + i * K, xr);
+    IO::store(r + i * K, rr);
+    IO::store(z + i * K, zr);
+}
 
 }  // namespace sla

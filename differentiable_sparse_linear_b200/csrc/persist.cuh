@@ -56,12 +56,13 @@ __device__ __forceinline__ bool wait_go(volatile int *go, volatile int *stop, vo
     if (*go >= target)
         return true;
     const unsigned long long t0 = global_ns();
-    for (;;) {
+    for (unsigned i = 1;; ++i) {
         if (*go >= target)
             break;
         if (*stop || *abort)
             return false;
-        if (global_ns() - t0 > WAIT_LIMIT_NS) {
+        __nanosleep(64);
+        if ((i & 15u) == 0 && global_ns() - t0 > WAIT_LIMIT_NS) {
             atomicOr(err, 4);
             *abort = 1;
             return false;
@@ -98,16 +99,26 @@ __device__ __forceinline__ bool wait_empty(uint64_t *bar, uint32_t parity, volat
     if (mbar_try_wait(bar, parity))
         return true;
     const unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    for (unsigned i = 1;; ++i) {
+        // a short suspension: the stop flag is polled between rounds
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(2000u)
+            : "memory");
+        if (ok)
+            return true;
         if (*stop || *abort)
             return false;
-        if (global_ns() - t0 > WAIT_LIMIT_NS) {
+        if ((i & 15u) == 0 && global_ns() - t0 > WAIT_LIMIT_NS) {
             atomicOr(err, 2);
             *abort = 1;
             return false;
         }
     }
-    return true;
 }
 
 template <typename VM, typename VV, int K, int MAXL>
@@ -310,13 +321,15 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
             atomicAdd(bar, 1ull);
             if (ld_acquire_gpu(bar) < target) {
                 const unsigned long long t0 = global_ns();
-                while (ld_acquire_gpu(bar) < target) {
-                    if (*abort)
-                        break;
-                    if (global_ns() - t0 > WAIT_LIMIT_NS) {
-                        atomicOr(a.err, 4);
-                        *abort = 1;
-                        break;
+                for (unsigned i = 1; ld_acquire_gpu(bar) < target; ++i) {
+                    if ((i & 15u) == 0) {
+                        if (*abort)
+                            break;
+                        if (global_ns() - t0 > WAIT_LIMIT_NS) {
+                            atomicOr(a.err, 4);
+                            *abort = 1;
+                            break;
+                        }
                     }
                 }
             }
@@ -380,24 +393,8 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
         zero();
         const int64_t n = a.A.n;
         const int64_t stride = (int64_t)gridDim.x * TC;
-        for (int64_t i = (int64_t)blockIdx.x * TC + tid; i < n; i += stride) {
-            const double di = (double)a.dinv[i];
-#pragma unroll
-            for (int c = 0; c < K; ++c) {
-                const int64_t e = i * K + c;
-                double rv = (double)a.ra[e];
-                if (s_scal[K + c] != 0.0) {
-                    a.x[e] = vfma<VV>(s_scal[c], p[e], a.x[e]);
-                    const VV rn = vfma<VV>(-s_scal[c], a.q[e], a.ra[e]);
-                    a.ra[e] = rn;
-                    rv = (double)rn;
-                }
-                const VV zv = (VV)(rv * di);
-                a.z[e] = zv;
-                part[c] += rv * rv;
-                part[K + c] += rv * (double)zv;
-            }
-        }
+        for (int64_t i = (int64_t)blockIdx.x * TC + tid; i < n; i += stride)
+            jacobi_row<VV, K>(i, a.x, a.ra, p, a.q, a.z, a.dinv, s_scal, s_scal + K, part);
         phase_end(part, 2 * K, PH_UJ);
         if (tid == 0) {
             finalize_residual(&s_st, s_sum);

@@ -36,7 +36,7 @@ namespace sla {
 // window rows per tile (0: no windows).
 template <int K>
 struct RowTmaCfg;
-template <> struct RowTmaCfg<1> { static constexpr int TC = 256, RPT = 2, D = 2048, NST = 2, WMAX = 2048; };
+template <> struct RowTmaCfg<1> { static constexpr int TC = 256, RPT = 2, D = 3072, NST = 2, WMAX = 2048; };
 template <> struct RowTmaCfg<2> { static constexpr int TC = 256, RPT = 2, D = 2048, NST = 2, WMAX = 1024; };
 template <> struct RowTmaCfg<4> { static constexpr int TC = 256, RPT = 1, D = 2048, NST = 2, WMAX = 0; };
 template <> struct RowTmaCfg<8> { static constexpr int TC = 256, RPT = 1, D = 2048, NST = 2, WMAX = 0; };
@@ -245,10 +245,15 @@ struct RowTma {
                 const int r = tid + q * TC;
 #pragma unroll
                 for (int v = 0; v < NV; ++v)
-                    if (Op::rv_src(v) < 0)
+                    if (Op::rv_src(v) < 0) {
+                        if (r < nr) {
+                            op.load_rv(v, (int64_t)r0 + r, rvals[q].v[v]);
+                        } else {
 #pragma unroll
-                        for (int c = 0; c < K; ++c)
-                            rvals[q].v[v][c] = r < nr ? op.row_vec(v)[((int64_t)r0 + r) * K + c] : (VV)0;
+                            for (int c = 0; c < K; ++c)
+                                rvals[q].v[v][c] = (VV)0;
+                        }
+                    }
             }
             double acc[RPT][K];
 #pragma unroll
@@ -311,10 +316,15 @@ struct RowTma {
             off[q] = live ? rpp[r] - kb32 : 0;
             len[q] = live ? rpp[r + 1] - kb32 - off[q] : 0;
 #pragma unroll
-            for (int v = 0; v < NV; ++v)
+            for (int v = 0; v < NV; ++v) {
+                if (live) {
+                    op.load_rv(v, (int64_t)r0 + r, rvals[q].v[v]);
+                } else {
 #pragma unroll
-                for (int c = 0; c < K; ++c)
-                    rvals[q].v[v][c] = live ? op.row_vec(v)[((int64_t)r0 + r) * K + c] : (VV)0;
+                    for (int c = 0; c < K; ++c)
+                        rvals[q].v[v][c] = (VV)0;
+                }
+            }
 #pragma unroll
             for (int u = 0; u < MAXL; ++u) {
                 cj[q][u] = u < len[q] ? cc[off[q] + u] : 0;
@@ -328,10 +338,15 @@ struct RowTma {
 #pragma unroll
         for (int q = 0; q < RPT; ++q)
 #pragma unroll
-            for (int u = 0; u < MAXL; ++u)
+            for (int u = 0; u < MAXL; ++u) {
+                if (u < len[q]) {
+                    op.operand_row(cj[q][u], ov[q][u], s_scal);
+                } else {
 #pragma unroll
-                for (int c = 0; c < K; ++c)
-                    ov[q][u][c] = u < len[q] ? op.operand(cj[q][u], c, s_scal) : (VV)0;
+                    for (int c = 0; c < K; ++c)
+                        ov[q][u][c] = (VV)0;
+                }
+            }
 #pragma unroll
         for (int q = 0; q < RPT; ++q) {
             const int r = tid + q * TC;

@@ -83,41 +83,49 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
+// try_wait that lets the hardware suspend the thread until the phase completes (or the
+// hinted time passes), so waiting warps leave the issue slots to the working ones.
+constexpr uint32_t SUSPEND_HINT_NS = 100000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(SUSPEND_HINT_NS)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ unsigned long long global_ns()
 {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for the phase with the given parity; give up after WAIT_LIMIT_NS and flag it.
-__device__ __forceinline__ void mbar_wait_bounded(uint64_t *bar, uint32_t parity, int *err)
-{
-    if (mbar_try_wait(bar, parity))
-        return;
-    const unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > WAIT_LIMIT_NS) {
-            atomicOr(err, 2);
-            return;
-        }
-    }
-}
-// Same, and also give up at once when *abort (a block-wide flag) is set; a wait that runs
+// Wait for the phase with the given parity; give up after WAIT_LIMIT_NS and flag it.  Also
+// give up at once when *abort (a block-wide flag, may be null) is set; a wait that runs
 // out sets it, so one stalled wait does not leave the block's later waits running out too.
+// The clock is read only every 16th round.
 __device__ __forceinline__ void mbar_wait_bounded(uint64_t *bar, uint32_t parity, int *err,
-                                                  volatile int *abort)
+                                                  volatile int *abort = nullptr)
 {
     if (mbar_try_wait(bar, parity))
         return;
     const unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (abort && *abort)
+    for (unsigned i = 1;; ++i) {
+        if (mbar_try_wait_sleep(bar, parity))
             return;
-        if (global_ns() - t0 > WAIT_LIMIT_NS) {
-            atomicOr(err, 2);
-            if (abort)
-                *abort = 1;
-            return;
+        if ((i & 15u) == 0) {
+            if (abort && *abort)
+                return;
+            if (global_ns() - t0 > WAIT_LIMIT_NS) {
+                atomicOr(err, 2);
+                if (abort)
+                    *abort = 1;
+                return;
+            }
         }
     }
 }
