@@ -100,7 +100,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self):
+        """Host time of a point in the run (samples are kept from the window between two marks)."""
+        return time.time()
 
     def wait_first_sample(self, limit_s: float = 10.0):
         """nvidia-smi's start-up takes driver locks; begin timing only once it samples."""
@@ -109,7 +113,8 @@ class ClockSampler:
             time.sleep(0.05)
         time.sleep(0.25)
 
-    def stop(self) -> dict:
+    def stop(self, window: tuple[float, float] | None = None) -> dict:
+        """Stop sampling; summarise the samples taken inside `window` (host times), or all."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -121,7 +126,10 @@ class ClockSampler:
             self.t.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = [ln for ts, ln in self.lines if window is None or window[0] <= ts <= window[1] + 0.25]
+        if not lines and self.lines:              # a timed region shorter than the sampling period
+            lines = [self.lines[-1][1]]
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -318,35 +326,44 @@ def run_ours(args):
                 x, lam)
 
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
-        step(b, wl, X)
-    torch.cuda.synchronize()
+    flush.zero_()
 
     def barrier():
         if world > 1:
             dist.barrier()
 
+    # the clock sampler starts before the warm-up, so its start-up stays out of the timed
+    # region; only the samples taken inside the timed region are summarised
     clocks = ClockSampler(gpu_bus_id(local) if rank == 0 else None)
-    barrier()
-    torch.cuda.synchronize()
     if rank == 0:
         clocks.start()
         clocks.wait_first_sample()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(b, wl, X)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     total_iters = 0
     total_launch = 0
+    t_begin = clocks.mark()
     ev0.record()
-    for _ in range(args.steps):
+    for k in range(args.steps):
         flush.zero_()
         it, nl, _, _ = step(b, wl, X)
+        evs[k].record()
         total_iters += it
         total_launch += nl + 1
     ev1.record()
     torch.cuda.synchronize()
+    t_end = clocks.mark()
     barrier()
-    clk = clocks.stop() if rank == 0 else {}
+    clk = clocks.stop((t_begin, t_end)) if rank == 0 else {}
     ms = ev0.elapsed_time(ev1)
+    step_ms = [ev0.elapsed_time(evs[0])] + [evs[k - 1].elapsed_time(evs[k]) for k in range(1, args.steps)]
     t = torch.tensor([ms, float(total_iters)], dtype=torch.float64, device=dev)
     if world > 1:
         tm = t.clone()
@@ -491,6 +508,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between steps (512 MiB write)", "setup_s": setup_s,
                        "engine": "+".join(sorted(engines_seen))},
+            "step_ms": {"min": min(step_ms), "median": float(np.median(step_ms)), "max": max(step_ms)},
             "roofline": roofline, "spmv": spmv, "kernels": kernels,
             "gpu_launches": total_launch, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }

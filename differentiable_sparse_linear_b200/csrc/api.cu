@@ -82,14 +82,8 @@ sla_status ensure_tiles(sla_csr *A, int D, int RMAX, cudaStream_t s, const TileP
     return SLA_SUCCESS;
 }
 
-// Operand windows: for each tile, the rows of the gathered vectors its columns (and its own
-// rows) touch, as at most WSEG 4-row-aligned ranges totalling at most wmax rows; tiles that
-// do not fit get nseg = 0 (global gathers).  Gaps of up to 32 rows are bridged.
-sla_status ensure_windows(sla_csr *A, const TilePart *tp_c, int wmax, cudaStream_t s)
+static sla_status fetch_host_cols(sla_csr *A, cudaStream_t s)
 {
-    TilePart *tp = const_cast<TilePart *>(tp_c);
-    if (tp->win_rows == wmax)
-        return SLA_SUCCESS;
     if (A->h_ci.size() != (size_t)A->nnz) {
         A->h_ci.resize((size_t)A->nnz);
         if (A->nnz > 0) {
@@ -98,79 +92,237 @@ sla_status ensure_windows(sla_csr *A, const TilePart *tp_c, int wmax, cudaStream
             SLA_CUDA_TRY(cudaStreamSynchronize(s));
         }
     }
+    return SLA_SUCCESS;
+}
+
+// Operand window of rows [r0, r1): the rows of the gathered vectors their columns (and the
+// rows themselves) touch, as at most WSEG 4-row-aligned ranges totalling at most wmax rows
+// and ending at most at row_limit; false when they do not fit.  Gaps of up to 32 rows are
+// bridged.
+static bool window_for_rows(const sla_csr *A, int64_t r0, int64_t r1, int wmax, int64_t row_limit,
+                            WinDesc *out)
+{
+    const int64_t GAP = 32;
+    WinDesc w{};
+    *out = w;
+    int64_t lo[8], hi[8];   // closed ranges
+    int ns = 0;
+    bool ok = wmax > 0;
+    auto add = [&](int64_t j) {
+        for (int i = 0; i < ns; ++i)
+            if (j >= lo[i] - GAP && j <= hi[i] + GAP) {
+                lo[i] = std::min(lo[i], j);
+                hi[i] = std::max(hi[i], j);
+                return;
+            }
+        if (ns == 8) {
+            ok = false;
+            return;
+        }
+        lo[ns] = hi[ns] = j;
+        ++ns;
+    };
+    for (int64_t r = r0; ok && r < r1; ++r)   // the rows themselves (own-row values)
+        add(r);
+    for (int64_t k = A->h_rp[(size_t)r0]; ok && k < (int64_t)A->h_rp[(size_t)r1]; ++k)
+        add(A->h_ci[(size_t)k]);
+    if (!ok)
+        return false;
+    // sort, align to 4 rows, merge
+    int64_t L[8], H[8];
+    int m = 0;
+    for (int i = 0; i < ns; ++i) {
+        int b = i;
+        for (int jdx = i + 1; jdx < ns; ++jdx)
+            if (lo[jdx] < lo[b])
+                b = jdx;
+        std::swap(lo[i], lo[b]);
+        std::swap(hi[i], hi[b]);
+    }
+    for (int i = 0; i < ns; ++i) {
+        const int64_t a = lo[i] & ~(int64_t)3, e = (hi[i] + 1 + 3) & ~(int64_t)3;
+        if (m > 0 && a <= H[m - 1] + GAP)
+            H[m - 1] = std::max(H[m - 1], e);
+        else {
+            L[m] = a;
+            H[m] = e;
+            ++m;
+        }
+    }
+    int64_t total = 0;
+    for (int i = 0; i < m; ++i)
+        total += H[i] - L[i];
+    if (m > WSEG || total > wmax || (m > 0 && H[m - 1] > row_limit))
+        return false;
+    w.nseg = m;
+    for (int i = 0; i < m; ++i) {
+        w.a[i] = (int)L[i];
+        w.l[i] = (int)(H[i] - L[i]);
+    }
+    *out = w;
+    return true;
+}
+
+// Operand windows of every tile of a partition (tiles that do not fit get nseg = 0 and
+// gather from global memory).  Windows end inside the vectors (row n at most), since the
+// gathered vectors can be the caller's.
+sla_status ensure_windows(sla_csr *A, const TilePart *tp_c, int wmax, cudaStream_t s)
+{
+    TilePart *tp = const_cast<TilePart *>(tp_c);
+    if (tp->win_rows == wmax)
+        return SLA_SUCCESS;
+    SLA_TRY(fetch_host_cols(A, s));
     std::vector<int2> desc((size_t)tp->n_tiles + 1);
     if (tp->n_tiles > 0)
         SLA_CUDA_TRY(cudaMemcpy(desc.data(), tp->d_desc, desc.size() * sizeof(int2), cudaMemcpyDeviceToHost));
     std::vector<WinDesc> win((size_t)std::max(tp->n_tiles, 1));
-    const int64_t GAP = 32;
-    for (int t = 0; t < tp->n_tiles; ++t) {
-        WinDesc w{};
-        int64_t lo[8], hi[8];   // closed ranges
-        int ns = 0;
-        bool ok = wmax > 0;
-        auto add = [&](int64_t j) {
-            for (int i = 0; i < ns; ++i)
-                if (j >= lo[i] - GAP && j <= hi[i] + GAP) {
-                    lo[i] = std::min(lo[i], j);
-                    hi[i] = std::max(hi[i], j);
-                    return;
-                }
-            if (ns == 8) {
-                ok = false;
-                return;
-            }
-            lo[ns] = hi[ns] = j;
-            ++ns;
-        };
-        const int r0 = desc[t].x, r1 = desc[t + 1].x;
-        if (r1 > r0) {
-            add(r0);
-            add(r1 - 1);
-        }
-        for (int64_t k = (uint32_t)desc[t].y; ok && k < (int64_t)(uint32_t)desc[t + 1].y; ++k)
-            add(A->h_ci[(size_t)k]);
-        // sort, align to 4 rows, merge
-        int64_t L[8], H[8];
-        int m = 0;
-        if (ok) {
-            for (int i = 0; i < ns; ++i) {
-                int b = i;
-                for (int jdx = i + 1; jdx < ns; ++jdx)
-                    if (lo[jdx] < lo[b])
-                        b = jdx;
-                std::swap(lo[i], lo[b]);
-                std::swap(hi[i], hi[b]);
-            }
-            for (int i = 0; i < ns; ++i) {
-                const int64_t a = lo[i] & ~(int64_t)3, e = (hi[i] + 1 + 3) & ~(int64_t)3;
-                if (m > 0 && a <= H[m - 1] + GAP)
-                    H[m - 1] = std::max(H[m - 1], e);
-                else {
-                    L[m] = a;
-                    H[m] = e;
-                    ++m;
-                }
-            }
-            int64_t total = 0;
-            for (int i = 0; i < m; ++i)
-                total += H[i] - L[i];
-            if (m > WSEG || total > wmax || (m > 0 && H[m - 1] > A->n))
-                ok = false;
-        }
-        if (ok) {
-            w.nseg = m;
-            for (int i = 0; i < m; ++i) {
-                w.a[i] = (int)L[i];
-                w.l[i] = (int)(H[i] - L[i]);
-            }
-        }
-        win[(size_t)t] = w;
-    }
+    for (int t = 0; t < tp->n_tiles; ++t)
+        window_for_rows(A, desc[t].x, desc[t + 1].x, wmax, A->n, &win[(size_t)t]);
     if (!tp->d_win)
         SLA_CUDA_TRY(cudaMalloc((void **)&tp->d_win, win.size() * sizeof(WinDesc)));
     SLA_CUDA_TRY(cudaMemcpyAsync(tp->d_win, win.data(), win.size() * sizeof(WinDesc), cudaMemcpyHostToDevice, s));
     SLA_CUDA_TRY(cudaStreamSynchronize(s));
     tp->win_rows = wmax;
+    return SLA_SUCCESS;
+}
+
+// Sliced copy (see SellPart).
+sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **out)
+{
+    if (A->sell && A->sell->maxl == maxl) {
+        *out = A->sell;
+        return SLA_SUCCESS;
+    }
+    SLA_TRY(fetch_host_cols(A, s));
+    const int64_t n = A->n;
+    const int64_t nsl = (n + 31) / 32;
+    std::vector<uint2> desc((size_t)std::max<int64_t>(nsl, 1));
+    std::vector<uint8_t> lens((size_t)std::max<int64_t>(nsl * 32, 1), 0);
+    std::vector<int32_t> offs;
+    std::vector<std::vector<int64_t>> slice_offs((size_t)nsl);
+    bool rel16 = true;
+    int64_t slot_rows = 0, n_diag = 0;
+    for (int64_t sl = 0; sl < nsl; ++sl) {
+        int64_t L = 0;
+        std::vector<int64_t> u;
+        bool diag = true;
+        for (int64_t r = sl * 32; r < std::min(n, sl * 32 + 32); ++r) {
+            const int64_t len = (int64_t)A->h_rp[(size_t)r + 1] - A->h_rp[(size_t)r];
+            lens[(size_t)r] = (uint8_t)len;
+            L = std::max(L, len);
+            for (int64_t k = A->h_rp[(size_t)r]; k < (int64_t)A->h_rp[(size_t)r + 1]; ++k) {
+                const int64_t d = (int64_t)A->h_ci[(size_t)k] - r;
+                if (d < -32768 || d > 32767)
+                    rel16 = false;
+                if (diag && std::find(u.begin(), u.end(), d) == u.end()) {
+                    u.push_back(d);
+                    if ((int64_t)u.size() > maxl)
+                        diag = false;
+                }
+            }
+        }
+        if (slot_rows >= ((int64_t)1 << 27) || (int64_t)offs.size() >= ((int64_t)1 << 31) - maxl)
+            return fail(SLA_ERR_UNSUPPORTED, "matrix too large for the sliced layout");
+        uint32_t w1 = 0;
+        if (diag && !u.empty()) {
+            std::sort(u.begin(), u.end());
+            w1 = (1u << 31) | (uint32_t)offs.size();
+            for (int64_t d : u)
+                offs.push_back((int32_t)d);
+            L = (int64_t)u.size();
+            slice_offs[(size_t)sl] = u;
+            ++n_diag;
+        }
+        desc[(size_t)sl] = make_uint2((uint32_t)(slot_rows << 5) | (uint32_t)L, w1);
+        slot_rows += L;
+    }
+    const int64_t slots = slot_rows * 32;
+    std::vector<int32_t> perm((size_t)std::max<int64_t>(slots, 1), -1);
+    std::vector<int16_t> i16;
+    std::vector<int32_t> i32;
+    if (rel16)
+        i16.assign((size_t)std::max<int64_t>(slots, 1), 0);
+    else
+        i32.assign((size_t)std::max<int64_t>(slots, 1), 0);
+    for (int64_t sl = 0; sl < nsl; ++sl) {
+        const int64_t e0 = (int64_t)(desc[(size_t)sl].x >> 5) * 32;
+        const bool diag = desc[(size_t)sl].y >> 31;
+        const std::vector<int64_t> &u = slice_offs[(size_t)sl];
+        for (int64_t l = 0; l < 32; ++l) {
+            const int64_t r = sl * 32 + l;
+            if (r >= n)
+                break;
+            const int64_t k0 = A->h_rp[(size_t)r], len = (int64_t)A->h_rp[(size_t)r + 1] - k0;
+            for (int64_t t = 0; t < len; ++t) {
+                const int64_t j = A->h_ci[(size_t)(k0 + t)];
+                // slot row of this entry: its offset's position (diagonal), else its rank
+                const int64_t pos = diag ? (int64_t)(std::lower_bound(u.begin(), u.end(), j - r) - u.begin()) : t;
+                const size_t e = (size_t)(e0 + pos * 32 + l);
+                perm[e] = (int32_t)(k0 + t);
+                if (rel16)
+                    i16[e] = (int16_t)(j - r);
+                else
+                    i32[e] = (int32_t)j;
+            }
+        }
+    }
+    if (A->sell) {
+        cudaFree(A->sell->d_desc);
+        cudaFree(A->sell->d_offs);
+        cudaFree(A->sell->d_lens);
+        cudaFree(A->sell->d_idx);
+        cudaFree(A->sell->d_perm);
+        cudaFree(A->sell->d_val);
+        delete A->sell;
+        A->sell = nullptr;
+    }
+    SellPart *sp = new SellPart();
+    sp->n_slices = nsl;
+    sp->n_slots = slots;
+    sp->rel16 = rel16 ? 1 : 0;
+    sp->maxl = maxl;
+    sp->n_diag = n_diag;
+    const size_t vsz = vbytes(A->dtype);
+    const size_t isz = rel16 ? 2 : 4;
+    auto cleanup = [&](cudaError_t e, const char *what) {
+        cudaFree(sp->d_desc);
+        cudaFree(sp->d_offs);
+        cudaFree(sp->d_lens);
+        cudaFree(sp->d_idx);
+        cudaFree(sp->d_perm);
+        cudaFree(sp->d_val);
+        delete sp;
+        return cuda_fail(e, what);
+    };
+    cudaError_t e = cudaMalloc((void **)&sp->d_desc, desc.size() * sizeof(uint2));
+    if (e == cudaSuccess)
+        e = cudaMalloc((void **)&sp->d_offs, std::max<size_t>(offs.size(), 1) * sizeof(int32_t));
+    if (e == cudaSuccess)
+        e = cudaMalloc((void **)&sp->d_lens, lens.size());
+    if (e == cudaSuccess)
+        e = cudaMalloc(&sp->d_idx, perm.size() * isz);
+    if (e == cudaSuccess)
+        e = cudaMalloc((void **)&sp->d_perm, perm.size() * 4);
+    if (e == cudaSuccess)
+        e = cudaMalloc(&sp->d_val, perm.size() * vsz);
+    if (e != cudaSuccess)
+        return cleanup(e, "sliced layout");
+    e = cudaMemcpyAsync(sp->d_desc, desc.data(), desc.size() * sizeof(uint2), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !offs.empty())
+        e = cudaMemcpyAsync(sp->d_offs, offs.data(), offs.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(sp->d_lens, lens.data(), lens.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(sp->d_idx, rel16 ? (const void *)i16.data() : (const void *)i32.data(),
+                            perm.size() * isz, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(sp->d_perm, perm.data(), perm.size() * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return cleanup(e, "sliced layout upload");
+    A->sell = sp;
+    *out = sp;
     return SLA_SUCCESS;
 }
 
@@ -343,6 +495,16 @@ static void free_csr(sla_csr *A)
         cudaFree(kv.second.d_desc);
         if (kv.second.d_win)
             cudaFree(kv.second.d_win);
+    }
+    if (A->sell) {
+        cudaFree(A->sell->d_desc);
+        cudaFree(A->sell->d_offs);
+        cudaFree(A->sell->d_lens);
+        cudaFree(A->sell->d_idx);
+        cudaFree(A->sell->d_perm);
+        cudaFree(A->sell->d_val);
+        delete A->sell;
+        A->sell = nullptr;
     }
     if (A->d_err)
         cudaFree(A->d_err);

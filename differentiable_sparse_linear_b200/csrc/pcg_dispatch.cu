@@ -146,6 +146,32 @@ sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t
     return SLA_SUCCESS;
 }
 
+// Packed values: slot s takes val[perm[s]] (0 for padding slots).
+template <typename V>
+__global__ void k_pack_values(int64_t n_slots, const int32_t *perm, const V *val, V *out)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_slots; i += stride) {
+        const int32_t k = perm[i];
+        out[i] = k >= 0 ? val[k] : (V)0;
+    }
+}
+
+sla_status launch_sell_values(const sla_csr *A, const SellPart *sp, cudaStream_t s)
+{
+    if (sp->n_slots == 0)
+        return SLA_SUCCESS;
+    const int grid = (int)std::min<int64_t>(vec_grid(A), (sp->n_slots + 255) / 256);
+    if (A->dtype == SLA_F32)
+        k_pack_values<float><<<grid, 256, 0, s>>>(sp->n_slots, sp->d_perm, (const float *)A->val,
+                                                  (float *)sp->d_val);
+    else
+        k_pack_values<double><<<grid, 256, 0, s>>>(sp->n_slots, sp->d_perm, (const double *)A->val,
+                                                   (double *)sp->d_val);
+    SLA_CUDA_TRY(cudaGetLastError());
+    return SLA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ dispatch
 sla_status capture_plan_graph(sla_csr *A, Plan *p)
 {

@@ -554,26 +554,29 @@ template <typename VM, typename VV, int K, int MAXL>
 static sla_status persist_launch(sla_csr *A, Plan *p, cudaStream_t s)
 {
     using Pk = Persist<VM, VV, K, MAXL>;
-    constexpr int THREADS = Pk::TC + 32;
     auto kern = k_pcg_persistent<VM, VV, K, MAXL>;
     PersistArgs<VM, VV> a{};
-    auto mat = [&](const sla_csr *M_, MatView<VM> &mv, const WinDesc *&w) -> sla_status {
-        const TilePart *tp;
-        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(M_), RowTmaCfg<K>::D,
-                             RowTmaCfg<K>::TC * RowTmaCfg<K>::RPT, s, &tp));
-        mv = view<VM>(M_, tp);
-        w = nullptr;
-        if (RowTmaCfg<K>::WMAX > 0) {
-            SLA_TRY(ensure_windows(const_cast<sla_csr *>(M_), tp, RowTmaCfg<K>::WMAX, s));
-            w = tp->d_win;   // workspace vectors are 256-byte aligned, as window copies need
-        }
+    // sliced ELL copies: built once per matrix; values gathered from the CSR arrays on every
+    // solve, so values changed in place since the last solve are used
+    auto sell = [&](const sla_csr *M_, SellView<VM> &v) -> sla_status {
+        const SellPart *sp;
+        SLA_TRY(ensure_sell(const_cast<sla_csr *>(M_), MAXL, s, &sp));
+        SLA_TRY(launch_sell_values(M_, sp, s));
+        v.desc = sp->d_desc;
+        v.offs = sp->d_offs;
+        v.lens = sp->d_lens;
+        v.idx16 = sp->rel16 ? (const int16_t *)sp->d_idx : nullptr;
+        v.idx32 = sp->rel16 ? nullptr : (const int32_t *)sp->d_idx;
+        v.val = (const VM *)sp->d_val;
+        v.n = M_->n;
+        v.n_slices = sp->n_slices;
         return SLA_SUCCESS;
     };
-    SLA_TRY(mat(A, a.A, a.winA));
     a.spai = p->kind == 2 ? 1 : 0;
+    SLA_TRY(sell(A, a.A));
     if (a.spai) {
-        SLA_TRY(mat(p->M->G, a.G, a.winG));
-        SLA_TRY(mat(p->M->GT, a.GT, a.winGT));
+        SLA_TRY(sell(p->M->G, a.G));
+        SLA_TRY(sell(p->M->GT, a.GT));
     }
     a.x = (VV *)p->x; a.ra = (VV *)p->ra; a.rb = (VV *)p->rb; a.pa = (VV *)p->pa; a.pb = (VV *)p->pb;
     a.q = (VV *)p->q; a.z = (VV *)p->z; a.y = (VV *)p->y;
@@ -585,25 +588,22 @@ static sla_status persist_launch(sla_csr *A, Plan *p, cudaStream_t s)
     a.partials = p->partials;
     a.err = &p->st->error;
     if (p->persist_grid == 0) {
-        SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Pk::SMEM));
         int per_sm = 0;
-        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, Pk::SMEM));
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Pk::TB, 0));
         if (per_sm < 1)
             return fail(SLA_ERR_UNSUPPORTED, "persistent solver kernel does not fit on an SM");
         // every block must be resident at once (cooperative launch); the partials buffer
-        // holds 2 slots of 2K doubles per block.  No more blocks than the largest phase
-        // has work units (tiles, or TC-row chunks for the elementwise phase): every block
+        // holds 2 slots of 2K doubles per block.  At least one slice per warp: every block
         // arrives at every grid barrier, so idle blocks only add to the barrier's cost.
         const int cap = (int)(((size_t)A->num_sms * 32 * 2 * KMAX) / (2 * 2 * K));
-        int64_t units = (A->n + Pk::TC - 1) / Pk::TC;
-        units = std::max<int64_t>(units, a.A.n_tiles);
+        int64_t slices = a.A.n_slices;
         if (a.spai)
-            units = std::max<int64_t>(units, std::max(a.G.n_tiles, a.GT.n_tiles));
+            slices = std::max(slices, std::max(a.G.n_slices, a.GT.n_slices));
+        const int64_t units = (slices + Pk::TB / 32 - 1) / (Pk::TB / 32);
         p->persist_grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, std::min(per_sm * A->num_sms, cap)));
     }
     void *args[] = {(void *)&a};
-    SLA_CUDA_TRY(cudaLaunchCooperativeKernel((const void *)kern, dim3(p->persist_grid), dim3(THREADS), args,
-                                             Pk::SMEM, s));
+    SLA_CUDA_TRY(cudaLaunchCooperativeKernel((const void *)kern, dim3(p->persist_grid), dim3(Pk::TB), args, 0, s));
     return SLA_SUCCESS;
 }
 

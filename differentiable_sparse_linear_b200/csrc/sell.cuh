@@ -1,0 +1,118 @@
+// Sliced SpMV with fused row epilogues for the persistent solver (short-row matrices; the
+// storage is described with SellPart).
+//
+// A warp owns a slice of 32 rows, one row per lane; a slot row of the slice is one
+// coalesced 128-byte access of values (64 bytes of 16-bit column offsets in an index
+// slice), and a lane's loop over its row's entries is fully unrolled up to MAXL with every
+// load independent.  Operands are gathered through L1/L2
+// (the vectors were written before the grid barrier that opened this phase); a block owns
+// a contiguous run of slices and its warps take consecutive slices, so the lines that hold
+// a row's vertical neighbours (a grid line away) were just brought in by the same warp.
+// Row sums are fp32 when values and vectors are fp32 (at most MAXL terms), fp64 otherwise.
+#pragma once
+
+#include <type_traits>
+
+#include "pcg_ops.cuh"
+
+namespace sla {
+
+template <typename VM>
+struct SellView {
+    const uint2 *desc;         // per slice: {first slot row << 5 | L, diagonal << 31 | offsets}
+    const int32_t *offs;       // offset lists of the diagonal slices
+    const uint8_t *lens;       // per row (index slices)
+    const int16_t *idx16;      // column - row (rel16), or null
+    const int32_t *idx32;      // columns, or null
+    const VM *val;
+    int64_t n;
+    int64_t n_slices;
+};
+
+// Own-row vector values of a lane's row.
+template <typename VV, int K, int NV>
+struct LaneVals {
+    VV v[NV > 0 ? NV : 1][K];
+    __device__ __forceinline__ VV get(int vi, int64_t, int c) const { return v[vi][c]; }
+};
+
+// The slices [s0, s1) of this block, warps round-robin over consecutive slices; `part`
+// takes the epilogue's dot-product partials in a fixed order.  In a diagonal slice the
+// operand rows are row + offs[u] (shared by the warp), so the operand loads and the value
+// loads go out together; a padding slot (value 0) reads a clamped row and adds 0.
+template <int K, typename VM, int MAXL, int TB, class Op, int NR>
+__device__ __forceinline__ void sell_phase(const SellView<VM> &m, const Op &op, double (&part)[NR],
+                                           const double *s_scal)
+{
+    using VV = typename Op::VV;
+    using Acc = typename std::conditional<sizeof(VM) == 4 && sizeof(VV) == 4, float, double>::type;
+    constexpr int NV = Op::NV;
+    constexpr int NW = TB / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t s0 = m.n_slices * blockIdx.x / gridDim.x;
+    const int64_t s1 = m.n_slices * (blockIdx.x + 1) / gridDim.x;
+    const int32_t nlast = (int32_t)m.n - 1;
+    uint2 dn = s0 + warp < s1 ? m.desc[s0 + warp] : make_uint2(0u, 0u);
+    for (int64_t sl = s0 + warp; sl < s1; sl += NW) {
+        const uint2 d = dn;
+        if (sl + NW < s1)
+            dn = m.desc[sl + NW];   // next slice's descriptor, one slice ahead
+        const int L = (int)(d.x & 31u);
+        const int64_t e0 = (int64_t)(d.x >> 5) * 32 + lane;
+        const int32_t row = (int32_t)(sl * 32 + lane);
+        const bool live = row < m.n;
+        LaneVals<VV, K, NV> rv;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            if (live) {
+                op.load_rv(v, row, rv.v[v]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    rv.v[v][c] = (VV)0;
+            }
+        }
+        Acc s[K];
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            s[c] = (Acc)0;
+        if (d.y >> 31) {
+            const int32_t *of = m.offs + (d.y & 0x7fffffffu);
+#pragma unroll
+            for (int u = 0; u < MAXL; ++u) {
+                if (u < L) {
+                    const int32_t j = min(max(row + of[u], 0), nlast);
+                    const Acc av = (Acc)m.val[e0 + u * 32];
+                    VV o[K];
+                    op.operand_row(j, o, s_scal);
+#pragma unroll
+                    for (int c = 0; c < K; ++c)
+                        s[c] = fma(av, (Acc)o[c], s[c]);
+                }
+            }
+        } else {
+            const int len = m.lens[row];   // 0 past the last row
+#pragma unroll
+            for (int u = 0; u < MAXL; ++u) {
+                if (u < len) {
+                    const int32_t j = m.idx16 ? row + (int32_t)m.idx16[e0 + u * 32] : m.idx32[e0 + u * 32];
+                    const Acc av = (Acc)m.val[e0 + u * 32];
+                    VV o[K];
+                    op.operand_row(j, o, s_scal);
+#pragma unroll
+                    for (int c = 0; c < K; ++c)
+                        s[c] = fma(av, (Acc)o[c], s[c]);
+                }
+            }
+        }
+        if (live) {
+            double acc[K];
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+                acc[c] = (double)s[c];
+            op.emit(row, acc, part, s_scal, rv);
+        }
+    }
+}
+
+}  // namespace sla

@@ -88,6 +88,34 @@ struct __align__(16) WinDesc {
     int pad[16 - 1 - 2 * WSEG];
 };
 
+// Sliced storage (slices of 32 rows) of a short-row matrix for the persistent solver.
+// Slice s holds rows [32 s, 32 s + 32); its entries sit in L_s slot rows of 32 (slot row u,
+// lane l: entry u of row 32 s + l), so a warp reads slot row u of its slice with one
+// coalesced access.  Two slice kinds:
+//   diagonal slice: every row's columns lie at offsets (column - row) from one sorted list
+//     of L_s offsets shared by the slice (a stencil's ±1, ±line, 0 ...); slot row u holds
+//     the values at offset u (0 where a row has no entry there), so no column index is
+//     stored per entry and the operand addresses need no per-entry load;
+//   index slice: slot row u holds entry u of each row, with its column as a 16-bit offset
+//     from the row (rel16, when every offset of the matrix fits) or a 32-bit column, and
+//     per-row lengths.
+// desc[s] = {first slot row << 5 | L_s, diagonal << 31 | position of its offsets}.  Values
+// are gathered from the CSR arrays by `perm` (slot -> CSR position, -1 for padding) before
+// each solve, so values changed in place are picked up.
+struct SellPart {
+    int64_t n_slices = 0;
+    int64_t n_slots = 0;                 // entry slots (32 per slot row), padding included
+    int rel16 = 0;
+    int maxl = 0;                        // offsets per diagonal slice at most
+    int64_t n_diag = 0;                  // diagonal slices
+    uint2 *d_desc = nullptr;
+    int32_t *d_offs = nullptr;           // offset lists of the diagonal slices
+    uint8_t *d_lens = nullptr;           // row lengths, n_slices * 32 (0 past the last row)
+    void *d_idx = nullptr;               // int16 offsets (rel16) or int32 columns
+    int32_t *d_perm = nullptr;
+    void *d_val = nullptr;               // the matrix's type
+};
+
 // Read-only view of a CSR matrix passed to kernels.
 template <typename V>
 struct MatView {
@@ -125,6 +153,7 @@ struct sla_csr {
     std::vector<int32_t> h_rp;
     std::vector<int32_t> h_ci;             // host copy of col (short-row matrices, for windows)
     std::map<int, sla::TilePart> tiles;    // by item budget D
+    sla::SellPart *sell = nullptr;         // sliced ELL copy (persistent solver)
     int device = 0;
     int num_sms = 148;
     std::vector<sla::Plan *> plans;
@@ -173,6 +202,10 @@ struct Plan {
 sla_status ensure_tiles(sla_csr *A, int D, int RMAX, cudaStream_t s, const TilePart **out);
 // Build (once) the operand windows of a tile partition, at most wmax rows per tile.
 sla_status ensure_windows(sla_csr *A, const TilePart *tp, int wmax, cudaStream_t s);
+// Build (once) the sliced copy of a short-row matrix (diagonal slices of at most maxl
+// offsets); gather its values.
+sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **out);
+sla_status launch_sell_values(const sla_csr *A, const SellPart *sp, cudaStream_t s);
 size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K, int vec64);
 sla_status get_plan(sla_csr *A, const sla_precond *M, int K, int vec64, Plan **out);
 void destroy_plan(Plan *p);

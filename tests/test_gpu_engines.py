@@ -74,7 +74,9 @@ def test_engines_agree(ora, cfg, size, vf64):
         assert a.status == 0 and b.status == 0
         assert abs(a.iters - b.iters) <= 1, (a.iters, b.iters)
     f64 = vf64 or w.dtype == np.float64
-    assert rel(host(xp), host(xg)) <= (1e-9 if f64 else 1e-4)
+    # both stop at relative residual w.tol; the summation orders differ, so the iterates
+    # agree to the solve tolerance, not to rounding
+    assert rel(host(xp), host(xg)) <= (max(1e-9, 10 * w.tol) if f64 else 1e-4)
     kw = dict(precond=w.precond, G=w.G, eps=w.eps, tol=w.tol)
     if w.nrhs > 1:
         xo, outs = ora.pcg_multi(w.A, w.B, **kw)
