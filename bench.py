@@ -164,7 +164,7 @@ def measured_peaks() -> tuple[float, str]:
         return 6650.0, "fallback"
 
 
-KERNEL_SOURCES = ("row_engine.cuh", "tile_engine.cuh", "pcg_ops.cuh", "persist.cuh", "pcg_impl.cuh")
+KERNEL_SOURCES = ("row_engine.cuh", "tile_engine.cuh", "pcg_ops.cuh", "persist.cuh", "sell.cuh", "pcg_impl.cuh")
 
 
 def kernel_source_hash() -> str:
@@ -177,8 +177,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str) -> int | None:
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+def profiled_traffic(kernel: str, workload: str, units: float = 1.0) -> int | None:
+    """DRAM bytes (read + write) of one launch, from the committed ncu summary if it was
+    taken on the current kernel sources: the summary holds bytes per unit (per launch, or per
+    PCG iteration for the persistent solver), scaled here by the launch's units."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
@@ -187,7 +189,7 @@ def profiled_traffic(kernel: str, workload: str) -> int | None:
         parts = ln.split()
         if len(parts) >= 4 and not ln.startswith("#") and parts[0] == kernel and parts[1] == workload:
             if parts[3] == src:
-                return int(float(parts[2]))
+                return int(float(parts[2]) * units)
     return None
 
 
@@ -449,7 +451,8 @@ def run_ours(args):
                            "timing": "in-kernel, grid barrier to grid barrier (block 0)"}
         ach = launch_bytes / (launch_ms * 1e6)
         roofline = {"bound": "hbm", "kernel": "k_pcg_persistent", "achieved": ach, "peak": peak, "unit": "GB/s",
-                    "frac": ach / peak, "traffic": profiled_traffic("k_pcg_persistent", w.name),
+                    "frac": ach / peak,
+                    "traffic": profiled_traffic("k_pcg_persistent", w.name, units=pcnt[0]),
                     "peak_source": peak_kind, "algorithmic_bytes": launch_bytes, "ms_per_launch": launch_ms,
                     "units_per_launch": {nm: pcnt[slot[nm]] for nm in names},
                     "note": "one launch = one forward solve; bytes = per-phase algorithmic bytes x phases run"}

@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <map>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -200,6 +201,7 @@ sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **ou
     std::vector<uint8_t> lens((size_t)std::max<int64_t>(nsl * 32, 1), 0);
     std::vector<int32_t> offs;
     std::vector<std::vector<int64_t>> slice_offs((size_t)nsl);
+    std::map<std::vector<int64_t>, uint32_t> list_pos;
     bool rel16 = true;
     int64_t slot_rows = 0, n_diag = 0;
     for (int64_t sl = 0; sl < nsl; ++sl) {
@@ -226,9 +228,14 @@ sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **ou
         uint32_t w1 = 0;
         if (diag && !u.empty()) {
             std::sort(u.begin(), u.end());
-            w1 = (1u << 31) | (uint32_t)offs.size();
-            for (int64_t d : u)
-                offs.push_back((int32_t)d);
+            // slices with the same offsets share one list (a stencil has a handful)
+            auto it = list_pos.find(u);
+            if (it == list_pos.end()) {
+                it = list_pos.emplace(u, (uint32_t)offs.size()).first;
+                for (int64_t d : u)
+                    offs.push_back((int32_t)d);
+            }
+            w1 = (1u << 31) | it->second;
             L = (int64_t)u.size();
             slice_offs[(size_t)sl] = u;
             ++n_diag;

@@ -593,9 +593,9 @@ static sla_status persist_launch(sla_csr *A, Plan *p, cudaStream_t s)
         if (per_sm < 1)
             return fail(SLA_ERR_UNSUPPORTED, "persistent solver kernel does not fit on an SM");
         // every block must be resident at once (cooperative launch); the partials buffer
-        // holds 2 slots of 2K doubles per block.  At least one slice per warp: every block
+        // holds 4 slots of 2K doubles per block.  At least one slice per warp: every block
         // arrives at every grid barrier, so idle blocks only add to the barrier's cost.
-        const int cap = (int)(((size_t)A->num_sms * 32 * 2 * KMAX) / (2 * 2 * K));
+        const int cap = (int)(((size_t)A->num_sms * 32 * 2 * KMAX) / (4 * 2 * K));
         int64_t slices = a.A.n_slices;
         if (a.spai)
             slices = std::max(slices, std::max(a.G.n_slices, a.GT.n_slices));

@@ -11,9 +11,9 @@
 // (alpha, the stopping test, beta) without a last-block ticket or a round trip through
 // global state.  Block 0 writes the final state back for the host.
 //
-// Memory ordering across the barrier follows the cooperative-groups grid barrier: block
-// barrier, then thread 0 fences and arrives, spins on the counter with acquire loads,
-// fences, and releases its block with another block barrier.
+// Memory ordering across the barrier: block barrier, then thread 0 arrives with a release
+// reduction on the counter and spins on it with acquire loads, then releases its block with
+// another block barrier (causality is transitive through the block barriers).
 //
 // The grid barrier's wait is bounded in time: a wait that runs out sets the solve's error
 // word and a block-wide abort flag, and the block stops at that phase end.
@@ -33,7 +33,7 @@ struct PersistArgs {
     VV *x, *ra, *rb, *pa, *pb, *q, *z, *y;
     const VV *dinv;                   // Jacobi (or ones without a preconditioner)
     PcgState *st;
-    double *partials;                 // 2 slots of [grid][2K]
+    double *partials;                 // 4 slots of [grid][2K]
     int spai;                         // 1: Q, U_S, Z phases; 0: Q, U_J phases
     int *err;
 };
@@ -52,6 +52,8 @@ struct Persist {
     // blocks per SM the register budget is cut for (two: 32 warps per SM) where the lane
     // code fits 64 registers without spills
     static constexpr int MINB = (K == 1 && MAXL == 8) ? 2 : 1;
+    // slices per warp round (their loads in flight together): two where that fits the registers
+    static constexpr int RS = (K == 1 || (K == 2 && sizeof(VV) == 4)) ? 2 : 1;
     using OQ = OpQ<VV, K>;
     using OUS = OpUS<VV, K>;
     using OZ = OpZ<VV, K>;
@@ -84,7 +86,7 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
 
     __shared__ double s_red[(TB / 32) * NR];
     __shared__ double s_scal[2 * K + 1];
-    __shared__ double s_sum[NR];
+    __shared__ double s_sum[2 * NR];
     __shared__ PcgState s_st;
     __shared__ int s_abort, s_quit;
 
@@ -109,10 +111,11 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
     if (blockIdx.x == 0 && tid == 0)
         t_phase = global_ns();
 
-    // End of a phase: block sum, publish, grid barrier, all blocks' partials in block order
-    // into s_sum (n of the NR values are used).
-    auto phase_end = [&](double (&part)[NR], int n, int kind) {
-        double *slot = a.partials + (size_t)(seq & 1) * gridDim.x * NR;
+    // End of a phase, first half: block sum, publish it in this phase's slot (4 slots in
+    // turn: a slot is written again only after a barrier every reader of it has passed),
+    // grid barrier.  Returns the slot.
+    auto publish = [&](double (&part)[NR], int n, int kind) -> double * {
+        double *slot = a.partials + (size_t)(seq & 3) * gridDim.x * NR;
         block_sum<TB, NR>(part, s_red, tid, sync);
         if (tid < n)
             slot[(size_t)blockIdx.x * NR + tid] = part[0];
@@ -120,8 +123,9 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
         if (tid == 0) {
             unsigned long long *bar = &a.st->gbar;
             const unsigned long long target = (unsigned long long)seq * gridDim.x;
-            __threadfence();
-            atomicAdd(bar, 1ull);
+            // release: the block's writes (ordered before this thread by the block barrier)
+            // are visible to every block that acquires the count
+            asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(bar) : "memory");
             if (ld_acquire_gpu(bar) < target) {
                 const unsigned long long t0 = global_ns();
                 for (unsigned i = 1; ld_acquire_gpu(bar) < target; ++i) {
@@ -136,7 +140,6 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
                     }
                 }
             }
-            __threadfence();
             if (blockIdx.x == 0) {
                 const unsigned long long t1 = global_ns();
                 s_st.phase_ns[kind] += t1 - t_phase;
@@ -145,6 +148,11 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
             }
         }
         __syncthreads();
+        ++seq;
+        return slot;
+    };
+    // Second half: all blocks' partials of a slot, in block order, into out[0..n).
+    auto reduce = [&](const double *slot, int n, double *out) {
         double v[NR];
 #pragma unroll
         for (int i = 0; i < NR; ++i)
@@ -157,10 +165,10 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
         }
         block_sum<TB, NR>(v, s_red, tid, sync);
         if (tid < n)
-            s_sum[tid] = v[0];
+            out[tid] = v[0];
         __syncthreads();
-        ++seq;
     };
+    auto phase_end = [&](double (&part)[NR], int n, int kind) { reduce(publish(part, n, kind), n, s_sum); };
     // After thread 0 finalised: stop when every column is done or a wait ran out.
     auto decide = [&]() -> bool {
         if (tid == 0)
@@ -204,42 +212,48 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
             op.stage(s_scal);
         __syncthreads();
         zero();
-        sell_phase<K, VM, MAXL, TB>(a.A, op, part, s_scal);
+        sell_phase<K, VM, MAXL, TB, P::RS>(a.A, op, part, s_scal);
         phase_end(part, K, PH_Q);
         if (tid == 0)
             finalize_alpha(&s_st, s_sum);
         return decide();
     };
-    auto run_us = [&](bool odd) -> bool {
-        const auto op = P::opUS(a, odd, &s_st);
-        if (tid == 0)
-            op.stage(s_scal);
-        __syncthreads();
-        zero();
-        sell_phase<K, VM, MAXL, TB>(a.GT, op, part, s_scal);
-        phase_end(part, K, PH_US);
+    // U_S then Z.  Z needs U_S's vectors (the barrier) but not its scalar, so U_S's
+    // partials are reduced together with Z's at Z's end; U_S's residual test then decides
+    // as before (a stop there leaves Z's results unused: x, r and the counts are U_S's).
+    auto run_us_z = [&](bool odd) -> bool {
+        {
+            const auto op = P::opUS(a, odd, &s_st);
+            if (tid == 0)
+                op.stage(s_scal);
+            __syncthreads();
+            zero();
+            sell_phase<K, VM, MAXL, TB, P::RS>(a.GT, op, part, s_scal);
+        }
+        const double *slot_us = publish(part, K, PH_US);
+        {
+            const auto op = P::opZ(a, odd, &s_st);
+            if (tid == 0)
+                op.stage(s_scal);
+            __syncthreads();
+            zero();
+            sell_phase<K, VM, MAXL, TB, P::RS>(a.G, op, part, s_scal);
+        }
+        const double *slot_z = publish(part, K, PH_Z);
+        reduce(slot_us, K, s_sum);
+        reduce(slot_z, K, s_sum + K);
         if (tid == 0) {
             finalize_residual(&s_st, s_sum);
             signal_if_done(&s_st);
+            if (!s_st.all_done)
+                finalize_beta(&s_st, s_sum + K);
         }
-        return decide();
-    };
-    auto run_z = [&](bool odd) -> bool {
-        const auto op = P::opZ(a, odd, &s_st);
-        if (tid == 0)
-            op.stage(s_scal);
-        __syncthreads();
-        zero();
-        sell_phase<K, VM, MAXL, TB>(a.G, op, part, s_scal);
-        phase_end(part, K, PH_Z);
-        if (tid == 0)
-            finalize_beta(&s_st, s_sum);
         return decide();
     };
 
     bool quit;
     if (a.spai)
-        quit = run_us(true) || run_z(true);
+        quit = run_us_z(true);
     else
         quit = run_uj(a.pa);
     for (int it = 0; !quit; ++it) {
@@ -247,7 +261,7 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
         if (run_q(odd))
             break;
         if (a.spai)
-            quit = run_us(odd) || run_z(odd);
+            quit = run_us_z(odd);
         else
             quit = run_uj(odd ? a.pa : a.pb);
     }

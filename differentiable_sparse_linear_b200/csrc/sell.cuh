@@ -36,11 +36,12 @@ struct LaneVals {
     __device__ __forceinline__ VV get(int vi, int64_t, int c) const { return v[vi][c]; }
 };
 
-// The slices [s0, s1) of this block, warps round-robin over consecutive slices; `part`
-// takes the epilogue's dot-product partials in a fixed order.  In a diagonal slice the
-// operand rows are row + offs[u] (shared by the warp), so the operand loads and the value
-// loads go out together; a padding slot (value 0) reads a clamped row and adds 0.
-template <int K, typename VM, int MAXL, int TB, class Op, int NR>
+// The slices [s0, s1) of this block, warps round-robin over consecutive slices, RS slices
+// per round (their loads all in flight together); `part` takes the epilogue's dot-product
+// partials in a fixed order.  In a diagonal slice the operand rows are row + offs[u]
+// (shared by the warp), so the operand loads and the value loads go out together; a
+// padding slot (value 0) reads a clamped row and adds 0.
+template <int K, typename VM, int MAXL, int TB, int RS, class Op, int NR>
 __device__ __forceinline__ void sell_phase(const SellView<VM> &m, const Op &op, double (&part)[NR],
                                            const double *s_scal)
 {
@@ -52,65 +53,85 @@ __device__ __forceinline__ void sell_phase(const SellView<VM> &m, const Op &op, 
     const int64_t s0 = m.n_slices * blockIdx.x / gridDim.x;
     const int64_t s1 = m.n_slices * (blockIdx.x + 1) / gridDim.x;
     const int32_t nlast = (int32_t)m.n - 1;
-    uint2 dn = s0 + warp < s1 ? m.desc[s0 + warp] : make_uint2(0u, 0u);
-    for (int64_t sl = s0 + warp; sl < s1; sl += NW) {
-        const uint2 d = dn;
-        if (sl + NW < s1)
-            dn = m.desc[sl + NW];   // next slice's descriptor, one slice ahead
-        const int L = (int)(d.x & 31u);
-        const int64_t e0 = (int64_t)(d.x >> 5) * 32 + lane;
-        const int32_t row = (int32_t)(sl * 32 + lane);
-        const bool live = row < m.n;
-        LaneVals<VV, K, NV> rv;
+    // descriptors are loaded one round ahead (L = 0 past the run: nothing to do)
+    uint2 dn[RS];
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            if (live) {
-                op.load_rv(v, row, rv.v[v]);
-            } else {
+    for (int q = 0; q < RS; ++q) {
+        const int64_t sl = s0 + warp + (int64_t)q * NW;
+        dn[q] = sl < s1 ? m.desc[sl] : make_uint2(0u, 0u);
+    }
+    for (int64_t sb = s0 + warp; sb < s1; sb += (int64_t)NW * RS) {
+        uint2 d[RS];
 #pragma unroll
-                for (int c = 0; c < K; ++c)
-                    rv.v[v][c] = (VV)0;
-            }
+        for (int q = 0; q < RS; ++q) {
+            d[q] = dn[q];
+            const int64_t sl = sb + (int64_t)(q + RS) * NW;
+            dn[q] = sl < s1 ? m.desc[sl] : make_uint2(0u, 0u);
         }
-        Acc s[K];
+        Acc s[RS][K];
+        LaneVals<VV, K, NV> rv[RS];
 #pragma unroll
-        for (int c = 0; c < K; ++c)
-            s[c] = (Acc)0;
-        if (d.y >> 31) {
-            const int32_t *of = m.offs + (d.y & 0x7fffffffu);
+        for (int q = 0; q < RS; ++q) {
+            const int64_t sl = sb + (int64_t)q * NW;
+            const int32_t row = (int32_t)(sl * 32 + lane);
+            const bool live = sl < s1 && row < m.n;
+            const int L = (int)(d[q].x & 31u);
+            const int64_t e0 = (int64_t)(d[q].x >> 5) * 32 + lane;
 #pragma unroll
-            for (int u = 0; u < MAXL; ++u) {
-                if (u < L) {
-                    const int32_t j = min(max(row + of[u], 0), nlast);
-                    const Acc av = (Acc)m.val[e0 + u * 32];
-                    VV o[K];
-                    op.operand_row(j, o, s_scal);
+            for (int v = 0; v < NV; ++v) {
+                if (live) {
+                    op.load_rv(v, row, rv[q].v[v]);
+                } else {
 #pragma unroll
                     for (int c = 0; c < K; ++c)
-                        s[c] = fma(av, (Acc)o[c], s[c]);
+                        rv[q].v[v][c] = (VV)0;
                 }
             }
-        } else {
-            const int len = m.lens[row];   // 0 past the last row
-#pragma unroll
-            for (int u = 0; u < MAXL; ++u) {
-                if (u < len) {
-                    const int32_t j = m.idx16 ? row + (int32_t)m.idx16[e0 + u * 32] : m.idx32[e0 + u * 32];
-                    const Acc av = (Acc)m.val[e0 + u * 32];
-                    VV o[K];
-                    op.operand_row(j, o, s_scal);
-#pragma unroll
-                    for (int c = 0; c < K; ++c)
-                        s[c] = fma(av, (Acc)o[c], s[c]);
-                }
-            }
-        }
-        if (live) {
-            double acc[K];
 #pragma unroll
             for (int c = 0; c < K; ++c)
-                acc[c] = (double)s[c];
-            op.emit(row, acc, part, s_scal, rv);
+                s[q][c] = (Acc)0;
+            if (d[q].y >> 31) {
+                const int32_t *of = m.offs + (d[q].y & 0x7fffffffu);
+#pragma unroll
+                for (int u = 0; u < MAXL; ++u) {
+                    if (u < L) {
+                        const int32_t j = min(max(row + of[u], 0), nlast);
+                        const Acc av = (Acc)m.val[e0 + u * 32];
+                        VV o[K];
+                        op.operand_row(j, o, s_scal);
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            s[q][c] = fma(av, (Acc)o[c], s[q][c]);
+                    }
+                }
+            } else {
+                const int len = sl < s1 ? m.lens[row] : 0;   // 0 past the last row
+#pragma unroll
+                for (int u = 0; u < MAXL; ++u) {
+                    if (u < len) {
+                        const int32_t j =
+                            m.idx16 ? row + (int32_t)m.idx16[e0 + u * 32] : m.idx32[e0 + u * 32];
+                        const Acc av = (Acc)m.val[e0 + u * 32];
+                        VV o[K];
+                        op.operand_row(j, o, s_scal);
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            s[q][c] = fma(av, (Acc)o[c], s[q][c]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < RS; ++q) {
+            const int64_t sl = sb + (int64_t)q * NW;
+            const int32_t row = (int32_t)(sl * 32 + lane);
+            if (sl < s1 && row < m.n) {
+                double acc[K];
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    acc[c] = (double)s[q][c];
+                op.emit(row, acc, part, s_scal, rv[q]);
+            }
         }
     }
 }
