@@ -61,6 +61,87 @@ k_update_jacobi(int64_t n, V *x, V *r, const V *p, const V *q, V *z, const V *di
     grid_reduce_finalize<VEC_T, 2 * K>(part, partials, st, fin, s_red, &s_flag, s_sum, (int)threadIdx.x, sync);
 }
 
+// E_p: p_new = z + beta p_old (all rows, K columns).
+template <typename V, int K>
+__global__ void __launch_bounds__(VEC_T)
+k_ep(int64_t n, const V *z, const V *p_old, V *p_new, PcgState *st)
+{
+    __shared__ double s_b[K];
+    if (*(volatile int *)&st->all_done)
+        return;
+    if (threadIdx.x < K)
+        s_b[threadIdx.x] = st->beta[threadIdx.x];
+    __syncthreads();
+    using IO = RowIO<V, K>;
+    const int64_t stride = (int64_t)gridDim.x * VEC_T;
+    for (int64_t i = (int64_t)blockIdx.x * VEC_T + threadIdx.x; i < n; i += stride) {
+        V zz[K], pp[K], pn[K];
+        IO::load(z + i * K, zz);
+        IO::load(p_old + i * K, pp);
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            pn[c] = vfma<V>(s_b[c], pp[c], zz[c]);
+        IO::store(p_new + i * K, pn);
+    }
+}
+
+struct ERFinal {
+    PcgState *st;
+    __device__ void finalize(const double *sums) const
+    {
+        finalize_residual(st, sums);
+        signal_if_done(st);
+    }
+};
+
+// E_r: r_new = r_old - alpha q and x += alpha p in the active columns; partial r_new.r_new,
+// then the stopping test (the last block).
+template <typename V, int K>
+__global__ void __launch_bounds__(VEC_T)
+k_er(int64_t n, const V *r_old, const V *q, const V *p, V *x, V *r_new, double *partials, PcgState *st)
+{
+    __shared__ double s_a[K];
+    __shared__ double s_on[K];
+    __shared__ double s_red[(VEC_T / 32) * K];
+    __shared__ double s_sum[K];
+    __shared__ int s_flag;
+    if (*(volatile int *)&st->all_done)
+        return;
+    if (threadIdx.x < K) {
+        s_a[threadIdx.x] = st->alpha[threadIdx.x];
+        s_on[threadIdx.x] = st->active[threadIdx.x] ? 1.0 : 0.0;
+    }
+    __syncthreads();
+    using IO = RowIO<V, K>;
+    double part[K];
+#pragma unroll
+    for (int c = 0; c < K; ++c)
+        part[c] = 0.0;
+    const int64_t stride = (int64_t)gridDim.x * VEC_T;
+    for (int64_t i = (int64_t)blockIdx.x * VEC_T + threadIdx.x; i < n; i += stride) {
+        V ro[K], qq[K], pp[K], xx[K], rn[K];
+        IO::load(r_old + i * K, ro);
+        IO::load(q + i * K, qq);
+        IO::load(p + i * K, pp);
+        IO::load(x + i * K, xx);
+#pragma unroll
+        for (int c = 0; c < K; ++c) {
+            if (s_on[c] != 0.0) {
+                rn[c] = vfma<V>(-s_a[c], qq[c], ro[c]);
+                xx[c] = vfma<V>(s_a[c], pp[c], xx[c]);
+            } else {
+                rn[c] = ro[c];
+            }
+            part[c] += (double)rn[c] * (double)rn[c];
+        }
+        IO::store(r_new + i * K, rn);
+        IO::store(x + i * K, xx);
+    }
+    ERFinal fin{st};
+    auto sync = [] { __syncthreads(); };
+    grid_reduce_finalize<VEC_T, K>(part, partials, st, fin, s_red, &s_flag, s_sum, (int)threadIdx.x, sync);
+}
+
 // Reset the state and load the right-hand sides: r = b (padded to K columns), x = p = q = 0.
 template <typename V, int K>
 __global__ void k_init(int64_t n, int nrhs, const V *B, V *x, V *r, V *p, V *q, V *z, V *y,
@@ -241,10 +322,7 @@ constexpr int ROWS_MAXL = 16;
 
 template <int K, typename VM, class Op>
 struct TileLaunch {
-    using L = StageLayout<K, VM, typename Op::VV, Op::NV>;
     using LR = RowTmaLayout<K, VM, typename Op::VV, Op::NG>;
-    static constexpr int THREADS = TileCfg<K>::TC + 32;
-    static constexpr size_t SMEM = TileCfg<K>::NST * L::BYTES;
     static constexpr int RTHREADS = RowTmaCfg<K>::TC + 32;
     static constexpr size_t RSMEM = RowTmaCfg<K>::NST * LR::BYTES;
     int grid = 0;
@@ -285,12 +363,11 @@ struct TileLaunch {
             return setup_rows<16>(A, s);
         }
         const TilePart *tp;
-        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), TileCfg<K>::D, TileCfg<K>::RMAX, s, &tp));
+        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), Tile2Cfg<K>::D, Tile2Cfg<K>::RMAX, s, &tp));
         m = view<VM>(A, tp);
-        auto kern = k_tile<K, VM, Op>;
-        SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM));
+        auto kern = k_tile2<K, VM, Op>;
         int per_sm = 0;
-        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, SMEM));
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Tile2Cfg<K>::T, 0));
         per_sm = std::max(per_sm, 1);
         grid = std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
         maxl = 0;
@@ -310,7 +387,7 @@ struct TileLaunch {
         case 6: k_rows_tma<K, VM, 6, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         case 8: k_rows_tma<K, VM, 8, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         case 16: k_rows_tma<K, VM, 16, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
-        default: k_tile<K, VM, Op><<<grid, THREADS, SMEM, s>>>(m, op, part, st, err); break;
+        default: k_tile2<K, VM, Op><<<grid, Tile2Cfg<K>::T, 0, s>>>(m, op, part, st); break;
         }
     }
 };
@@ -352,6 +429,10 @@ struct PlanKernels {
     TileLaunch<K, VM, OpQ<VV, K>> LQ;
     TileLaunch<K, VM, OpUS<VV, K>> LUS;
     TileLaunch<K, VM, OpZ<VV, K>> LZ;
+    // matrices with long rows: operand vectors formed first (k_ep / k_er), one gather per entry
+    TileLaunch<K, VM, OpQm<VV, K>> LQm;
+    TileLaunch<K, VM, OpUSm<VV, K>> LUSm;
+    bool formA = false, formGT = false;
     int64_t n = 0;
     VV *x, *ra, *rb, *pa, *pb, *q, *z, *y;
     const VV *dinv = nullptr;
@@ -370,6 +451,9 @@ struct PlanKernels {
         part = p->partials;
         err = &p->st->error;
         SLA_TRY(LQ.setup(A, s));
+        formA = LQ.maxl == 0;
+        if (formA)
+            SLA_TRY(LQm.setup(A, s));
         gv = vec_grid(A);
         if (p->kind == 1)
             dinv = (const VV *)(sizeof(VV) == 8 ? M->d_dinv64 : M->d_dinv);
@@ -378,6 +462,9 @@ struct PlanKernels {
         if (p->kind == 2) {
             SLA_TRY(LZ.setup(M->G, s));
             SLA_TRY(LUS.setup(M->GT, s));
+            formGT = LUS.maxl == 0;
+            if (formGT)
+                SLA_TRY(LUSm.setup(M->GT, s));
         }
         p->grid_tiles_A = LQ.grid;
         p->grid_tiles_G = LZ.grid;
@@ -387,7 +474,12 @@ struct PlanKernels {
     }
     void Q(cudaStream_t s, const VV *pold, VV *pnew) const
     {
-        LQ.launch(s, OpQ<VV, K>{z, pold, pnew, q, st}, part, st, err);
+        if (formA) {
+            k_ep<VV, K><<<gv, VEC_T, 0, s>>>(n, z, pold, pnew, st);
+            LQm.launch(s, OpQm<VV, K>{pnew, q, st}, part, st, err);
+        } else {
+            LQ.launch(s, OpQ<VV, K>{z, pold, pnew, q, st}, part, st, err);
+        }
     }
     void UJ(cudaStream_t s, const VV *pcur) const
     {
@@ -395,7 +487,12 @@ struct PlanKernels {
     }
     void US(cudaStream_t s, const VV *rold, VV *rnew, const VV *pcur) const
     {
-        LUS.launch(s, OpUS<VV, K>{rold, q, pcur, x, rnew, x, y, st}, part, st, err);
+        if (formGT) {
+            k_er<VV, K><<<gv, VEC_T, 0, s>>>(n, rold, q, pcur, x, rnew, part, st);
+            LUSm.launch(s, OpUSm<VV, K>{rnew, y, st}, part, st, err);
+        } else {
+            LUS.launch(s, OpUS<VV, K>{rold, q, pcur, x, rnew, x, y, st}, part, st, err);
+        }
     }
     void Z(cudaStream_t s, const VV *rcur) const
     {

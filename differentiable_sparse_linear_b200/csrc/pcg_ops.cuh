@@ -415,6 +415,86 @@ struct OpZ {
     __device__ void finalize(const double *sums) const { finalize_beta(st, sums); }
 };
 
+// Operations for matrices with long rows, whose SpMVs are bound by the random operand
+// gathers: the operand vector is formed by an elementwise pass first (k_ep, k_er), so each
+// stored entry gathers one value instead of two.
+// Q': q = A p_new, partial p_new.q (p_new already formed).
+template <typename V, int K>
+struct OpQm {
+    using VV = V;
+    using IO = RowIO<V, K>;
+    static constexpr int NP = 1, NS = 0, NV = 1, NG = 1;
+    const V *pn;
+    V *q;
+    PcgState *st;
+    __device__ const V *row_vec(int) const { return pn; }
+    __host__ __device__ const V *gvec(int) const { return pn; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int) { return 0; }
+    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
+    __device__ void stage(double *) const {}
+    __device__ __forceinline__ V combine(const V (&g)[NG], int, const double *) const { return g[0]; }
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const { return pn[j * K + c]; }
+    __device__ __forceinline__ void operand_row(int64_t j, V (&o)[K], const double *) const
+    {
+        IO::load(pn + j * K, o);
+    }
+    __device__ __forceinline__ void load_rv(int, int64_t i, V (&o)[K]) const { IO::load(pn + i * K, o); }
+    template <int N, class RV>
+    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&part)[N],
+                                         const double *, const RV &rv) const
+    {
+        V qv[K];
+#pragma unroll
+        for (int c = 0; c < K; ++c) {
+            qv[c] = (V)acc[c];
+            part[c] += (double)rv.get(0, i, c) * (double)qv[c];
+        }
+        IO::store(q + i * K, qv);
+    }
+    __device__ void finalize(const double *sums) const { finalize_alpha(st, sums); }
+};
+
+// U_S': y = G^T r_new (r_new already formed, with the residual test).
+template <typename V, int K>
+struct OpUSm {
+    using VV = V;
+    using IO = RowIO<V, K>;
+    static constexpr int NP = 0, NS = 0, NV = 0, NG = 1;
+    const V *rn;
+    V *y;
+    PcgState *st;
+    __device__ const V *row_vec(int) const { return nullptr; }
+    __host__ __device__ const V *gvec(int) const { return rn; }
+    __host__ __device__ int gstride() const { return K; }
+    static __device__ constexpr int rv_src(int) { return -1; }
+    __device__ bool skip() const { return *(volatile int *)&st->all_done; }
+    __device__ void stage(double *) const {}
+    __device__ __forceinline__ V combine(const V (&g)[NG], int, const double *) const { return g[0]; }
+    __device__ __forceinline__ V operand(int64_t j, int c, const double *) const { return rn[j * K + c]; }
+    __device__ __forceinline__ void operand_row(int64_t j, V (&o)[K], const double *) const
+    {
+        IO::load(rn + j * K, o);
+    }
+    __device__ __forceinline__ void load_rv(int, int64_t, V (&o)[K]) const
+    {
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            o[c] = (V)0;
+    }
+    template <int N, class RV>
+    __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N], const double *,
+                                         const RV &) const
+    {
+        V yv[K];
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            yv[c] = (V)acc[c];
+        IO::store(y + i * K, yv);
+    }
+    __device__ void finalize(const double *) const {}
+};
+
 // U_J on row i: x += alpha p and r -= alpha q in the active columns, z = D^-1 r; adds r.r
 // to part[c] and r.z to part[K + c].  Stopped columns are rewritten with their own values.
 template <typename V, int K>
