@@ -16,6 +16,7 @@ CPU oracle on the host cores (bounded sample per step).
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import os
@@ -351,6 +352,8 @@ def run_ours(args):
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     total_iters = 0
     total_launch = 0
+    gc.collect()
+    gc.disable()            # no collector pause inside the timed region
     t_begin = clocks.mark()
     ev0.record()
     for k in range(args.steps):
@@ -361,6 +364,7 @@ def run_ours(args):
         total_launch += nl + 1
     ev1.record()
     torch.cuda.synchronize()
+    gc.enable()
     t_end = clocks.mark()
     barrier()
     clk = clocks.stop((t_begin, t_end)) if rank == 0 else {}
@@ -389,6 +393,8 @@ def run_ours(args):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e_iters = 0
+    gc.collect()
+    gc.disable()
     e0.record()
     for _ in range(args.steps):
         flush.zero_()
@@ -400,6 +406,7 @@ def run_ours(args):
         e_iters += it
     e1.record()
     torch.cuda.synchronize()
+    gc.enable()
     barrier()
     ems = e0.elapsed_time(e1)
     te = torch.tensor([ems, float(e_iters)], dtype=torch.float64, device=dev)

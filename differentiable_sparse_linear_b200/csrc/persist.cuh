@@ -86,6 +86,7 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
 
     __shared__ double s_red[(TB / 32) * NR];
     __shared__ double s_scal[2 * K + 1];
+    __shared__ double s_eps[1];
     __shared__ double s_sum[2 * NR];
     __shared__ PcgState s_st;
     __shared__ int s_abort, s_quit;
@@ -105,22 +106,52 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
         return;
     }
     volatile int *abort = &s_abort;
-    auto sync = [] { __syncthreads(); };
+    const int lane = tid & 31, warp = tid >> 5;
     int seq = 1;
     unsigned long long t_phase = 0;
     if (blockIdx.x == 0 && tid == 0)
         t_phase = global_ns();
+    // scalars of the operations, staged by thread 0 at the end of the phase before:
+    // s_scal = {alpha, active} for U_S / U_J, {beta} for Q; Z's eps is constant
+    auto stage_update = [&]() {
+        for (int c = 0; c < K; ++c) {
+            s_scal[c] = s_st.alpha[c];
+            s_scal[K + c] = s_st.active[c] ? 1.0 : 0.0;
+        }
+    };
+    auto stage_q = [&]() {
+        for (int c = 0; c < K; ++c)
+            s_scal[c] = s_st.beta[c];
+    };
+    if (tid == 0) {
+        s_eps[0] = s_st.eps;
+        stage_update();
+    }
+    __syncthreads();
 
-    // End of a phase, first half: block sum, publish it in this phase's slot (4 slots in
-    // turn: a slot is written again only after a barrier every reader of it has passed),
-    // grid barrier.  Returns the slot.
+    // End of a phase, first half: warp sums, then thread 0 adds the warps' sums in a fixed
+    // order, publishes the block's partial in this phase's slot (4 slots in turn: a slot is
+    // written again only after a barrier every reader of it has passed) and passes the
+    // grid barrier; the block waits for it.  Returns the slot.
     auto publish = [&](double (&part)[NR], int n, int kind) -> double * {
         double *slot = a.partials + (size_t)(seq & 3) * gridDim.x * NR;
-        block_sum<TB, NR>(part, s_red, tid, sync);
-        if (tid < n)
-            slot[(size_t)blockIdx.x * NR + tid] = part[0];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            double v = part[i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                v += __shfl_down_sync(0xffffffffu, v, off);
+            if (lane == 0)
+                s_red[warp * NR + i] = v;
+        }
         __syncthreads();
         if (tid == 0) {
+            for (int i = 0; i < n; ++i) {
+                double t = 0.0;
+                for (int w = 0; w < TB / 32; ++w)
+                    t += s_red[w * NR + i];
+                slot[(size_t)blockIdx.x * NR + i] = t;
+            }
             unsigned long long *bar = &a.st->gbar;
             const unsigned long long target = (unsigned long long)seq * gridDim.x;
             // release: the block's writes (ordered before this thread by the block barrier)
@@ -151,31 +182,43 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
         ++seq;
         return slot;
     };
-    // Second half: all blocks' partials of a slot, in block order, into out[0..n).
-    auto reduce = [&](const double *slot, int n, double *out) {
-        double v[NR];
+    // Second half, warp 0 only: all blocks' partials of up to two slots, in block order (lane
+    // l takes blocks l, l + 32, ...; then a fixed shuffle tree), into out[0..n) and
+    // out[n..2n); the same arithmetic in every block.
+    auto reduce_w0 = [&](const double *slot0, const double *slot1, int n, double *out) {
+        double v[NR], w[NR];
 #pragma unroll
-        for (int i = 0; i < NR; ++i)
+        for (int i = 0; i < NR; ++i) {
             v[i] = 0.0;
-        for (int b = tid; b < (int)gridDim.x; b += TB) {
+            w[i] = 0.0;
+        }
+        for (int b = lane; b < (int)gridDim.x; b += 32) {
 #pragma unroll
             for (int i = 0; i < NR; ++i)
-                if (i < n)
-                    v[i] += __ldcg(&slot[(size_t)b * NR + i]);
+                if (i < n) {
+                    v[i] += __ldcg(&slot0[(size_t)b * NR + i]);
+                    if (slot1)
+                        w[i] += __ldcg(&slot1[(size_t)b * NR + i]);
+                }
         }
-        block_sum<TB, NR>(v, s_red, tid, sync);
-        if (tid < n)
-            out[tid] = v[0];
-        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                v[i] += __shfl_down_sync(0xffffffffu, v[i], off);
+                w[i] += __shfl_down_sync(0xffffffffu, w[i], off);
+            }
+        }
+        if (lane == 0)
+            for (int i = 0; i < n; ++i) {
+                out[i] = v[i];
+                if (slot1)
+                    out[n + i] = w[i];
+            }
+        __syncwarp();
     };
-    auto phase_end = [&](double (&part)[NR], int n, int kind) { reduce(publish(part, n, kind), n, s_sum); };
-    // After thread 0 finalised: stop when every column is done or a wait ran out.
-    auto decide = [&]() -> bool {
-        if (tid == 0)
-            s_quit = s_st.all_done || *abort || *(volatile int *)a.err;
-        __syncthreads();
-        return s_quit != 0;
-    };
+    // thread 0, after finalising: stop when every column is done or a wait ran out
+    auto quit_now = [&]() { return s_st.all_done || *abort || *(volatile int *)a.err; };
 
     double part[NR];
     auto zero = [&]() {
@@ -187,68 +230,62 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
     // U_J over this block's rows: x += alpha p, r -= alpha q, z = D^-1 r; partials r.r
     // (0..K-1) and r.z (K..2K-1).  The block takes the rows of its run of slices.
     auto run_uj = [&](const VV *p) -> bool {
-        if (tid == 0) {
-            for (int c = 0; c < K; ++c) {
-                s_scal[c] = s_st.alpha[c];
-                s_scal[K + c] = s_st.active[c] ? 1.0 : 0.0;
-            }
-        }
-        __syncthreads();
         zero();
         const int64_t r0 = a.A.n_slices * blockIdx.x / gridDim.x * 32;
         const int64_t r1 = min(a.A.n, a.A.n_slices * (blockIdx.x + 1) / gridDim.x * 32);
         for (int64_t i = r0 + tid; i < r1; i += TB)
             jacobi_row<VV, K>(i, a.x, a.ra, p, a.q, a.z, a.dinv, s_scal, s_scal + K, part);
-        phase_end(part, 2 * K, PH_UJ);
-        if (tid == 0) {
-            finalize_residual(&s_st, s_sum);
-            finalize_beta(&s_st, s_sum + K);
+        const double *sl = publish(part, 2 * K, PH_UJ);
+        if (warp == 0) {
+            reduce_w0(sl, nullptr, 2 * K, s_sum);
+            if (lane == 0) {
+                finalize_residual(&s_st, s_sum);
+                finalize_beta(&s_st, s_sum + K);
+                stage_q();
+                s_quit = quit_now();
+            }
         }
-        return decide();
+        __syncthreads();
+        return s_quit != 0;
     };
     auto run_q = [&](bool odd) -> bool {
-        const auto op = P::opQ(a, odd, &s_st);
-        if (tid == 0)
-            op.stage(s_scal);
-        __syncthreads();
         zero();
-        sell_phase<K, VM, MAXL, TB, P::RS>(a.A, op, part, s_scal);
-        phase_end(part, K, PH_Q);
-        if (tid == 0)
-            finalize_alpha(&s_st, s_sum);
-        return decide();
+        sell_phase<K, VM, MAXL, TB, P::RS>(a.A, P::opQ(a, odd, &s_st), part, s_scal);
+        const double *sl = publish(part, K, PH_Q);
+        if (warp == 0) {
+            reduce_w0(sl, nullptr, K, s_sum);
+            if (lane == 0) {
+                finalize_alpha(&s_st, s_sum);
+                stage_update();
+                s_quit = quit_now();
+            }
+        }
+        __syncthreads();
+        return s_quit != 0;
     };
     // U_S then Z.  Z needs U_S's vectors (the barrier) but not its scalar, so U_S's
     // partials are reduced together with Z's at Z's end; U_S's residual test then decides
     // as before (a stop there leaves Z's results unused: x, r and the counts are U_S's).
     auto run_us_z = [&](bool odd) -> bool {
-        {
-            const auto op = P::opUS(a, odd, &s_st);
-            if (tid == 0)
-                op.stage(s_scal);
-            __syncthreads();
-            zero();
-            sell_phase<K, VM, MAXL, TB, P::RS>(a.GT, op, part, s_scal);
-        }
+        zero();
+        sell_phase<K, VM, MAXL, TB, P::RS>(a.GT, P::opUS(a, odd, &s_st), part, s_scal);
         const double *slot_us = publish(part, K, PH_US);
-        {
-            const auto op = P::opZ(a, odd, &s_st);
-            if (tid == 0)
-                op.stage(s_scal);
-            __syncthreads();
-            zero();
-            sell_phase<K, VM, MAXL, TB, P::RS>(a.G, op, part, s_scal);
-        }
+        zero();
+        sell_phase<K, VM, MAXL, TB, P::RS>(a.G, P::opZ(a, odd, &s_st), part, s_eps);
         const double *slot_z = publish(part, K, PH_Z);
-        reduce(slot_us, K, s_sum);
-        reduce(slot_z, K, s_sum + K);
-        if (tid == 0) {
-            finalize_residual(&s_st, s_sum);
-            signal_if_done(&s_st);
-            if (!s_st.all_done)
-                finalize_beta(&s_st, s_sum + K);
+        if (warp == 0) {
+            reduce_w0(slot_us, slot_z, K, s_sum);
+            if (lane == 0) {
+                finalize_residual(&s_st, s_sum);
+                signal_if_done(&s_st);
+                if (!s_st.all_done)
+                    finalize_beta(&s_st, s_sum + K);
+                stage_q();
+                s_quit = quit_now();
+            }
         }
-        return decide();
+        __syncthreads();
+        return s_quit != 0;
     };
 
     bool quit;
