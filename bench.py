@@ -463,6 +463,38 @@ def run_ours(args):
                     "peak_source": peak_kind, "algorithmic_bytes": launch_bytes, "ms_per_launch": launch_ms,
                     "units_per_launch": {nm: pcnt[slot[nm]] for nm in names},
                     "note": "one launch = one forward solve; bytes = per-phase algorithmic bytes x phases run"}
+    elif is_list:
+        # one launch of the list kernel = one batched solve (a block per system); bytes per
+        # system iteration in the streaming form: the system's matrix + 13 vector passes
+        sys_off = np.asarray(A.sys_row_off, dtype=np.int64)
+        sys_n = np.diff(sys_off)
+        sys_nnz = A.row_ptr[sys_off[1:]].astype(np.int64) - A.row_ptr[sys_off[:-1]].astype(np.int64)
+        sv = vbytes(w.dtype)
+        per_iter = sys_nnz * (sv + 4) + (sys_n + 1) * 4 + 13 * sys_n * sv
+        reps = 3
+        tot = 0.0
+        infos = None
+        for r in range(reps + 1):
+            flush.zero_()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record()
+            _, infos = sla.sla_pcg_solve_batched(Ad, M, b, X, rtol=w.tol)
+            s1.record()
+            torch.cuda.synchronize()
+            if r >= 1:
+                tot += s0.elapsed_time(s1)
+        launch_ms = tot / reps
+        its = np.array([i.iters for i in infos], dtype=np.int64)
+        launch_bytes = int((per_iter * its).sum())
+        ach = launch_bytes / (launch_ms * 1e6)
+        roofline = {"bound": "hbm", "kernel": "k_list_pcg", "achieved": ach, "peak": peak, "unit": "GB/s",
+                    "frac": ach / peak, "traffic": None, "peak_source": peak_kind,
+                    "algorithmic_bytes": launch_bytes, "ms_per_launch": launch_ms,
+                    "units_per_launch": {"system_iterations": int(its.sum())},
+                    "note": "one launch = one batched forward solve; bytes per system iteration = "
+                            "nnz_s*(s_v+4) + (n_s+1)*4 + 13*n_s*s_v (streaming form; the kernel keeps "
+                            "each system's vectors in shared memory)"}
     elif not is_list:
         kt = sla.sla_pcg_kernel_times(Ad, M, nrhs, reps=args.kernel_reps)
         names = list(kernel_bytes(w))

@@ -54,7 +54,12 @@ struct Persist {
     static constexpr int MINB = (K == 1 && MAXL == 8) ? 2 : 1;
     // slices per warp round (their loads in flight together): two where that fits the registers
     static constexpr int RS = (K == 1 || (K == 2 && sizeof(VV) == 4)) ? 2 : 1;
+    // wide rows (K >= 4 right-hand sides): p_new is formed in a phase of its own, so Q
+    // gathers one K-row per stored entry instead of two (the extra grid barrier costs far
+    // less than the gathers it saves)
+    static constexpr bool FORM_P = K >= 4;
     using OQ = OpQ<VV, K>;
+    using OQM = OpQm<VV, K>;
     using OUS = OpUS<VV, K>;
     using OZ = OpZ<VV, K>;
 
@@ -63,6 +68,10 @@ struct Persist {
     static __device__ __forceinline__ OQ opQ(const PersistArgs<VM, VV> &a, bool odd, PcgState *s)
     {
         return OQ{a.z, odd ? a.pb : a.pa, odd ? a.pa : a.pb, a.q, s};
+    }
+    static __device__ __forceinline__ OQM opQm(const PersistArgs<VM, VV> &a, bool odd, PcgState *s)
+    {
+        return OQM{odd ? a.pa : a.pb, a.q, s};
     }
     static __device__ __forceinline__ OUS opUS(const PersistArgs<VM, VV> &a, bool odd, PcgState *s)
     {
@@ -151,7 +160,7 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
                 for (int w = 0; w < TB / 32; ++w)
                     t += s_red[w * NR + i];
                 slot[(size_t)blockIdx.x * NR + i] = t;
-            }
+            }   // n == 0: a plain grid barrier
             unsigned long long *bar = &a.st->gbar;
             const unsigned long long target = (unsigned long long)seq * gridDim.x;
             // release: the block's writes (ordered before this thread by the block barrier)
@@ -171,7 +180,7 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
                     }
                 }
             }
-            if (blockIdx.x == 0) {
+            if (blockIdx.x == 0 && kind >= 0) {   // kind < 0: timed with the next phase
                 const unsigned long long t1 = global_ns();
                 s_st.phase_ns[kind] += t1 - t_phase;
                 s_st.phase_cnt[kind] += 1;
@@ -250,7 +259,27 @@ k_pcg_persistent(const PersistArgs<VM, VV> a)
     };
     auto run_q = [&](bool odd) -> bool {
         zero();
-        sell_phase<K, VM, MAXL, TB, P::RS>(a.A, P::opQ(a, odd, &s_st), part, s_scal);
+        if constexpr (P::FORM_P) {
+            // p_new = z + beta p_old over this block's rows, then a grid barrier
+            VV *pn = odd ? a.pa : a.pb;
+            const VV *po = odd ? a.pb : a.pa;
+            const int64_t r0 = a.A.n_slices * blockIdx.x / gridDim.x * 32;
+            const int64_t r1 = min(a.A.n, a.A.n_slices * (blockIdx.x + 1) / gridDim.x * 32);
+            using IO = RowIO<VV, K>;
+            for (int64_t i = r0 + tid; i < r1; i += TB) {
+                VV zz[K], pp[K], o[K];
+                IO::load(a.z + i * K, zz);
+                IO::load(po + i * K, pp);
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    o[c] = vfma<VV>(s_scal[c], pp[c], zz[c]);
+                IO::store(pn + i * K, o);
+            }
+            publish(part, 0, -1);
+            sell_phase<K, VM, MAXL, TB, P::RS>(a.A, P::opQm(a, odd, &s_st), part, s_scal);
+        } else {
+            sell_phase<K, VM, MAXL, TB, P::RS>(a.A, P::opQ(a, odd, &s_st), part, s_scal);
+        }
         const double *sl = publish(part, K, PH_Q);
         if (warp == 0) {
             reduce_w0(sl, nullptr, K, s_sum);
