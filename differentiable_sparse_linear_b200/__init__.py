@@ -253,11 +253,15 @@ def sla_pcg_solve(A: Matrix, M: Optional[Preconditioner], b: torch.Tensor,
 
 def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLdx: torch.Tensor, *,
                     want_dA: bool = True, rtol: float = 0.0, maxit: int = 0, vector_f64: bool = False,
-                    engine: str = "auto", stream=None):
-    """Returns (dL/db, dL/dA on A's pattern or None, info)."""
+                    engine: str = "auto", dLdb: Optional[torch.Tensor] = None,
+                    dLdA: Optional[torch.Tensor] = None, stream=None):
+    """Returns (dL/db, dL/dA on A's pattern or None, info); dLdb / dLdA: optional outputs."""
     _check_vec(A, dLdx, vector_f64)
-    dLdb = torch.empty_like(dLdx)
-    dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdx.device) if want_dA else None
+    dLdb = torch.empty_like(dLdx) if dLdb is None else dLdb
+    if want_dA and dLdA is None:
+        dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdx.device)
+    elif not want_dA:
+        dLdA = None
     info = _lib.sla_pcg_info()
     opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_adjoint(A.handle, _mh(M), _ptr(x), _ptr(dLdx), _ptr(dLdb), _ptr(dLdA),
@@ -295,12 +299,17 @@ def sla_pcg_solve_batched_noalloc(A: Matrix, M: Optional[Preconditioner], B: tor
 
 def sla_pcg_adjoint_batched(A: Matrix, M: Optional[Preconditioner], X: torch.Tensor, dLdX: torch.Tensor,
                             *, want_dA: bool = True, rtol: float = 0.0, maxit: int = 0,
-                            vector_f64: bool = False, engine: str = "auto", stream=None):
+                            vector_f64: bool = False, engine: str = "auto", dLdB: Optional[torch.Tensor] = None,
+                            dLdA: Optional[torch.Tensor] = None, stream=None):
+    """Returns (dL/dB, dL/dA on A's pattern or None, infos); dLdB / dLdA: optional outputs."""
     _check_vec(A, dLdX, vector_f64)
     nrhs = 1 if (dLdX.dim() == 1 or A.batch > 1) else dLdX.shape[1]
     count = A.batch if A.batch > 1 else nrhs
-    dLdB = torch.empty_like(dLdX)
-    dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdX.device) if want_dA else None
+    dLdB = torch.empty_like(dLdX) if dLdB is None else dLdB
+    if want_dA and dLdA is None:
+        dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdX.device)
+    elif not want_dA:
+        dLdA = None
     infos = (_lib.sla_pcg_info * count)()
     opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_adjoint_batched(A.handle, _mh(M), nrhs, _ptr(X), _ptr(dLdX), _ptr(dLdB),

@@ -188,8 +188,11 @@ sla_status ensure_windows(sla_csr *A, const TilePart *tp_c, int wmax, cudaStream
 }
 
 // Sliced copy (see SellPart).
-sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **out)
+sla_status ensure_sell(sla_csr *A, cudaStream_t s, const SellPart **out)
 {
+    // offsets per diagonal slice at most: the matrix's own row-length class (a kernel that
+    // reads the layout unrolls to at least this)
+    const int maxl = A->max_row_len <= 8 ? 8 : 16;
     if (A->sell && A->sell->maxl == maxl) {
         *out = A->sell;
         return SLA_SUCCESS;
@@ -223,9 +226,16 @@ sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **ou
                 }
             }
         }
-        if (slot_rows >= ((int64_t)1 << 27) || (int64_t)offs.size() >= ((int64_t)1 << 31) - maxl)
+        if (slot_rows >= ((int64_t)1 << 27) || (int64_t)offs.size() >= ((int64_t)1 << 30) - maxl)
             return fail(SLA_ERR_UNSUPPORTED, "matrix too large for the sliced layout");
         uint32_t w1 = 0;
+        // a diagonal slice is "full" when every row holds every offset of the list: entry u of
+        // row r is then CSR entry row_ptr[r] + u, so the product can skip the column indices
+        bool full = true;
+        if (diag && !u.empty())
+            for (int64_t r = sl * 32; r < std::min(n, sl * 32 + 32); ++r)
+                if ((int64_t)A->h_rp[(size_t)r + 1] - A->h_rp[(size_t)r] != (int64_t)u.size())
+                    full = false;
         if (diag && !u.empty()) {
             std::sort(u.begin(), u.end());
             // slices with the same offsets share one list (a stencil has a handful)
@@ -235,7 +245,7 @@ sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **ou
                 for (int64_t d : u)
                     offs.push_back((int32_t)d);
             }
-            w1 = (1u << 31) | it->second;
+            w1 = (1u << 31) | (full ? (1u << 30) : 0u) | it->second;
             L = (int64_t)u.size();
             slice_offs[(size_t)sl] = u;
             ++n_diag;

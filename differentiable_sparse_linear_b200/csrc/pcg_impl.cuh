@@ -392,9 +392,31 @@ struct TileLaunch {
     }
 };
 
+template <typename V, int K, int MAXL>
+static sla_status spmv_slices_k(const sla_csr *A, int nc, const void *x, void *y, cudaStream_t s)
+{
+    const SellPart *sp;
+    SLA_TRY(ensure_sell(const_cast<sla_csr *>(A), s, &sp));
+    auto kern = k_spmv_slices<V, K, MAXL>;
+    int per_sm = 0;
+    SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, SPS_T, 0));
+    const int64_t want = (sp->n_slices + 2 * (SPS_T / 32) - 1) / (2 * (SPS_T / 32));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)std::max(per_sm, 1) * A->num_sms));
+    kern<<<grid, SPS_T, 0, s>>>(A->n, sp->n_slices, sp->d_desc, sp->d_offs, A->rp, A->ci, (const V *)A->val,
+                                (const V *)x, (V *)y, nc, nc);
+    SLA_CUDA_TRY(cudaGetLastError());
+    return SLA_SUCCESS;
+}
+
 template <typename V, int K>
 static sla_status spmv_k(const sla_csr *A, int nc, const void *x, void *y, cudaStream_t s)
 {
+    // short rows: CSR-direct product over the slice descriptors
+    if (A->n > 0 && A->batch == 1 && A->max_row_len <= 16 && K <= 4) {
+        if (A->max_row_len <= 8)
+            return spmv_slices_k<V, K, 8>(A, nc, x, y, s);
+        return spmv_slices_k<V, K, 16>(A, nc, x, y, s);
+    }
     using Op = OpSpmv<V, K>;
     Op op{(const V *)x, (V *)y, nc, nc};
     TileLaunch<K, V, Op> L;
@@ -657,7 +679,7 @@ static sla_status persist_launch(sla_csr *A, Plan *p, cudaStream_t s)
     // solve, so values changed in place since the last solve are used
     auto sell = [&](const sla_csr *M_, SellView<VM> &v) -> sla_status {
         const SellPart *sp;
-        SLA_TRY(ensure_sell(const_cast<sla_csr *>(M_), MAXL, s, &sp));
+        SLA_TRY(ensure_sell(const_cast<sla_csr *>(M_), s, &sp));
         SLA_TRY(launch_sell_values(M_, sp, s));
         v.desc = sp->d_desc;
         v.offs = sp->d_offs;

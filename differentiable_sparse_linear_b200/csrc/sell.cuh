@@ -19,7 +19,7 @@ namespace sla {
 
 template <typename VM>
 struct SellView {
-    const uint2 *desc;         // per slice: {first slot row << 5 | L, diagonal << 31 | offsets}
+    const uint2 *desc;         // per slice: {first slot row << 5 | L, diagonal << 31 | full << 30 | offsets}
     const int32_t *offs;       // offset lists of the diagonal slices
     const uint8_t *lens;       // per row (index slices)
     const int16_t *idx16;      // column - row (rel16), or null
@@ -91,7 +91,7 @@ __device__ __forceinline__ void sell_phase(const SellView<VM> &m, const Op &op, 
             for (int c = 0; c < K; ++c)
                 s[q][c] = (Acc)0;
             if (d[q].y >> 31) {
-                const int32_t *of = m.offs + (d[q].y & 0x7fffffffu);
+                const int32_t *of = m.offs + (d[q].y & 0x3fffffffu);
 #pragma unroll
                 for (int u = 0; u < MAXL; ++u) {
                     if (u < L) {
@@ -132,6 +132,75 @@ __device__ __forceinline__ void sell_phase(const SellView<VM> &m, const Op &op, 
                     acc[c] = (double)s[q][c];
                 op.emit(row, acc, part, s_scal, rv[q]);
             }
+        }
+    }
+}
+
+// y = A x straight from the caller's CSR arrays (K right-hand sides with leading dimension
+// ld, columns c >= nc zero), using the slice descriptors only for the pattern: in a full
+// diagonal slice entry u of row r is CSR entry row_ptr[r] + u and its column is
+// r + offs[u], so the column indices are not read at all; other slices read them.  A warp
+// owns a slice (lane = row), a block a contiguous run of slices; two slices per round.
+constexpr int SPS_T = 256;
+
+template <typename V, int K, int MAXL>
+__global__ void __launch_bounds__(SPS_T)
+k_spmv_slices(int64_t n, int64_t n_slices, const uint2 *__restrict__ desc, const int32_t *__restrict__ offs,
+              const int32_t *__restrict__ rp, const int32_t *__restrict__ ci, const V *__restrict__ val,
+              const V *__restrict__ x, V *__restrict__ y, int ld, int nc)
+{
+    constexpr int NW = SPS_T / 32, RS = 2;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t s0 = n_slices * blockIdx.x / gridDim.x;
+    const int64_t s1 = n_slices * (blockIdx.x + 1) / gridDim.x;
+    for (int64_t sb = s0 + warp; sb < s1; sb += (int64_t)NW * RS) {
+        double acc[RS][K];
+#pragma unroll
+        for (int q = 0; q < RS; ++q) {
+            const int64_t sl = sb + (int64_t)q * NW;
+            const int64_t row = sl * 32 + lane;
+            const bool live = sl < s1 && row < n;
+            const uint2 d = sl < s1 ? desc[sl] : make_uint2(0u, 0u);
+            const int L = (int)(d.x & 31u);
+            const int32_t k0 = live ? rp[row] : 0;
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+                acc[q][c] = 0.0;
+            if ((d.y >> 30) == 3u) {
+                const int32_t *of = offs + (d.y & 0x3fffffffu);
+#pragma unroll
+                for (int u = 0; u < MAXL; ++u)
+                    if (live && u < L) {
+                        const int64_t j = row + of[u];
+                        const double a = (double)val[k0 + u];
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            if (c < nc)
+                                acc[q][c] = fma(a, (double)__ldg(&x[j * ld + c]), acc[q][c]);
+                    }
+            } else {
+                const int len = live ? rp[row + 1] - k0 : 0;
+#pragma unroll
+                for (int u = 0; u < MAXL; ++u)
+                    if (u < len) {
+                        const int64_t j = ci[k0 + u];
+                        const double a = (double)val[k0 + u];
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            if (c < nc)
+                                acc[q][c] = fma(a, (double)__ldg(&x[j * ld + c]), acc[q][c]);
+                    }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < RS; ++q) {
+            const int64_t sl = sb + (int64_t)q * NW;
+            const int64_t row = sl * 32 + lane;
+            if (sl < s1 && row < n)
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    if (c < nc)
+                        y[row * ld + c] = (V)acc[q][c];
         }
     }
 }

@@ -99,7 +99,9 @@ struct __align__(16) WinDesc {
 //   index slice: slot row u holds entry u of each row, with its column as a 16-bit offset
 //     from the row (rel16, when every offset of the matrix fits) or a 32-bit column, and
 //     per-row lengths.
-// desc[s] = {first slot row << 5 | L_s, diagonal << 31 | position of its offsets}.  Values
+// desc[s] = {first slot row << 5 | L_s, diagonal << 31 | full << 30 | position of its
+// offsets}; "full": every row of the slice holds every offset of the list, so entry u of row
+// r is CSR entry row_ptr[r] + u (the CSR-direct product uses that).  Values
 // are gathered from the CSR arrays by `perm` (slot -> CSR position, -1 for padding) before
 // each solve, so values changed in place are picked up.
 struct SellPart {
@@ -202,9 +204,9 @@ struct Plan {
 sla_status ensure_tiles(sla_csr *A, int D, int RMAX, cudaStream_t s, const TilePart **out);
 // Build (once) the operand windows of a tile partition, at most wmax rows per tile.
 sla_status ensure_windows(sla_csr *A, const TilePart *tp, int wmax, cudaStream_t s);
-// Build (once) the sliced copy of a short-row matrix (diagonal slices of at most maxl
-// offsets); gather its values.
-sla_status ensure_sell(sla_csr *A, int maxl, cudaStream_t s, const SellPart **out);
+// Build (once) the sliced copy of a short-row matrix (diagonal slices of at most 8 offsets,
+// 16 for rows of 9 to 16 entries); gather its values.
+sla_status ensure_sell(sla_csr *A, cudaStream_t s, const SellPart **out);
 sla_status launch_sell_values(const sla_csr *A, const SellPart *sp, cudaStream_t s);
 size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K, int vec64);
 sla_status get_plan(sla_csr *A, const sla_precond *M, int K, int vec64, Plan **out);

@@ -128,6 +128,9 @@ SLA_API const char *sla_last_error(void);
  * n_rows == n_cols is required (the solver works on square SPD systems); nnz = row_ptr[n].
  * d_row_ptr (n+1), d_col (nnz), d_val (nnz, `dtype`) are borrowed, not copied, and must be
  * 16-byte aligned (SLA_ERR_INVALID_ARG otherwise): the SpMV streams them by bulk copies.
+ * The pattern (d_row_ptr, d_col) must not change while the handle lives: the library
+ * derives row partitions and sliced layouts from it at first use.  The values may change
+ * between calls; every product and solve reads the current values. 
  * Set-up work (load-balanced tile partition of the rows, optional validation) runs on
  * `stream` and is synchronised before return.  Returns SLA_ERR_INVALID_CSR on a pattern
  * that fails SLA_VALIDATE. */
