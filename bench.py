@@ -217,6 +217,22 @@ def cpu_baseline(w, budget_s: float = 15.0) -> dict:
                       f"({dt:.1f} s, one host thread)"}
 
 
+# ------------------------------------------------------------------------- ranks
+def reduce_over_ranks(ms: float, iters: float, world: int, device) -> tuple[float, float]:
+    """Whole-job numbers of a replicated run: the slowest rank's time and the iterations of
+    all ranks (each rank solves its own replica).  One rank: the inputs unchanged."""
+    if world <= 1:
+        return float(ms), float(iters)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms), float(iters)], dtype=torch.float64, device=device)
+    tm = t.clone()
+    dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    ti = t.clone()
+    dist.all_reduce(ti, op=dist.ReduceOp.SUM)
+    return float(tm[0]), float(ti[1])
+
+
 # ------------------------------------------------------------------------- reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -384,15 +400,7 @@ def run_ours(args):
     clk = clocks.stop((t_begin, t_end)) if rank == 0 else {}
     ms = ev0.elapsed_time(ev1)
     step_ms = [ev0.elapsed_time(evs[0])] + [evs[k - 1].elapsed_time(evs[k]) for k in range(1, args.steps)]
-    t = torch.tensor([ms, float(total_iters)], dtype=torch.float64, device=dev)
-    if world > 1:
-        tm = t.clone()
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        ti = t.clone()
-        dist.all_reduce(ti, op=dist.ReduceOp.SUM)
-        ms_max, iters_all = float(tm[0]), float(ti[1])
-    else:
-        ms_max, iters_all = ms, float(total_iters)
+    ms_max, iters_all = reduce_over_ranks(ms, total_iters, world, dev)
     value = iters_all / (ms_max / 1e3)
 
     # end to end: host inputs in pinned memory, result read back every step
@@ -423,13 +431,7 @@ def run_ours(args):
     gc.enable()
     barrier()
     ems = e0.elapsed_time(e1)
-    te = torch.tensor([ems, float(e_iters)], dtype=torch.float64, device=dev)
-    if world > 1:
-        tm = te.clone()
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        ti = te.clone()
-        dist.all_reduce(ti, op=dist.ReduceOp.SUM)
-        ems, e_iters = float(tm[0]), float(ti[1])
+    ems, e_iters = reduce_over_ranks(ems, e_iters, world, dev)
     e2e = {"value": e_iters / (ems / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": int(hb.numel() * hb.element_size() + hw.numel() * hw.element_size()),
            "d2h_bytes_per_step": int(hx.numel() * hx.element_size() + hl.numel() * hl.element_size())}
