@@ -27,7 +27,7 @@ import sla_workloads as W  # noqa: E402
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--config", type=int, default=2)
-    ap.add_argument("--size", default="full", choices=["full", "small", "tiny"])
+    ap.add_argument("--size", default="full", choices=["full", "medium", "small", "tiny"])
     ap.add_argument("--engine", default="auto", choices=["auto", "graph", "persistent"])
     ap.add_argument("--maxit", type=int, default=0)
     ap.add_argument("--solves", type=int, default=1)

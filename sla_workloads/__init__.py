@@ -367,8 +367,12 @@ def workload(cfg: int, size: str = "full") -> Workload:
     size="full" gives the stated sizes.  size="small" keeps each recipe (pattern law,
     value law, precision, preconditioner, tolerance, seeds) at a size the fp64 oracle
     finishes in seconds.  size="tiny" is smaller still, for exhaustive CPU checks.
+    size="medium" (workload 5 only) is a quarter of the full system -- still larger than
+    a GPU's L2 but a few hundred MB on the device -- for profiler captures.
     """
-    small = size != "full"
+    if size == "medium" and cfg != 5:
+        raise ValueError("size 'medium' is defined for workload 5 only")
+    small = size not in ("full", "medium")
     tiny = size == "tiny"
     if cfg == 1:
         N = 64 if not tiny else 12
@@ -402,10 +406,10 @@ def workload(cfg: int, size: str = "full") -> Workload:
                         rhs_uniform(4001, N, dtype=np.float64), rhs_uniform(4002, N, dtype=np.float64),
                         1e-10, "jacobi", dtype=np.float64, info={"nsys": nsys, "n": n})
     if cfg == 5:
-        n = 4194304 if not small else (49152 if not tiny else 600)
+        n = (4194304 if size == "full" else 1048576) if not small else (49152 if not tiny else 600)
         A = powerlaw_spd(n, seed=5000, dtype=np.float32)
         G = spai_factor_G(A, seed=5003, dtype=np.float32)
-        return Workload(CONFIG_NAMES[5] if not small else f"powerlaw_{n}_f32_spai", A,
+        return Workload(CONFIG_NAMES[5] if size == "full" else f"powerlaw_{n}_f32_spai", A,
                         rhs_normal(5001, n, np.float32), rhs_uniform(5002, n, dtype=np.float32),
                         1e-6, "spai", G=G, eps=3e-3, dtype=np.float32, info={"n": n})
     raise ValueError(f"unknown workload {cfg}")
