@@ -1,7 +1,7 @@
 """One solve of a seeded workload, for profiler captures (ncu) of the solver kernels.
 
     python -m differentiable_sparse_linear_b200.profile_run --config 2 [--size full]
-        [--engine auto|graph|persistent] [--maxit N] [--solves S]
+        [--engine auto|graph|persistent] [--maxit N] [--solves S] [--kernel-times R]
 
 Builds the workload's matrices and preconditioner on cuda:0, runs S forward solves (the
 first one also sets the solver up) with an optional iteration cap, so a capture of the
@@ -31,6 +31,9 @@ def main(argv=None) -> int:
     ap.add_argument("--engine", default="auto", choices=["auto", "graph", "persistent"])
     ap.add_argument("--maxit", type=int, default=0)
     ap.add_argument("--solves", type=int, default=1)
+    ap.add_argument("--kernel-times", type=int, default=0,
+                    help="then launch one iteration's kernels alone this many times (graph engine: "
+                         "profilers do not see the kernels of a graph with a conditional node)")
     a = ap.parse_args(argv)
     w = W.workload(a.config, a.size)
     d = torch.device("cuda", 0)
@@ -57,6 +60,10 @@ def main(argv=None) -> int:
         torch.cuda.synchronize()
         print(f"solve {s}: {w.name} iters {[i.iters for i in infos][:8]} status "
               f"{sorted(set(i.status for i in infos))} engine {infos[0].engine}", flush=True)
+    if a.kernel_times > 0 and w.A.sys_row_off is None:
+        ms = sla.sla_pcg_kernel_times(Ad, M, w.nrhs, reps=a.kernel_times)
+        torch.cuda.synchronize()
+        print(f"kernel times (ms): {[round(t, 4) for t in ms]}", flush=True)
     return 0
 
 
