@@ -325,6 +325,9 @@ struct TileLaunch {
     using LR = RowTmaLayout<K, VM, typename Op::VV, Op::NG>;
     static constexpr int RTHREADS = RowTmaCfg<K>::TC + 32;
     static constexpr size_t RSMEM = RowTmaCfg<K>::NST * LR::BYTES;
+    // long-row matrices: warp-owned tiles up to 4 right-hand sides, block-owned tiles above
+    // (a warp's share of shared memory no longer holds a useful tile there)
+    static constexpr bool WARP_TILES = K <= 4;
     int grid = 0;
     int maxl = 0;                 // 0: tile engine; else the short-row engine's MAXL
     MatView<VM> m{};
@@ -363,11 +366,17 @@ struct TileLaunch {
             return setup_rows<16>(A, s);
         }
         const TilePart *tp;
-        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), Tile2Cfg<K>::D, Tile2Cfg<K>::RMAX, s, &tp));
-        m = view<VM>(A, tp);
-        auto kern = k_tile2<K, VM, Op>;
         int per_sm = 0;
-        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Tile2Cfg<K>::T, 0));
+        if constexpr (WARP_TILES) {
+            SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), WTileCfg<K>::D, WTileCfg<K>::D, s, &tp));
+            SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_wtile<K, VM, Op>,
+                                                                       WTileCfg<K>::T, 0));
+        } else {
+            SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), Tile2Cfg<K>::D, Tile2Cfg<K>::RMAX, s, &tp));
+            SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_tile2<K, VM, Op>,
+                                                                       Tile2Cfg<K>::T, 0));
+        }
+        m = view<VM>(A, tp);
         per_sm = std::max(per_sm, 1);
         grid = std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
         maxl = 0;
@@ -387,7 +396,12 @@ struct TileLaunch {
         case 6: k_rows_tma<K, VM, 6, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         case 8: k_rows_tma<K, VM, 8, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         case 16: k_rows_tma<K, VM, 16, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
-        default: k_tile2<K, VM, Op><<<grid, Tile2Cfg<K>::T, 0, s>>>(m, op, part, st); break;
+        default:
+            if constexpr (WARP_TILES)
+                k_wtile<K, VM, Op><<<grid, WTileCfg<K>::T, 0, s>>>(m, op, part, st);
+            else
+                k_tile2<K, VM, Op><<<grid, Tile2Cfg<K>::T, 0, s>>>(m, op, part, st);
+            break;
         }
     }
 };

@@ -424,4 +424,171 @@ k_tile2(const MatView<VM> m, const Op op, double *partials, PcgState *st)
         grid_reduce_finalize<T, NPK>(part, partials, st, op, s_red, &s_flag, s_sum, tid, sync);
 }
 
+// ------------------------------------------------------------------ warp-tile kernel
+// The same decomposition with a warp as the unit: each warp takes whole tiles of at most D
+// items (rows + entries; 8 per lane for one right-hand side), forms the products, splits
+// the items over its lanes along the merge path and finishes rows that span lanes with a
+// fixed-order carry walk -- all under warp barriers, so no block barrier stalls one warp on
+// another.  A row longer than a tile is streamed by one warp, 8 entries per lane per step,
+// and reduced with a fixed shuffle tree.  Tiles go to warps round-robin over the grid.
+template <int K>
+struct WTileCfg {
+    static constexpr int T = 256;                        // threads per block
+    static constexpr int D = K == 1 ? 256 : K == 2 ? 128 : 64;   // <= 2^15: 16-bit row ends
+    static constexpr int MINB = K == 1 ? 8 : K == 2 ? 4 : 1;
+};
+
+template <int K, typename VM, class Op>
+__global__ void __launch_bounds__(WTileCfg<K>::T, WTileCfg<K>::MINB)
+k_wtile(const MatView<VM> m, const Op op, double *partials, PcgState *st)
+{
+    constexpr int T = WTileCfg<K>::T;
+    constexpr int NW = T / 32;
+    constexpr int D = WTileCfg<K>::D;
+    constexpr int EPL = D / 32;                          // entries per lane
+    constexpr int NPK = Op::NP * K;
+    constexpr int NR = NPK > K ? NPK : K;
+    using VV = typename Op::VV;
+
+    __shared__ double s_prod[NW][D * K];
+    __shared__ int16_t s_rp[NW][D + 1];        // row ends relative to the tile's first entry
+    __shared__ int32_t s_crow[NW][32];
+    __shared__ double s_cval[NW][32 * K];
+    __shared__ double s_red[NW * NR];
+    __shared__ double s_scal[Op::NS > 0 ? Op::NS : 1];
+    __shared__ double s_sum[NR];
+    __shared__ int s_flag;
+
+    if (op.skip())
+        return;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0)
+        op.stage(s_scal);
+    __syncthreads();
+    GlobalRows<Op, K> rv{op};
+    double part[NPK > 0 ? NPK : 1];
+#pragma unroll
+    for (int i = 0; i < (NPK > 0 ? NPK : 1); ++i)
+        part[i] = 0.0;
+    double *prod = s_prod[wid];
+    int16_t *rpp = s_rp[wid];
+
+    const int gw = blockIdx.x * NW + wid, nw = gridDim.x * NW;
+    for (int t = gw; t < m.n_tiles; t += nw) {
+        const int2 d0 = m.desc[t], d1 = m.desc[t + 1];
+        const int r0 = d0.x, r1 = d1.x;
+        const int64_t k0 = (int64_t)(uint32_t)d0.y, k1 = (int64_t)(uint32_t)d1.y;
+        const int nr = r1 - r0;
+        if ((int64_t)nr + (k1 - k0) > D) {
+            // one long row: lane-strided partial sums, all of a step's loads in flight
+            double lacc[K];
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+                lacc[c] = 0.0;
+            for (int64_t kb = k0; kb < k1; kb += 32 * EPL) {
+#pragma unroll
+                for (int u = 0; u < EPL; ++u) {
+                    const int64_t e = kb + lane + 32 * u;
+                    if (e < k1) {
+                        const double a = (double)m.val[e];
+                        VV o[K];
+                        op.operand_row(m.ci[e], o, s_scal);
+#pragma unroll
+                        for (int c = 0; c < K; ++c)
+                            lacc[c] = fma(a, (double)o[c], lacc[c]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    lacc[c] += __shfl_down_sync(0xffffffffu, lacc[c], off);
+            if (lane == 0)
+                op.emit(r0, lacc, part, s_scal, rv);
+            continue;
+        }
+        const int nk = (int)(k1 - k0);
+        // 1. products (matrix loads, then gathers, all in flight) and row ends
+#pragma unroll
+        for (int u = 0; u < EPL; ++u) {
+            const int e = lane + 32 * u;
+            if (e < nk) {
+                const double a = (double)m.val[k0 + e];
+                VV o[K];
+                op.operand_row(m.ci[k0 + e], o, s_scal);
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    prod[e * K + c] = a * (double)o[c];
+            }
+        }
+        for (int x = lane; x <= nr; x += 32)
+            rpp[x] = (int16_t)((int64_t)m.rp[r0 + x] - k0);
+        __syncwarp();
+        // 2. merge-path split of the tile's items over the lanes
+        const int items = nr + nk;
+        const int ipt = (items + 31) / 32;
+        const int d0i = min(lane * ipt, items);
+        const int d1i = min(d0i + ipt, items);
+        int lo = max(0, d0i - nk), hi = min(d0i, nr);
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (rpp[mid] <= d0i - mid)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        int r = lo, k = d0i - lo;
+        double acc[K], facc[K];
+#pragma unroll
+        for (int c = 0; c < K; ++c) {
+            acc[c] = 0.0;
+            facc[c] = 0.0;
+        }
+        int frow = -1;
+        for (int d = d0i; d < d1i; ++d) {
+            if (k < rpp[r + 1]) {
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    acc[c] += prod[k * K + c];
+                ++k;
+            } else {
+                if (frow < 0) {
+                    frow = r;
+#pragma unroll
+                    for (int c = 0; c < K; ++c)
+                        facc[c] = acc[c];
+                } else {
+                    op.emit(r0 + r, acc, part, s_scal, rv);
+                }
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    acc[c] = 0.0;
+                ++r;
+            }
+        }
+        // 3. rows spanning lanes: the lane holding a row's end adds the partial sums the
+        //    earlier lanes left, in a fixed order
+        s_crow[wid][lane] = (r < nr) ? r : -1;
+#pragma unroll
+        for (int c = 0; c < K; ++c)
+            s_cval[wid][lane * K + c] = acc[c];
+        __syncwarp();
+        if (frow >= 0) {
+            for (int u = lane - 1; u >= 0 && s_crow[wid][u] == frow; --u) {
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    facc[c] += s_cval[wid][u * K + c];
+            }
+            op.emit(r0 + frow, facc, part, s_scal, rv);
+        }
+        __syncwarp();
+    }
+
+    if constexpr (NPK > 0) {
+        auto sync = [] { __syncthreads(); };
+        grid_reduce_finalize<T, NPK>(part, partials, st, op, s_red, &s_flag, s_sum, tid, sync);
+    }
+}
+
 }  // namespace sla
