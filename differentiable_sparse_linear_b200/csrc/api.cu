@@ -3,6 +3,7 @@
 
 #include <algorithm>
 #include <map>
+#include <memory>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -164,6 +165,49 @@ static bool window_for_rows(const sla_csr *A, int64_t r0, int64_t r1, int wmax, 
     return true;
 }
 
+sla_status ensure_groups(sla_csr *A, cudaStream_t s, const GroupPart **out)
+{
+    if (A->groups) {
+        *out = A->groups;
+        return SLA_SUCCESS;
+    }
+    std::vector<int32_t> bin_rows[GBINS];
+    for (int64_t r = 0; r < A->n; ++r) {
+        const int64_t len = (int64_t)A->h_rp[(size_t)r + 1] - A->h_rp[(size_t)r];
+        int b = GBINS - 1;                  // G = 1
+        while (b > 0 && 4 * (int64_t(1) << (GBINS - 1 - b)) < len)
+            --b;
+        bin_rows[b].push_back((int32_t)r);
+    }
+    auto len_of = [&](int32_t r) { return A->h_rp[(size_t)r + 1] - A->h_rp[(size_t)r]; };
+    std::stable_sort(bin_rows[0].begin(), bin_rows[0].end(),
+                     [&](int32_t a, int32_t b) { return len_of(a) > len_of(b); });
+    auto gp = std::make_unique<GroupPart>();
+    std::vector<int4> rows;
+    rows.reserve((size_t)A->n);
+    int tasks = 0;
+    for (int b = 0; b < GBINS; ++b) {
+        const int per_task = 1 << b;        // 32 / G rows per warp task
+        gp->task0[b] = tasks;
+        gp->pos0[b] = (int)rows.size();
+        tasks += (int)((bin_rows[b].size() + per_task - 1) / per_task);
+        for (int32_t r : bin_rows[b])
+            rows.push_back(make_int4(r, A->h_rp[(size_t)r], A->h_rp[(size_t)r + 1], 0));
+    }
+    gp->task0[GBINS] = tasks;
+    gp->pos0[GBINS] = (int)rows.size();
+    gp->n_tasks = tasks;
+    if (!rows.empty()) {
+        SLA_CUDA_TRY(cudaMalloc((void **)&gp->d_rows, rows.size() * sizeof(int4)));
+        SLA_CUDA_TRY(cudaMemcpyAsync(gp->d_rows, rows.data(), rows.size() * sizeof(int4),
+                                     cudaMemcpyHostToDevice, s));
+        SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    }
+    A->groups = gp.release();
+    *out = A->groups;
+    return SLA_SUCCESS;
+}
+
 // Operand windows of every tile of a partition (tiles that do not fit get nseg = 0 and
 // gather from global memory).  Windows end inside the vectors (row n at most), since the
 // gathered vectors can be the caller's.
@@ -282,6 +326,11 @@ sla_status ensure_sell(sla_csr *A, cudaStream_t s, const SellPart **out)
                     i32[e] = (int32_t)j;
             }
         }
+    }
+    if (A->groups) {
+        cudaFree(A->groups->d_rows);
+        delete A->groups;
+        A->groups = nullptr;
     }
     if (A->sell) {
         cudaFree(A->sell->d_desc);

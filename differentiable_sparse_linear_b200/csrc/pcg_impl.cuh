@@ -309,15 +309,16 @@ static MatView<V> view(const sla_csr *A, const TilePart *tp)
     m.rp = A->rp;
     m.ci = A->ci;
     m.val = (const V *)A->val;
-    m.desc = tp->d_desc;
-    m.n_tiles = tp->n_tiles;
+    m.desc = tp ? tp->d_desc : nullptr;
+    m.n_tiles = tp ? tp->n_tiles : 0;
     m.n = A->n;
     m.nnz = A->nnz;
     return m;
 }
 
 // Launch configuration of one fused SpMV operation: the short-row engine when every row
-// holds at most 16 entries, the load-balanced tile engine otherwise.
+// holds at most 16 entries; otherwise the lane-group engine up to 4 right-hand sides and
+// the load-balanced tile engine above.
 constexpr int ROWS_MAXL = 16;
 
 template <int K, typename VM, class Op>
@@ -325,13 +326,14 @@ struct TileLaunch {
     using LR = RowTmaLayout<K, VM, typename Op::VV, Op::NG>;
     static constexpr int RTHREADS = RowTmaCfg<K>::TC + 32;
     static constexpr size_t RSMEM = RowTmaCfg<K>::NST * LR::BYTES;
-    // long-row matrices: warp-owned tiles up to 4 right-hand sides, block-owned tiles above
-    // (a warp's share of shared memory no longer holds a useful tile there)
-    static constexpr bool WARP_TILES = K <= 4;
+    // long-row matrices: rows grouped by length, a lane group per row, up to 4 right-hand
+    // sides; above that, block-owned tiles (a lane's gathers would not fit its registers)
+    static constexpr bool LANE_GROUPS = K <= 4;
     int grid = 0;
-    int maxl = 0;                 // 0: tile engine; else the short-row engine's MAXL
+    int maxl = 0;                 // 0: tile engine; -1: lane-group engine; else the short-row MAXL
     MatView<VM> m{};
     const WinDesc *win = nullptr; // operand windows (short-row engine, K <= 2)
+    GroupView gv{};               // length-grouped rows (lane-group engine)
 
     template <int MAXL>
     sla_status setup_rows(const sla_csr *A, cudaStream_t s)
@@ -365,17 +367,29 @@ struct TileLaunch {
                 return setup_rows<8>(A, s);
             return setup_rows<16>(A, s);
         }
-        const TilePart *tp;
         int per_sm = 0;
-        if constexpr (WARP_TILES) {
-            SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), WTileCfg<K>::D, WTileCfg<K>::D, s, &tp));
-            SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_wtile<K, VM, Op>,
-                                                                       WTileCfg<K>::T, 0));
-        } else {
-            SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), Tile2Cfg<K>::D, Tile2Cfg<K>::RMAX, s, &tp));
-            SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_tile2<K, VM, Op>,
-                                                                       Tile2Cfg<K>::T, 0));
+        if constexpr (LANE_GROUPS) {
+            const GroupPart *gp;
+            SLA_TRY(ensure_groups(const_cast<sla_csr *>(A), s, &gp));
+            m = view<VM>(A, nullptr);
+            gv.rows = gp->d_rows;
+            for (int b = 0; b <= GBINS; ++b) {
+                gv.task0[b] = gp->task0[b];
+                gv.pos0[b] = gp->pos0[b];
+            }
+            gv.n_tasks = gp->n_tasks;
+            SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_rowgroup<K, VM, Op>,
+                                                                       GroupCfg<K>::T, 0));
+            per_sm = std::max(per_sm, 1);
+            const int per_block = GroupCfg<K>::T / 32;
+            grid = std::max(1, std::min((gp->n_tasks + per_block - 1) / per_block, per_sm * A->num_sms));
+            maxl = -1;
+            return SLA_SUCCESS;
         }
+        const TilePart *tp;
+        SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), Tile2Cfg<K>::D, Tile2Cfg<K>::RMAX, s, &tp));
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_tile2<K, VM, Op>,
+                                                                   Tile2Cfg<K>::T, 0));
         m = view<VM>(A, tp);
         per_sm = std::max(per_sm, 1);
         grid = std::max(1, std::min(tp->n_tiles, per_sm * A->num_sms));
@@ -384,7 +398,7 @@ struct TileLaunch {
     }
     void launch(cudaStream_t s, const Op &op, double *part, PcgState *st, int *err) const
     {
-        if (m.n_tiles == 0)
+        if (maxl == -1 ? gv.n_tasks == 0 : m.n_tiles == 0)
             return;
         // windows are bulk-copied from the gathered vectors: they need 16-byte alignment
         bool aligned = true;
@@ -396,10 +410,12 @@ struct TileLaunch {
         case 6: k_rows_tma<K, VM, 6, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         case 8: k_rows_tma<K, VM, 8, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         case 16: k_rows_tma<K, VM, 16, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
+        case -1:
+            if constexpr (LANE_GROUPS)
+                k_rowgroup<K, VM, Op><<<grid, GroupCfg<K>::T, 0, s>>>(m, gv, op, part, st);
+            break;
         default:
-            if constexpr (WARP_TILES)
-                k_wtile<K, VM, Op><<<grid, WTileCfg<K>::T, 0, s>>>(m, op, part, st);
-            else
+            if constexpr (!LANE_GROUPS)
                 k_tile2<K, VM, Op><<<grid, Tile2Cfg<K>::T, 0, s>>>(m, op, part, st);
             break;
         }
@@ -487,7 +503,7 @@ struct PlanKernels {
         part = p->partials;
         err = &p->st->error;
         SLA_TRY(LQ.setup(A, s));
-        formA = LQ.maxl == 0;
+        formA = LQ.maxl <= 0;
         if (formA)
             SLA_TRY(LQm.setup(A, s));
         gv = vec_grid(A);
@@ -498,7 +514,7 @@ struct PlanKernels {
         if (p->kind == 2) {
             SLA_TRY(LZ.setup(M->G, s));
             SLA_TRY(LUS.setup(M->GT, s));
-            formGT = LUS.maxl == 0;
+            formGT = LUS.maxl <= 0;
             if (formGT)
                 SLA_TRY(LUSm.setup(M->GT, s));
         }

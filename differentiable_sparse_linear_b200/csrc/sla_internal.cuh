@@ -77,6 +77,19 @@ struct TilePart {
     int win_rows = -1;                     // WMAX the windows were built for (-1: not built)
 };
 
+// Rows of a long-row matrix grouped by length for the lane-group SpMV: a row of len entries
+// goes to a group of G lanes, G the smallest power of two with 4 G >= len (G = 1 up to 32;
+// rows longer than 128 entries get a whole warp).  The rows of one G form a bin; bins are
+// ordered G = 32, 16, ..., 1, and a warp task is 32 / G consecutive rows of one bin.  In
+// the G = 32 bin rows are ordered by length, longest first, elsewhere by index.
+constexpr int GBINS = 6;
+struct GroupPart {
+    int n_tasks = 0;
+    int task0[GBINS + 1] = {};             // first task of each bin; task0[GBINS] = n_tasks
+    int pos0[GBINS + 1] = {};              // first row position of each bin
+    int4 *d_rows = nullptr;                // per position: {row, first entry, end entry, 0}
+};
+
 // Operand window of a tile of a banded matrix: the tile's columns (and its own rows) lie in
 // nseg ranges of rows [a[s], a[s] + l[s]) of the gathered vectors, 4-row aligned; nseg = 0
 // means the tile gathers from global memory.
@@ -156,6 +169,7 @@ struct sla_csr {
     std::vector<int32_t> h_ci;             // host copy of col (short-row matrices, for windows)
     std::map<int, sla::TilePart> tiles;    // by item budget D
     sla::SellPart *sell = nullptr;         // sliced ELL copy (persistent solver)
+    sla::GroupPart *groups = nullptr;      // rows grouped by length (long-row matrices)
     int device = 0;
     int num_sms = 148;
     std::vector<sla::Plan *> plans;
@@ -207,6 +221,8 @@ sla_status ensure_windows(sla_csr *A, const TilePart *tp, int wmax, cudaStream_t
 // Build (once) the sliced copy of a short-row matrix (diagonal slices of at most 8 offsets,
 // 16 for rows of 9 to 16 entries); gather its values.
 sla_status ensure_sell(sla_csr *A, cudaStream_t s, const SellPart **out);
+// Build (once) the length-grouped row list of a matrix.
+sla_status ensure_groups(sla_csr *A, cudaStream_t s, const GroupPart **out);
 sla_status launch_sell_values(const sla_csr *A, const SellPart *sp, cudaStream_t s);
 size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K, int vec64);
 sla_status get_plan(sla_csr *A, const sla_precond *M, int K, int vec64, Plan **out);

@@ -19,7 +19,12 @@
 //   the merge path of (row ends, entries) -- the merge-based SpMV decomposition -- and
 //   each thread sums its run; a row spanning threads is finished by the thread holding its
 //   end, which adds the partial sums the earlier threads left, in a fixed order.  Several
-//   blocks per SM hide the latency.
+//   blocks per SM hide the latency.  Used above 4 right-hand sides.
+// * k_rowgroup, the SpMV with fused row epilogues for long-row matrices up to 4 right-hand
+//   sides: rows binned by length (GroupPart), a lane group sized to the row owns it and
+//   reduces with a fixed shuffle tree.  No shared-memory staging and no block barrier: a
+//   stored entry costs its two loads, its gather and one FMA, where the tile kernel also
+//   spends a merge-path split and a carry walk on it.
 #pragma once
 
 #include "sla_internal.cuh"
@@ -424,36 +429,61 @@ k_tile2(const MatView<VM> m, const Op op, double *partials, PcgState *st)
         grid_reduce_finalize<T, NPK>(part, partials, st, op, s_red, &s_flag, s_sum, tid, sync);
 }
 
-// ------------------------------------------------------------------ warp-tile kernel
-// The same decomposition with a warp as the unit: each warp takes whole tiles of at most D
-// items (rows + entries; 8 per lane for one right-hand side), forms the products, splits
-// the items over its lanes along the merge path and finishes rows that span lanes with a
-// fixed-order carry walk -- all under warp barriers, so no block barrier stalls one warp on
-// another.  A row longer than a tile is streamed by one warp, 8 entries per lane per step,
-// and reduced with a fixed shuffle tree.  Tiles go to warps round-robin over the grid.
-template <int K>
-struct WTileCfg {
-    static constexpr int T = 256;                        // threads per block
-    static constexpr int D = K == 1 ? 256 : K == 2 ? 128 : 64;   // <= 2^15: 16-bit row ends
-    static constexpr int MINB = K == 1 ? 8 : K == 2 ? 4 : 1;
+// ------------------------------------------------------------------ lane-group kernel
+// Rows grouped by length (GroupPart): a group of G lanes owns a row, each lane takes the
+// row's entries G apart (up to 4 per pass for G < 32, 8 per pass for whole-warp rows; all
+// of a pass's loads in flight) and the group sums its lanes with a fixed xor-shuffle tree.
+// A warp takes one task (32 / G rows of one bin) at a time, the tasks round-robin over the
+// grid's warps; the next task's row list entries are loaded while the current one runs.
+struct GroupView {
+    const int4 *rows;
+    int task0[GBINS + 1];
+    int pos0[GBINS + 1];
+    int n_tasks;
 };
 
-template <int K, typename VM, class Op>
-__global__ void __launch_bounds__(WTileCfg<K>::T, WTileCfg<K>::MINB)
-k_wtile(const MatView<VM> m, const Op op, double *partials, PcgState *st)
+template <int K>
+struct GroupCfg {
+    static constexpr int T = 256;
+    static constexpr int MINB = K == 1 ? 6 : K == 2 ? 5 : 4;
+};
+
+template <int U, int K, typename VM, class Op>
+__device__ __forceinline__ void group_row_sum(const MatView<VM> &m, const Op &op, int k, int k1, int G,
+                                              const double *s_scal, double (&acc)[K])
 {
-    constexpr int T = WTileCfg<K>::T;
+    using VV = typename Op::VV;
+    for (; k < k1; k += U * G) {
+        VM a[U];
+        int32_t j[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = k + u * G;
+            a[u] = e < k1 ? m.val[e] : (VM)0;
+            j[u] = e < k1 ? m.ci[e] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (j[u] >= 0) {
+                VV o[K];
+                op.operand_row(j[u], o, s_scal);
+#pragma unroll
+                for (int c = 0; c < K; ++c)
+                    acc[c] = fma((double)a[u], (double)o[c], acc[c]);
+            }
+        }
+    }
+}
+
+template <int K, typename VM, class Op>
+__global__ void __launch_bounds__(GroupCfg<K>::T, GroupCfg<K>::MINB)
+k_rowgroup(const MatView<VM> m, const GroupView g, const Op op, double *partials, PcgState *st)
+{
+    constexpr int T = GroupCfg<K>::T;
     constexpr int NW = T / 32;
-    constexpr int D = WTileCfg<K>::D;
-    constexpr int EPL = D / 32;                          // entries per lane
     constexpr int NPK = Op::NP * K;
     constexpr int NR = NPK > K ? NPK : K;
-    using VV = typename Op::VV;
 
-    __shared__ double s_prod[NW][D * K];
-    __shared__ int16_t s_rp[NW][D + 1];        // row ends relative to the tile's first entry
-    __shared__ int32_t s_crow[NW][32];
-    __shared__ double s_cval[NW][32 * K];
     __shared__ double s_red[NW * NR];
     __shared__ double s_scal[Op::NS > 0 ? Op::NS : 1];
     __shared__ double s_sum[NR];
@@ -461,7 +491,7 @@ k_wtile(const MatView<VM> m, const Op op, double *partials, PcgState *st)
 
     if (op.skip())
         return;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
     if (tid == 0)
         op.stage(s_scal);
     __syncthreads();
@@ -470,119 +500,55 @@ k_wtile(const MatView<VM> m, const Op op, double *partials, PcgState *st)
 #pragma unroll
     for (int i = 0; i < (NPK > 0 ? NPK : 1); ++i)
         part[i] = 0.0;
-    double *prod = s_prod[wid];
-    int16_t *rpp = s_rp[wid];
 
-    const int gw = blockIdx.x * NW + wid, nw = gridDim.x * NW;
-    for (int t = gw; t < m.n_tiles; t += nw) {
-        const int2 d0 = m.desc[t], d1 = m.desc[t + 1];
-        const int r0 = d0.x, r1 = d1.x;
-        const int64_t k0 = (int64_t)(uint32_t)d0.y, k1 = (int64_t)(uint32_t)d1.y;
-        const int nr = r1 - r0;
-        if ((int64_t)nr + (k1 - k0) > D) {
-            // one long row: lane-strided partial sums, all of a step's loads in flight
-            double lacc[K];
+    // this lane's row position in task t (-1: none) and the task's bin
+    // (static indices only: the bin table stays in the parameter bank)
+    auto locate = [&](int t, int &bin) {
+        int b = 0, t0 = g.task0[0], p0 = g.pos0[0], p1 = g.pos0[1];
 #pragma unroll
-            for (int c = 0; c < K; ++c)
-                lacc[c] = 0.0;
-            for (int64_t kb = k0; kb < k1; kb += 32 * EPL) {
-#pragma unroll
-                for (int u = 0; u < EPL; ++u) {
-                    const int64_t e = kb + lane + 32 * u;
-                    if (e < k1) {
-                        const double a = (double)m.val[e];
-                        VV o[K];
-                        op.operand_row(m.ci[e], o, s_scal);
-#pragma unroll
-                        for (int c = 0; c < K; ++c)
-                            lacc[c] = fma(a, (double)o[c], lacc[c]);
-                    }
-                }
+        for (int i = 1; i < GBINS; ++i)
+            if (t >= g.task0[i]) {
+                b = i;
+                t0 = g.task0[i];
+                p0 = g.pos0[i];
+                p1 = g.pos0[i + 1];
             }
-#pragma unroll
-            for (int c = 0; c < K; ++c)
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    lacc[c] += __shfl_down_sync(0xffffffffu, lacc[c], off);
-            if (lane == 0)
-                op.emit(r0, lacc, part, s_scal, rv);
-            continue;
-        }
-        const int nk = (int)(k1 - k0);
-        // 1. products (matrix loads, then gathers, all in flight) and row ends
-#pragma unroll
-        for (int u = 0; u < EPL; ++u) {
-            const int e = lane + 32 * u;
-            if (e < nk) {
-                const double a = (double)m.val[k0 + e];
-                VV o[K];
-                op.operand_row(m.ci[k0 + e], o, s_scal);
-#pragma unroll
-                for (int c = 0; c < K; ++c)
-                    prod[e * K + c] = a * (double)o[c];
-            }
-        }
-        for (int x = lane; x <= nr; x += 32)
-            rpp[x] = (int16_t)((int64_t)m.rp[r0 + x] - k0);
-        __syncwarp();
-        // 2. merge-path split of the tile's items over the lanes
-        const int items = nr + nk;
-        const int ipt = (items + 31) / 32;
-        const int d0i = min(lane * ipt, items);
-        const int d1i = min(d0i + ipt, items);
-        int lo = max(0, d0i - nk), hi = min(d0i, nr);
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (rpp[mid] <= d0i - mid)
-                lo = mid;
-            else
-                hi = mid - 1;
-        }
-        int r = lo, k = d0i - lo;
-        double acc[K], facc[K];
-#pragma unroll
-        for (int c = 0; c < K; ++c) {
-            acc[c] = 0.0;
-            facc[c] = 0.0;
-        }
-        int frow = -1;
-        for (int d = d0i; d < d1i; ++d) {
-            if (k < rpp[r + 1]) {
-#pragma unroll
-                for (int c = 0; c < K; ++c)
-                    acc[c] += prod[k * K + c];
-                ++k;
-            } else {
-                if (frow < 0) {
-                    frow = r;
-#pragma unroll
-                    for (int c = 0; c < K; ++c)
-                        facc[c] = acc[c];
-                } else {
-                    op.emit(r0 + r, acc, part, s_scal, rv);
-                }
-#pragma unroll
-                for (int c = 0; c < K; ++c)
-                    acc[c] = 0.0;
-                ++r;
-            }
-        }
-        // 3. rows spanning lanes: the lane holding a row's end adds the partial sums the
-        //    earlier lanes left, in a fixed order
-        s_crow[wid][lane] = (r < nr) ? r : -1;
+        bin = b;
+        const int pos = p0 + ((t - t0) << b) + (lane >> (GBINS - 1 - b));
+        return pos < p1 ? pos : -1;
+    };
+    const int nw = gridDim.x * NW;
+    int t = blockIdx.x * NW + (tid >> 5);
+    int bin = 0, pos = t < g.n_tasks ? locate(t, bin) : -1;
+    int4 cur = pos >= 0 ? __ldg(&g.rows[pos]) : make_int4(0, 0, 0, 0);
+    for (; t < g.n_tasks; t += nw) {
+        const int G = 32 >> bin;
+        const bool live = pos >= 0;
+        const int4 row = cur;
+        // the next task's entries, in flight during this one
+        const int tn = t + nw;
+        int bin_n = 0, pos_n = tn < g.n_tasks ? locate(tn, bin_n) : -1;
+        cur = pos_n >= 0 ? __ldg(&g.rows[pos_n]) : make_int4(0, 0, 0, 0);
+
+        double acc[K];
 #pragma unroll
         for (int c = 0; c < K; ++c)
-            s_cval[wid][lane * K + c] = acc[c];
-        __syncwarp();
-        if (frow >= 0) {
-            for (int u = lane - 1; u >= 0 && s_crow[wid][u] == frow; --u) {
-#pragma unroll
-                for (int c = 0; c < K; ++c)
-                    facc[c] += s_cval[wid][u * K + c];
-            }
-            op.emit(r0 + frow, facc, part, s_scal, rv);
+            acc[c] = 0.0;
+        const int gl = lane & (G - 1);
+        if (live) {
+            if (G == 32)
+                group_row_sum<8, K>(m, op, row.y + gl, row.z, G, s_scal, acc);
+            else
+                group_row_sum<4, K>(m, op, row.y + gl, row.z, G, s_scal, acc);
         }
-        __syncwarp();
+        for (int off = G >> 1; off > 0; off >>= 1)
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+                acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], off);
+        if (live && gl == 0)
+            op.emit(row.x, acc, part, s_scal, rv);
+        bin = bin_n;
+        pos = pos_n;
     }
 
     if constexpr (NPK > 0) {
