@@ -379,9 +379,9 @@ struct TileLaunch {
             }
             gv.n_tasks = gp->n_tasks;
             SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_rowgroup<K, VM, Op>,
-                                                                       GroupCfg<K>::T, 0));
+                                                                       GroupCfg<K, Op>::T, 0));
             per_sm = std::max(per_sm, 1);
-            const int per_block = GroupCfg<K>::T / 32;
+            const int per_block = GroupCfg<K, Op>::T / 32;
             grid = std::max(1, std::min((gp->n_tasks + per_block - 1) / per_block, per_sm * A->num_sms));
             maxl = -1;
             return SLA_SUCCESS;
@@ -412,7 +412,7 @@ struct TileLaunch {
         case 16: k_rows_tma<K, VM, 16, Op><<<grid, RTHREADS, RSMEM, s>>>(m, w, op, part, st, err); break;
         case -1:
             if constexpr (LANE_GROUPS)
-                k_rowgroup<K, VM, Op><<<grid, GroupCfg<K>::T, 0, s>>>(m, gv, op, part, st);
+                k_rowgroup<K, VM, Op><<<grid, GroupCfg<K, Op>::T, 0, s>>>(m, gv, op, part, st);
             break;
         default:
             if constexpr (!LANE_GROUPS)

@@ -188,6 +188,7 @@ template <typename V, int K>
 struct OpSpmv {
     using VV = V;
     static constexpr int NP = 0, NS = 0, NV = 0;
+    static constexpr bool ANY_LD = true;
     static constexpr int NG = 1;
     const V *x;
     V *y;

@@ -27,6 +27,8 @@
 //   spends a merge-path split and a carry walk on it.
 #pragma once
 
+#include <type_traits>
+
 #include "sla_internal.cuh"
 
 namespace sla {
@@ -431,10 +433,10 @@ k_tile2(const MatView<VM> m, const Op op, double *partials, PcgState *st)
 
 // ------------------------------------------------------------------ lane-group kernel
 // Rows grouped by length (GroupPart): a group of G lanes owns a row, each lane takes the
-// row's entries G apart (up to 4 per pass for G < 32, 8 per pass for whole-warp rows; all
-// of a pass's loads in flight) and the group sums its lanes with a fixed xor-shuffle tree.
-// A warp takes one task (32 / G rows of one bin) at a time, the tasks round-robin over the
-// grid's warps; the next task's row list entries are loaded while the current one runs.
+// row's entries G apart (4 per pass, all of a pass's loads in flight) and the group sums
+// its lanes with a fixed xor-shuffle tree.  A warp takes one task (32 / G rows of one bin)
+// at a time, the tasks round-robin over the grid's warps; the next task's row list entries
+// are loaded while the current one runs.
 struct GroupView {
     const int4 *rows;
     int task0[GBINS + 1];
@@ -442,10 +444,18 @@ struct GroupView {
     int n_tasks;
 };
 
-template <int K>
+// Ops that read caller vectors with a runtime leading dimension (the standalone SpMV) mark
+// themselves ANY_LD: their 64-bit operand addressing needs more registers.
+template <class Op, class = void>
+struct any_ld : std::false_type {};
+template <class Op>
+struct any_ld<Op, std::void_t<decltype(Op::ANY_LD)>> : std::bool_constant<Op::ANY_LD> {};
+
+template <int K, class Op>
 struct GroupCfg {
     static constexpr int T = 256;
-    static constexpr int MINB = K == 1 ? 6 : K == 2 ? 5 : 4;
+    static constexpr int U = 4;                          // entries per lane per pass
+    static constexpr int MINB = K == 1 ? (any_ld<Op>::value ? 6 : 8) : K == 2 ? 5 : 4;
 };
 
 template <int U, int K, typename VM, class Op>
@@ -476,10 +486,10 @@ __device__ __forceinline__ void group_row_sum(const MatView<VM> &m, const Op &op
 }
 
 template <int K, typename VM, class Op>
-__global__ void __launch_bounds__(GroupCfg<K>::T, GroupCfg<K>::MINB)
+__global__ void __launch_bounds__(GroupCfg<K, Op>::T, GroupCfg<K, Op>::MINB)
 k_rowgroup(const MatView<VM> m, const GroupView g, const Op op, double *partials, PcgState *st)
 {
-    constexpr int T = GroupCfg<K>::T;
+    constexpr int T = GroupCfg<K, Op>::T;
     constexpr int NW = T / 32;
     constexpr int NPK = Op::NP * K;
     constexpr int NR = NPK > K ? NPK : K;
@@ -535,12 +545,8 @@ k_rowgroup(const MatView<VM> m, const GroupView g, const Op op, double *partials
         for (int c = 0; c < K; ++c)
             acc[c] = 0.0;
         const int gl = lane & (G - 1);
-        if (live) {
-            if (G == 32)
-                group_row_sum<8, K>(m, op, row.y + gl, row.z, G, s_scal, acc);
-            else
-                group_row_sum<4, K>(m, op, row.y + gl, row.z, G, s_scal, acc);
-        }
+        if (live)
+            group_row_sum<GroupCfg<K, Op>::U, K>(m, op, row.y + gl, row.z, G, s_scal, acc);
         for (int off = G >> 1; off > 0; off >>= 1)
 #pragma unroll
             for (int c = 0; c < K; ++c)
