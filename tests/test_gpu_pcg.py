@@ -258,3 +258,60 @@ def test_handle_destruction_any_order(order):
         assert info.status == 0
         Gd.close()
         Ad.close()
+
+
+def _mixed_length_spd(n=6000, hubs=150, seed=11):
+    """fp32 SPD matrix whose row lengths fill every lane-group length bin: ordinary rows link
+    to 0-40 others, mostly hub rows (1 to ~45 entries per row); the hub rows collect a few
+    hundred entries each."""
+    rng = np.random.default_rng(seed)
+    deg = rng.choice([0, 1, 2, 3, 6, 12, 25, 40], size=n, p=[.2, .2, .15, .15, .1, .1, .06, .04])
+    lo, hi = [], []
+    for i in range(hubs, n):
+        d = int(deg[i])
+        if d == 0:
+            continue
+        js = np.where(rng.random(d) < 0.8, rng.integers(0, hubs, d), rng.integers(0, n, d))
+        js = js[js != i]
+        lo.append(np.minimum(js, i))
+        hi.append(np.maximum(js, i))
+    lo = np.concatenate(lo).astype(np.int64)
+    hi = np.concatenate(hi).astype(np.int64)
+    key = np.unique(lo * n + hi)
+    return W._assemble_symmetric(key // n, key % n, n, seed, 0.1, np.float32)
+
+
+@pytest.mark.parametrize("nrhs", [1, 2, 3, 4, 8])
+def test_mixed_row_lengths_multi_rhs(ora, nrhs):
+    """The long-row engines (lane groups up to 4 right-hand sides, row tiles above) on a
+    SPAI-preconditioned matrix whose rows fill every length bin, from 1 entry to hundreds:
+    lockstep iterates, then converged solve and adjoint against the oracle."""
+    import differentiable_sparse_linear_b200 as sla
+    A = _mixed_length_spd()
+    lens = np.diff(A.row_ptr)
+    assert lens.min() == 1 and lens.max() > 128
+    G = W.spai_factor_G(A, seed=12)
+    eps = 3e-3
+    kw = dict(precond="spai", G=G, eps=eps)
+    Ad, Gd = matrix(A), matrix(G)
+    M = sla.sla_precond_spai(Ad, Gd, eps)
+    B = np.random.default_rng(13).standard_normal((A.n_rows, nrhs)).astype(np.float32)
+    k = 7
+    X, infos = sla.sla_pcg_solve_batched(Ad, M, dev(B), rtol=1e-300, maxit=k)
+    assert all(i.engine == "graph" and i.iters == k for i in infos)
+    Xo, _ = ora.pcg_multi(A, B, fixed_iters=k, **kw)
+    assert rel(host(X), Xo) <= 1e-5
+    # converged, fp64 vectors: the iteration counts match the oracle's
+    X, infos = sla.sla_pcg_solve_batched(Ad, M, dev(B, np.float64), rtol=1e-6, vector_f64=True)
+    Xo, outs = ora.pcg_multi(A, B, tol=1e-6, **kw)
+    for c in range(nrhs):
+        assert infos[c].status == 0
+        assert iters_close(infos[c].iters, outs[c].iters), (c, infos[c].iters, outs[c].iters)
+    assert rel(host(X), Xo) <= 1e-5
+    Wt = np.random.default_rng(14).uniform(-1, 1, size=(A.n_rows, nrhs))
+    Lam, g, ainf = sla.sla_pcg_adjoint_batched(Ad, M, X, dev(Wt), rtol=1e-6, vector_f64=True)
+    Lo, go, aouts = ora.adjoint_multi(A, Xo, Wt, tol=1e-6, **kw)
+    for c in range(nrhs):
+        assert iters_close(ainf[c].iters, aouts[c].iters)
+    assert rel(host(Lam), Lo) <= SOL_TOL[np.float32]
+    assert rel(host(g), go) <= SOL_TOL[np.float32]
