@@ -87,6 +87,11 @@ class Oracle:
         lib.ora_pcg.restype = C.c_int
         lib.ora_pattern_grad.argtypes = [C.c_int64, _i32p, _i32p, _f64p, _f64p, _f64p]
         lib.ora_pattern_grad.restype = None
+        lib.ora_bsr_spmv.argtypes = [C.c_int64, C.c_int32, _i32p, _i32p, _f64p, _f64p, _f64p]
+        lib.ora_bsr_spmv.restype = None
+        lib.ora_bsr_to_csr.argtypes = [C.c_int64, C.c_int32, _i32p, _i32p, _f64p, _i32p, _i32p, _f64p,
+                                       np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")]
+        lib.ora_bsr_to_csr.restype = None
         self.lib = lib
 
     # ---------------------------------------------------------------- basic operations
@@ -216,6 +221,39 @@ class Oracle:
             g = g + r.grad
             out.append(r)
         return Lam, g, out
+
+    # ---------------------------------------------------------------- block sparse rows
+    def bsr_spmv(self, A, x) -> np.ndarray:
+        """y = A x for a BSR matrix (``A.val`` is [nnzb, b, b]) in fp64."""
+        x = _f64(x)
+        y = np.empty(A.n_rows, dtype=np.float64)
+        self.lib.ora_bsr_spmv(A.n_brows, A.b, _i32(A.row_ptr), _i32(A.col), _f64(A.val).reshape(-1), x, y)
+        return y
+
+    def bsr_to_csr(self, A):
+        """(scalar CSR of the BSR matrix A with fp64 values, BSR value position of each entry)."""
+        from sla_workloads import CSR
+        nnz = A.nnzb * A.b * A.b
+        rp = np.empty(A.n_rows + 1, dtype=np.int32)
+        ci = np.empty(nnz, dtype=np.int32)
+        v = np.empty(nnz, dtype=np.float64)
+        pos = np.empty(nnz, dtype=np.int64)
+        self.lib.ora_bsr_to_csr(A.n_brows, A.b, _i32(A.row_ptr), _i32(A.col), _f64(A.val).reshape(-1),
+                                rp, ci, v, pos)
+        return CSR(A.n_rows, A.n_rows, rp, ci, v), pos
+
+    def pcg_bsr(self, A, b, **kw) -> SolveResult:
+        """PCG on a BSR matrix: the same iteration on its scalar CSR form."""
+        return self.pcg(self.bsr_to_csr(A)[0], b, **kw)
+
+    def adjoint_bsr(self, A, x, w, **kw) -> AdjointResult:
+        """Adjoint on a BSR matrix; the gradient comes back in BSR value order ([nnzb, b, b])."""
+        Ac, pos = self.bsr_to_csr(A)
+        r = self.adjoint(Ac, x, w, **kw)
+        g = np.empty(pos.size, dtype=np.float64)
+        g[pos] = r.grad
+        r.grad = g.reshape(A.nnzb, A.b, A.b)
+        return r
 
     @staticmethod
     def system(A, s: int):

@@ -233,3 +233,48 @@ void ora_pattern_grad(int64_t n_rows, const int32_t *rp, const int32_t *ci, cons
         for (int64_t k = rp[i]; k < rp[i + 1]; ++k)
             g[k] = -lam[i] * x[ci[k]];
 }
+
+/* Block sparse row (BSR) storage -- [SM] "Efficient Sparse Matrix Algebra in Python for
+ * Mathematics", "Key sparse formats and memory tradeoffs" (block sparse layouts store
+ * dense blocks) and "Block sparse patterns and sharding strategies" (one index per block).
+ * The matrix is a CSR pattern of b x b dense blocks: block row I holds blocks
+ * k = rp[I] .. rp[I+1]-1 in block columns ci[k], and block k keeps its b*b values row-major
+ * at val[k*b*b].  Scalar entry (I*b + r, ci[k]*b + c) is val[k*b*b + r*b + c].
+ *
+ * y = A x: scalar row I*b + r is the sum, over the blocks of block row I in storage order
+ * and over c = 0 .. b-1, of val[k*b*b + r*b + c] * x[ci[k]*b + c]. */
+void ora_bsr_spmv(int64_t n_brows, int32_t b, const int32_t *rp, const int32_t *ci, const double *val,
+                  const double *x, double *y)
+{
+    for (int64_t I = 0; I < n_brows; ++I)
+        for (int32_t r = 0; r < b; ++r) {
+            double s = 0.0;
+            for (int64_t k = rp[I]; k < rp[I + 1]; ++k)
+                for (int32_t c = 0; c < b; ++c)
+                    s += val[k * b * b + (int64_t)r * b + c] * x[(int64_t)ci[k] * b + c];
+            y[I * b + r] = s;
+        }
+}
+
+/* The same matrix as scalar CSR: scalar row I*b + r lists, for each block k of block row I
+ * in storage order, the b entries (r, c) -- ascending columns when the block columns are
+ * ascending.  pos[e] is the BSR value position of CSR entry e, so a result on the CSR
+ * pattern maps back to BSR order by g_bsr[pos[e]] = g_csr[e]. */
+void ora_bsr_to_csr(int64_t n_brows, int32_t b, const int32_t *rp, const int32_t *ci, const double *val,
+                    int32_t *out_rp, int32_t *out_ci, double *out_val, int64_t *pos)
+{
+    int64_t e = 0;
+    out_rp[0] = 0;
+    for (int64_t I = 0; I < n_brows; ++I)
+        for (int32_t r = 0; r < b; ++r) {
+            for (int64_t k = rp[I]; k < rp[I + 1]; ++k)
+                for (int32_t c = 0; c < b; ++c) {
+                    const int64_t p = k * b * b + (int64_t)r * b + c;
+                    out_ci[e] = (int32_t)((int64_t)ci[k] * b + c);
+                    out_val[e] = val[p];
+                    pos[e] = p;
+                    ++e;
+                }
+            out_rp[I * b + r + 1] = (int32_t)e;
+        }
+}

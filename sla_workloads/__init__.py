@@ -19,6 +19,9 @@ stand in for the pages' benchmarks:
   Inverse Preconditioners for Conjugate Gradient Solvers on GPUs", Key results).
 * The SPAI factor G with A's lower-triangular pattern (same page, Approach:
   M^-1 = G G^T + eps I, G sharing A's sparsity), here synthetic rather than learned.
+* A vector-valued 3D problem stored in 3 x 3 blocks (BSR), standing in for the same page's
+  hyperelasticity benchmark; block sparse storage as "Efficient Sparse Matrix Algebra in
+  Python for Mathematics" describes it (Key sparse formats and memory tradeoffs).
 
 Random draws use numpy's PCG64 ``default_rng``.  Off-diagonal values of the random SPD
 matrices come from the SplitMix64 mixing function (Steele, Lea and Flood, "Fast
@@ -33,7 +36,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = [
-    "CSR", "Workload", "splitmix64", "hash_uniform01", "sorted_unique",
+    "CSR", "BSR", "Workload", "coupling_block", "elastic3d_bsr", "random_bsr", "splitmix64", "hash_uniform01", "sorted_unique",
     "poisson2d", "heat3d", "random_spd_list", "powerlaw_spd", "spai_factor_G",
     "rhs_uniform", "rhs_normal", "workload", "CONFIG_NAMES",
 ]
@@ -61,6 +64,38 @@ class CSR:
 
     def rows_of_entries(self) -> np.ndarray:
         return np.repeat(np.arange(self.n_rows, dtype=np.int64), np.diff(self.row_ptr))
+
+
+@dataclass
+class BSR:
+    """Block sparse row matrix: a CSR pattern of b x b dense blocks.
+
+    int32 row_ptr (n_brows+1) and col (nnzb) index blocks; val is [nnzb, b, b], each block
+    row-major, so scalar entry (I*b + r, col[k]*b + c) is val[k, r, c].
+    """
+    n_brows: int
+    b: int
+    row_ptr: np.ndarray
+    col: np.ndarray
+    val: np.ndarray
+
+    @property
+    def n_rows(self) -> int:
+        return self.n_brows * self.b
+
+    @property
+    def n_cols(self) -> int:
+        return self.n_rows
+
+    @property
+    def nnzb(self) -> int:
+        return int(self.row_ptr[-1])
+
+    @property
+    def nnz(self) -> int:
+        return self.nnzb * self.b * self.b
+
+    sys_row_off = None
 
 
 @dataclass
@@ -186,6 +221,44 @@ def poisson1d(N: int, dtype=np.float64) -> CSR:
 def heat3d(N: int, dt: float = 0.1, dtype=np.float32) -> CSR:
     """Implicit heat step A = I + dt*L, L the unscaled 7-point Laplacian (diag 6, off -1)."""
     return _stencil_csr((N, N, N), 1.0 + 6.0 * dt, -dt, dtype)
+
+
+def coupling_block(b: int) -> np.ndarray:
+    """The b x b SPD coupling S = tridiag(1/2, 1, 1/2), eigenvalues 1 + cos(m pi / (b+1))."""
+    S = np.eye(b)
+    for r in range(b - 1):
+        S[r, r + 1] = S[r + 1, r] = 0.5
+    return S
+
+
+def elastic3d_bsr(N: int, b: int = 3, shift: float = 0.1, dtype=np.float32) -> BSR:
+    """Vector-valued 3D model problem in b x b blocks: A = L (x) S + shift*I on an N^3 grid.
+
+    L is the unscaled 7-point Dirichlet Laplacian (diagonal 6, neighbours -1), S the SPD
+    coupling above, so a node couples its b unknowns to each neighbour's through -S and
+    its own through 6 S + shift I -- the block structure of a vector PDE (the pages'
+    hyperelasticity benchmark has 3 unknowns per node).  A is SPD: its eigenvalues are
+    lambda_L * mu_S + shift.
+    """
+    P = _stencil_csr((N, N, N), 6.0, -1.0, np.float64)
+    S = coupling_block(b)
+    rows = P.rows_of_entries()
+    val = P.val[:, None, None] * S[None, :, :]
+    diag = rows == P.col.astype(np.int64)
+    val[diag] += shift * np.eye(b)[None, :, :]
+    return BSR(P.n_rows, b, P.row_ptr, P.col, val.astype(dtype))
+
+
+def random_bsr(n_brows: int, b: int, lens: np.ndarray, seed: int, dtype=np.float32) -> BSR:
+    """Unstructured BSR pattern (block row I holds lens[I] distinct block columns, ascending)
+    with values U[-1, 1]: SpMV and layout tests, not a solvable system."""
+    rng = np.random.default_rng(seed)
+    rp = np.zeros(n_brows + 1, dtype=np.int64)
+    np.cumsum(lens, out=rp[1:])
+    col = np.concatenate([np.sort(rng.choice(n_brows, size=int(l), replace=False)) if l else
+                          np.zeros(0, np.int64) for l in lens]).astype(np.int32)
+    val = rng.uniform(-1, 1, size=(col.size, b, b)).astype(dtype)
+    return BSR(n_brows, b, rp.astype(np.int32), col, val)
 
 
 # ----------------------------------------------------------------------------------------
@@ -358,11 +431,12 @@ CONFIG_NAMES = {
     3: "heat3d_128_f32_jacobi_8rhs",
     4: "spd_list_4096x1024_f64_jacobi",
     5: "powerlaw_4M_f32_spai",
+    6: "elastic3d_128_bsr3_f32_jacobi",
 }
 
 
 def workload(cfg: int, size: str = "full") -> Workload:
-    """Build synthetic workload ``cfg`` (1..5).
+    """Build synthetic workload ``cfg`` (1..6; 6 is the block-sparse (BSR) vector problem).
 
     size="full" gives the stated sizes.  size="small" keeps each recipe (pattern law,
     value law, precision, preconditioner, tolerance, seeds) at a size the fp64 oracle
@@ -412,4 +486,11 @@ def workload(cfg: int, size: str = "full") -> Workload:
         return Workload(CONFIG_NAMES[5] if size == "full" else f"powerlaw_{n}_f32_spai", A,
                         rhs_normal(5001, n, np.float32), rhs_uniform(5002, n, dtype=np.float32),
                         1e-6, "spai", G=G, eps=3e-3, dtype=np.float32, info={"n": n})
+    if cfg == 6:
+        N = 128 if not small else (16 if not tiny else 5)
+        A = elastic3d_bsr(N, 3, 0.1, np.float32)
+        n = A.n_rows
+        return Workload(CONFIG_NAMES[6] if not small else f"elastic3d_{N}_bsr3_f32_jacobi", A,
+                        rhs_normal(6001, n, np.float32), rhs_uniform(6002, n, dtype=np.float32),
+                        1e-6, "jacobi", dtype=np.float32, info={"grid": N, "block": 3})
     raise ValueError(f"unknown workload {cfg}")

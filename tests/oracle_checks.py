@@ -17,6 +17,10 @@ What pins what:
   * SPAI apply -- the dense product (G G^T + eps I) r.
   * adjoint    -- A lam = w; w.x = lam.b; sum A_ij g_ij = -L; central finite differences
                   of L = w.A^-1 b (dense LU) in single stored entries and in b.
+  * BSR        -- a dense matrix assembled block by block (numpy) for the block SpMV and the
+                  scalar CSR expansion; closed-form eigenpairs of L (x) S + shift I (the
+                  block vector problem) for the SpMV and one-step PCG; central finite
+                  differences of L in single block entries for the gradient in block order.
 """
 from __future__ import annotations
 
@@ -312,9 +316,80 @@ def check_list_blocks(ora):
     assert rel(x, np.linalg.solve(Ad, b)) < 1e-10, "block-diagonal list vs dense solve"
 
 
+# ------------------------------------------------------------------------------ BSR
+def dense_bsr(A) -> np.ndarray:
+    """Dense matrix of a BSR matrix, placed block by block."""
+    b = A.b
+    D = np.zeros((A.n_rows, A.n_rows), dtype=np.float64)
+    for I in range(A.n_brows):
+        for k in range(int(A.row_ptr[I]), int(A.row_ptr[I + 1])):
+            J = int(A.col[k])
+            D[I * b:(I + 1) * b, J * b:(J + 1) * b] = A.val[k].astype(np.float64)
+    return D
+
+
+def check_bsr_spmv_dense(ora):
+    for b, seed in ((1, 41), (2, 42), (3, 43), (4, 44)):
+        lens = np.random.default_rng(seed).integers(0, 5, size=37)
+        lens[[3, 20]] = [0, 30]
+        A = W.random_bsr(37, b, lens, seed, np.float64)
+        D = dense_bsr(A)
+        x = np.random.default_rng(seed + 100).uniform(-1, 1, A.n_rows)
+        assert rel(ora.bsr_spmv(A, x), D @ x) < TOL_TIGHT, f"BSR SpMV, b = {b}"
+        Ac, pos = ora.bsr_to_csr(A)
+        assert np.array_equal(dense(Ac), D), f"BSR -> CSR expansion, b = {b}"
+        assert np.array_equal(np.sort(pos), np.arange(A.nnz)), "BSR positions are a permutation"
+        assert np.array_equal(Ac.val, A.val.reshape(-1)[pos].astype(np.float64)), "BSR positions"
+
+
+def _elastic_eigvec(N, b, jkl, m):
+    """Eigenvector v_jkl (x) s_m of L (x) S on the N^3 grid, and its eigenvalue factors."""
+    ax = np.arange(1, N + 1)
+    v = np.einsum("i,j,k->ijk", *[np.sin(j * np.pi * ax / (N + 1)) for j in jkl]).reshape(-1)
+    lam = sum(2.0 - 2.0 * np.cos(j * np.pi / (N + 1)) for j in jkl)
+    s = np.sin(m * np.pi * np.arange(1, b + 1) / (b + 1))
+    mu = 1.0 + np.cos(m * np.pi / (b + 1))
+    return np.kron(v, s), lam, mu
+
+
+def check_bsr_closed_form(ora):
+    for b in (2, 3):
+        N, shift = 4, 0.1
+        A = W.elastic3d_bsr(N, b, shift, np.float64)
+        for jkl, m in (((1, 1, 1), 1), ((2, 3, 1), b), ((4, 2, 3), 2)):
+            u, lam, mu = _elastic_eigvec(N, b, jkl, m)
+            ev = lam * mu + shift
+            assert rel(ora.bsr_spmv(A, u), ev * u) < TOL_TIGHT, f"BSR eigenpair b={b} {jkl} {m}"
+            # constant diagonal (6 + shift): Jacobi is a multiple of I, CG stops in one step
+            r = ora.pcg_bsr(A, u, precond="jacobi", tol=1e-12)
+            assert r.status == 0 and r.iters == 1, f"one-step PCG on a BSR eigenvector ({r.iters})"
+            assert rel(r.x, u / ev) < 1e-12
+
+
+def check_bsr_grad_fd(ora):
+    A = W.elastic3d_bsr(2, 2, 0.3, np.float64)
+    D = dense_bsr(A)
+    rng = np.random.default_rng(45)
+    bvec = rng.uniform(-1, 1, A.n_rows)
+    w = rng.uniform(-1, 1, A.n_rows)
+    x = np.linalg.solve(D, bvec)
+    adj = ora.adjoint_bsr(A, x, w, precond="jacobi", tol=1e-14)
+    assert adj.grad.shape == A.val.shape
+    for k, r, c in ((0, 0, 1), (3, 1, 0), (int(A.nnzb) - 1, 1, 1)):
+        I = int(np.searchsorted(A.row_ptr, k, side="right")) - 1
+        i, j = I * A.b + r, int(A.col[k]) * A.b + c
+        h = 1e-6 * max(1.0, abs(D[i, j]))
+        Dp, Dm = D.copy(), D.copy()
+        Dp[i, j] += h
+        Dm[i, j] -= h
+        fd = (w @ np.linalg.solve(Dp, bvec) - w @ np.linalg.solve(Dm, bvec)) / (2 * h)
+        assert abs(adj.grad[k, r, c] - fd) <= 1e-7 * max(1.0, abs(fd)), f"BSR dL/dA block {k} ({r},{c})"
+
+
 ALL_CHECKS = [
     check_spmv_closed_form, check_spmv_dense, check_transpose, check_spai_apply,
     check_pcg_krylov_optimal, check_pcg_eigvec_one_step, check_pcg_m_distinct,
     check_pcg_dense_solve, check_pcg_scaling, check_pcg_status, check_adjoint_identities,
     check_grad_fd, check_grad_fd_symmetric, check_list_blocks,
+    check_bsr_spmv_dense, check_bsr_closed_form, check_bsr_grad_fd,
 ]

@@ -33,6 +33,14 @@ MUTANTS = {
     "absolute_stop_test": ("*relres = rnorm / bnorm;", "*relres = rnorm;"),
     "grad_sign": ("g[k] = -lam[i] * x[ci[k]];", "g[k] = lam[i] * x[ci[k]];"),
     "grad_transposed": ("g[k] = -lam[i] * x[ci[k]];", "g[k] = -lam[ci[k]] * x[i];"),
+    "bsr_block_transposed": ("s += val[k * b * b + (int64_t)r * b + c] * x[(int64_t)ci[k] * b + c];",
+                             "s += val[k * b * b + (int64_t)c * b + r] * x[(int64_t)ci[k] * b + c];"),
+    "bsr_operand_row": ("s += val[k * b * b + (int64_t)r * b + c] * x[(int64_t)ci[k] * b + c];",
+                        "s += val[k * b * b + (int64_t)r * b + c] * x[(int64_t)ci[k] * b + r];"),
+    "bsr_expansion_position": ("const int64_t p = k * b * b + (int64_t)r * b + c;",
+                               "const int64_t p = k * b * b + (int64_t)c * b + r;"),
+    "bsr_expansion_column": ("out_ci[e] = (int32_t)((int64_t)ci[k] * b + c);",
+                             "out_ci[e] = (int32_t)((int64_t)ci[k] + c);"),
 }
 
 
