@@ -7,7 +7,7 @@ Poisson problem (1024 x 1024 grid, fp32 values and vectors, fp64 reductions,
 M^-1 = G G^T + 3e-3 I, tolerance 1e-6).  value = PCG iterations (forward + adjoint) per
 second over all ranks.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..5]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..6]
 
 Multi-GPU (torchrun): every rank solves its own replica (the single-system solve does not
 shard here), weak scaling; time is the max over ranks.  --impl reference times the fp64
@@ -30,6 +30,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+
+import sla_workloads as W  # noqa: E402  (seeded inputs; no method arithmetic)
 
 METRIC = "PCG iterations/sec and SpMV HBM GB/s (fraction of ~8 TB/s) at 1 B200"
 UNIT = "iterations/s"
@@ -59,12 +61,25 @@ def matrix_bytes(n, nnz, sv) -> int:
     return nnz * (sv + 4) + (n + 1) * 4
 
 
+def stream_bytes(A, sv) -> int:
+    """Algorithmic bytes to stream matrix A: CSR as above; BSR one column index and b*b
+    values per block plus the block row pointers."""
+    if isinstance(A, W.BSR):
+        return A.nnzb * (A.b * A.b * sv + 4) + (A.n_brows + 1) * 4
+    return matrix_bytes(A.n_rows, A.nnz, sv)
+
+
+def oracle_matrix(ora, A):
+    """The matrix as the oracle takes it: a BSR matrix as its scalar CSR expansion."""
+    return ora.bsr_to_csr(A)[0] if isinstance(A, W.BSR) else A
+
+
 def kernel_bytes(w) -> dict:
     """Algorithmic bytes per launch of each kernel of one PCG iteration (K right-hand sides)."""
     A = w.A
     n, nnz, sv = A.n_rows, A.nnz, vbytes(w.dtype)
     K = w.nrhs
-    out = {"q_spmv": matrix_bytes(n, nnz, sv) + 4 * n * K * sv}   # read z, p_old; write p_new, q
+    out = {"q_spmv": stream_bytes(A, sv) + 4 * n * K * sv}   # read z, p_old; write p_new, q
     if w.precond == "spai":
         ng = w.G.nnz
         out["update_gt_spmv"] = matrix_bytes(n, ng, sv) + 7 * n * K * sv   # r,q gathered; p,x; write r,x,y
@@ -200,6 +215,7 @@ def cpu_baseline(w, budget_s: float = 15.0) -> dict:
     ora = oracle.get()
     B = w.B if w.B.ndim == 1 else w.B[:, 0]
     A = w.A
+    A = oracle_matrix(ora, A)
     if A.sys_row_off is not None:
         A = ora.system(A, 0)
         B = B[: A.n_rows]
@@ -244,6 +260,7 @@ def run_reference(args):
     ora = oracle.get()
     B = w.B if w.B.ndim == 1 else w.B[:, 0]
     A = w.A
+    A = oracle_matrix(ora, A)
     if A.sys_row_off is not None:
         A = ora.system(A, 0)
         B = B[: A.n_rows]
@@ -299,6 +316,8 @@ def run_ours(args):
     is_list = A.sys_row_off is not None
     if is_list:
         Ad = sla.sla_csr_create_list(list(A.sys_row_off), rp, ci, va)
+    elif isinstance(A, W.BSR):
+        Ad = sla.sla_bsr_create(rp, ci, va)
     else:
         Ad = sla.sla_csr_create(rp, ci, va)
     Gd = None
@@ -315,8 +334,14 @@ def run_ours(args):
     setup_s = time.perf_counter() - t_setup
     nrhs = w.nrhs
     multi = is_list or nrhs > 1
-    body_kernels = 6 if w.precond == "spai" else 4       # two iterations per graph loop body
-    prologue = 2 if w.precond == "spai" else 1
+    # graph engine: matrices with rows of more than 16 entries (and BSR matrices) get their
+    # operand vectors formed by an elementwise kernel first (Q: k_ep + SpMV; U_S: k_er + SpMV)
+    spai = w.precond == "spai"
+    form_a = isinstance(A, W.BSR) or (not is_list and int(np.diff(A.row_ptr).max(initial=0)) > 16)
+    form_gt = spai and int(np.bincount(w.G.col, minlength=A.n_rows).max(initial=0)) > 16
+    q_k, us_k = (2 if form_a else 1), (2 if form_gt else 1)
+    body_kernels = 2 * (q_k + us_k + 1) if spai else 2 * (q_k + 1)   # two iterations per loop body
+    prologue = us_k + 1 if spai else 1
     engines_seen = set()
 
     def launches(iters: int, engine: str) -> int:
@@ -542,7 +567,7 @@ def run_ours(args):
             torch.cuda.synchronize()
             if r >= 2:
                 tot += s0.elapsed_time(s1)
-        sb = matrix_bytes(A.n_rows, A.nnz, vbytes(w.dtype)) + 2 * A.n_rows * nrhs * vbytes(w.dtype)
+        sb = stream_bytes(A, vbytes(w.dtype)) + 2 * A.n_rows * nrhs * vbytes(w.dtype)
         sp_ms = tot / reps
         spmv = {"gbs": sb / (sp_ms * 1e6), "frac": sb / (sp_ms * 1e6) / peak, "ms": sp_ms, "bytes": sb,
                 "l2": "flushed before each launch (512 MiB write + 256 MiB read)"}

@@ -25,7 +25,7 @@ from ._lib import (SLA_BREAKDOWN, SLA_ERR_CUDA, SLA_ERR_INVALID_ARG, SLA_ERR_INV
 
 __all__ = [
     "SlaError", "Matrix", "Preconditioner", "PcgInfo", "lib",
-    "sla_version", "sla_csr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
+    "sla_version", "sla_csr_create", "sla_bsr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
     "sla_pcg_solve_batched_noalloc",
@@ -120,12 +120,13 @@ class Matrix:
     The tensors are borrowed by the library; this object keeps them alive.
     """
 
-    def __init__(self, handle: int, row_ptr, col, val, sys_row_off=None):
+    def __init__(self, handle: int, row_ptr, col, val, sys_row_off=None, block: int = 1):
         self._h = C.c_void_p(handle)
         self.row_ptr, self.col, self.val = row_ptr, col, val
         self.sys_row_off = sys_row_off
-        self.n = row_ptr.numel() - 1
-        self.nnz = col.numel()
+        self.block = block                       # BSR block size (1: CSR)
+        self.n = (row_ptr.numel() - 1) * block   # scalar rows
+        self.nnz = col.numel() * block * block   # stored scalar values
         self.dtype = val.dtype
         self.batch = 1 if sys_row_off is None else len(sys_row_off) - 1
 
@@ -197,6 +198,25 @@ def sla_csr_create(row_ptr: torch.Tensor, col: torch.Tensor, val: torch.Tensor, 
     _check(lib().sla_csr_create(C.byref(h), n, n, col.numel(), _ptr(row_ptr), _ptr(col), _ptr(val),
                                 _dtype_code(val.dtype), flags, _stream(stream)), "sla_csr_create")
     return Matrix(h.value, row_ptr, col, val)
+
+
+def sla_bsr_create(row_ptr: torch.Tensor, col: torch.Tensor, val: torch.Tensor, *,
+                   validate: bool = True, spd: bool = True, stream=None) -> Matrix:
+    """sla_bsr_create: one square block sparse row matrix; val is [nnzb, b, b] (row-major
+    blocks), row_ptr / col index the blocks.  Gradients on its pattern come back flat,
+    aligned with val's elements."""
+    if row_ptr.dtype != torch.int32 or col.dtype != torch.int32:
+        raise ValueError("row_ptr and col must be int32")
+    if val.dim() != 3 or val.shape[1] != val.shape[2] or val.shape[0] != col.numel():
+        raise ValueError("val must be [nnzb, b, b]")
+    if not val.is_contiguous():
+        raise ValueError("val must be contiguous")
+    b = int(val.shape[1])
+    h = C.c_void_p()
+    flags = (SLA_VALIDATE if validate else 0) | (SLA_SPD if spd else 0)
+    _check(lib().sla_bsr_create(C.byref(h), row_ptr.numel() - 1, b, col.numel(), _ptr(row_ptr), _ptr(col),
+                                _ptr(val), _dtype_code(val.dtype), flags, _stream(stream)), "sla_bsr_create")
+    return Matrix(h.value, row_ptr, col, val, block=b)
 
 
 def sla_csr_create_list(sys_row_off: Sequence[int], row_ptr: torch.Tensor, col: torch.Tensor,

@@ -47,6 +47,8 @@ SIGNATURES = {
                              C.c_int, C.c_uint32, _vp]),
     "sla_csr_create_list": (_st, [C.POINTER(_vp), C.c_int32, C.POINTER(C.c_int64), C.c_int64, _vp,
                                   _vp, _vp, C.c_int, C.c_uint32, _vp]),
+    "sla_bsr_create": (_st, [C.POINTER(_vp), C.c_int64, C.c_int32, C.c_int64, _vp, _vp, _vp,
+                             C.c_int, C.c_uint32, _vp]),
     "sla_csr_destroy": (_st, [_vp]),
     "sla_csr_shape": (_st, [_vp, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int32)]),
     "sla_spmv": (_st, [_vp, _vp, _vp, _vp]),

@@ -172,10 +172,12 @@ sla_status ensure_groups(sla_csr *A, cudaStream_t s, const GroupPart **out)
         return SLA_SUCCESS;
     }
     std::vector<int32_t> bin_rows[GBINS];
-    for (int64_t r = 0; r < A->n; ++r) {
+    const int64_t per_lane = A->bdim > 1 ? 2 : 4;   // items a lane takes per pass
+    const int64_t nrows = pattern_rows(A);
+    for (int64_t r = 0; r < nrows; ++r) {
         const int64_t len = (int64_t)A->h_rp[(size_t)r + 1] - A->h_rp[(size_t)r];
         int b = GBINS - 1;                  // G = 1
-        while (b > 0 && 4 * (int64_t(1) << (GBINS - 1 - b)) < len)
+        while (b > 0 && per_lane * (int64_t(1) << (GBINS - 1 - b)) < len)
             --b;
         bin_rows[b].push_back((int32_t)r);
     }
@@ -483,22 +485,23 @@ static sla_status current_device(sla_csr *A)
 // check the column pattern on the device.
 static sla_status setup_pattern(sla_csr *A, uint32_t flags, cudaStream_t s)
 {
-    A->h_rp.resize((size_t)A->n + 1);
-    SLA_CUDA_TRY(cudaMemcpyAsync(A->h_rp.data(), A->rp, ((size_t)A->n + 1) * sizeof(int32_t),
+    const int64_t np = pattern_rows(A);
+    A->h_rp.resize((size_t)np + 1);
+    SLA_CUDA_TRY(cudaMemcpyAsync(A->h_rp.data(), A->rp, ((size_t)np + 1) * sizeof(int32_t),
                                  cudaMemcpyDeviceToHost, s));
     SLA_CUDA_TRY(cudaStreamSynchronize(s));
     if (A->h_rp[0] != 0)
         return fail(SLA_ERR_INVALID_CSR, "row_ptr[0] must be 0");
-    if ((int64_t)A->h_rp[(size_t)A->n] != A->nnz)
+    if ((int64_t)A->h_rp[(size_t)np] != pattern_nnz(A))
         return fail(SLA_ERR_INVALID_CSR, "row_ptr[n] must equal nnz");
     int64_t mx = 0;
-    for (int64_t r = 0; r < A->n; ++r) {
+    for (int64_t r = 0; r < np; ++r) {
         const int64_t len = (int64_t)A->h_rp[r + 1] - A->h_rp[r];
         if (len < 0)
             return fail(SLA_ERR_INVALID_CSR, "row_ptr must be non-decreasing (row " + std::to_string(r) + ")");
         mx = std::max(mx, len);
     }
-    A->max_row_len = mx;
+    A->max_row_len = mx * A->bdim;          // scalar entries of the longest row
     if (flags & SLA_VALIDATE) {
         int *d_err = nullptr;
         SLA_CUDA_TRY(cudaMallocAsync((void **)&d_err, sizeof(int), s));
@@ -650,6 +653,49 @@ sla_status sla_csr_create(sla_csr **out, int64_t n_rows, int64_t n_cols, int64_t
     return SLA_SUCCESS;
 }
 
+sla_status sla_bsr_create(sla_csr **out, int64_t n_block_rows, int32_t block_dim, int64_t nnzb,
+                          const int32_t *d_row_ptr, const int32_t *d_col, const void *d_val,
+                          sla_dtype dtype, uint32_t flags, void *stream)
+{
+    if (!out)
+        return fail(SLA_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (block_dim < 2 || block_dim > 4)
+        return fail(SLA_ERR_INVALID_ARG, "block_dim must be 2, 3 or 4 (use sla_csr_create for 1)");
+    if (n_block_rows < 0 || nnzb < 0)
+        return fail(SLA_ERR_INVALID_ARG, "n_block_rows and nnzb must be >= 0");
+    const int64_t b = block_dim;
+    if (n_block_rows * b >= (int64_t)INT32_MAX || nnzb * b * b >= (int64_t)INT32_MAX)
+        return fail(SLA_ERR_INVALID_ARG, "scalar rows and values must fit int32 indices");
+    if (dtype != SLA_F32 && dtype != SLA_F64)
+        return fail(SLA_ERR_INVALID_ARG, "dtype must be SLA_F32 or SLA_F64");
+    if (!d_row_ptr || (nnzb > 0 && (!d_col || !d_val)))
+        return fail(SLA_ERR_INVALID_ARG, "NULL row_ptr, col or val");
+    if (((uintptr_t)d_row_ptr & 15) || ((uintptr_t)d_col & 15) || ((uintptr_t)d_val & 15))
+        return fail(SLA_ERR_INVALID_ARG, "row_ptr, col and val must be 16-byte aligned device pointers");
+    cudaStream_t s = (cudaStream_t)stream;
+    sla_csr *A = new sla_csr();
+    A->bdim = block_dim;
+    A->n = n_block_rows * b;
+    A->nnz = nnzb * b * b;
+    A->dtype = dtype;
+    A->flags = flags;
+    A->rp = d_row_ptr;
+    A->ci = d_col;
+    A->val = d_val;
+    A->max_sys_n = A->n;
+    A->max_sys_nnz = A->nnz;
+    sla_status st = current_device(A);
+    if (st == SLA_SUCCESS)
+        st = setup_pattern(A, flags, s);
+    if (st != SLA_SUCCESS) {
+        free_csr(A);
+        return st;
+    }
+    *out = A;
+    return SLA_SUCCESS;
+}
+
 sla_status sla_csr_create_list(sla_csr **out, int32_t batch, const int64_t *h_sys_row_off,
                                int64_t nnz_total, const int32_t *d_row_ptr, const int32_t *d_col,
                                const void *d_val, sla_dtype dtype, uint32_t flags, void *stream)
@@ -739,6 +785,8 @@ sla_status sla_spmv_multi(const sla_csr *A, int32_t nrhs, const void *d_X, void 
         return fail(SLA_ERR_INVALID_ARG, "NULL handle");
     if (nrhs < 1 || nrhs > KMAX)
         return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    if (A->bdim > 1 && nrhs > BSR_KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "a BSR matrix takes at most 4 right-hand sides");
     if (A->n > 0 && (!d_X || !d_Y || d_X == d_Y))
         return fail(SLA_ERR_INVALID_ARG, "NULL or overlapping X/Y");
     return launch_spmv(A, nrhs, d_X, d_Y, (cudaStream_t)stream);
@@ -890,6 +938,8 @@ sla_status sla_precond_spai(sla_precond **out, const sla_csr *A, const sla_csr *
     *out = nullptr;
     if (G->n != A->n || G->dtype != A->dtype)
         return fail(SLA_ERR_INVALID_ARG, "G must match A's size and dtype");
+    if (G->bdim > 1)
+        return fail(SLA_ERR_INVALID_ARG, "G must be a CSR matrix (A may be BSR)");
     if (!(eps >= 0.0))
         return fail(SLA_ERR_INVALID_ARG, "eps must be >= 0");
     sla_precond *M = new sla_precond();
@@ -999,6 +1049,8 @@ sla_status sla_pcg_solve_batched(const sla_csr *A, const sla_precond *M, int32_t
     }
     if (nrhs < 1 || nrhs > KMAX)
         return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    if (A->bdim > 1 && nrhs > BSR_KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "a BSR matrix takes at most 4 right-hand sides");
     if (A->n == 0) {
         for (int c = 0; c < nrhs; ++c)
             h_info[c] = sla_pcg_info{0, 0.0, SLA_SUCCESS, 0};
@@ -1031,6 +1083,8 @@ sla_status sla_pcg_adjoint_batched(const sla_csr *A, const sla_precond *M, int32
     }
     if (nrhs < 1 || nrhs > KMAX)
         return fail(SLA_ERR_INVALID_ARG, "nrhs must be in [1, 16]");
+    if (A->bdim > 1 && nrhs > BSR_KMAX)
+        return fail(SLA_ERR_INVALID_ARG, "a BSR matrix takes at most 4 right-hand sides");
     if (A->n == 0)
         return SLA_SUCCESS;
     int K = 1;

@@ -86,6 +86,30 @@ __global__ void k_jacobi_dinv(int64_t n, const int32_t *rp, const int32_t *ci, c
     }
 }
 
+// The same for a BSR matrix: the diagonal entries of scalar rows I*b .. I*b + b-1 sit on the
+// diagonal of block row I's diagonal block.
+template <typename VM>
+__global__ void k_bsr_dinv(int64_t nbr, int b, const int32_t *rp, const int32_t *ci, const VM *val,
+                           double *dinv64, float *dinv32, int *err)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t I = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; I < nbr; I += stride) {
+        int64_t kd = -1;
+        for (int64_t k = rp[I]; k < rp[I + 1]; ++k)
+            if (ci[k] == I)
+                kd = k;
+        for (int r = 0; r < b; ++r) {
+            const double d = kd >= 0 ? (double)val[kd * b * b + (int64_t)r * b + r] : 0.0;
+            const double inv = d > 0.0 ? 1.0 / d : 0.0;
+            if (!(d > 0.0))
+                atomicOr(err, 1);
+            dinv64[I * b + r] = inv;
+            if (dinv32)
+                dinv32[I * b + r] = (float)inv;
+        }
+    }
+}
+
 template <typename V>
 __global__ void k_gather_values(int64_t nnz, const int32_t *perm, const V *src, V *dst)
 {
@@ -113,7 +137,8 @@ sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s)
 {
     if (A->n == 0)
         return SLA_SUCCESS;
-    k_validate<<<vec_grid(A), 256, 0, s>>>(A->n, A->rp, A->ci, A->d_sys_off, A->batch, d_err);
+    // the stored pattern: block rows and block columns of a BSR matrix
+    k_validate<<<vec_grid(A), 256, 0, s>>>(pattern_rows(A), A->rp, A->ci, A->d_sys_off, A->batch, d_err);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
 }
@@ -122,6 +147,18 @@ sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv64, void *dinv32, int 
 {
     if (A->n == 0)
         return SLA_SUCCESS;
+    if (A->bdim > 1) {
+        if (A->dtype == SLA_F32)
+            k_bsr_dinv<float><<<vec_grid(A), 256, 0, s>>>(pattern_rows(A), A->bdim, A->rp, A->ci,
+                                                          (const float *)A->val, (double *)dinv64,
+                                                          (float *)dinv32, d_err);
+        else
+            k_bsr_dinv<double><<<vec_grid(A), 256, 0, s>>>(pattern_rows(A), A->bdim, A->rp, A->ci,
+                                                           (const double *)A->val, (double *)dinv64,
+                                                           nullptr, d_err);
+        SLA_CUDA_TRY(cudaGetLastError());
+        return SLA_SUCCESS;
+    }
     if (A->dtype == SLA_F32)
         k_jacobi_dinv<float><<<vec_grid(A), 256, 0, s>>>(A->n, A->rp, A->ci, (const float *)A->val,
                                                          (double *)dinv64, (float *)dinv32, d_err);

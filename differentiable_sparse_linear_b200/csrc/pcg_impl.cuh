@@ -14,6 +14,7 @@
 #include "persist.cuh"
 #include "row_engine.cuh"
 #include "tile_engine.cuh"
+#include "bsr.cuh"
 
 namespace sla {
 
@@ -330,10 +331,11 @@ struct TileLaunch {
     // sides; above that, block-owned tiles (a lane's gathers would not fit its registers)
     static constexpr bool LANE_GROUPS = K <= 4;
     int grid = 0;
-    int maxl = 0;                 // 0: tile engine; -1: lane-group engine; else the short-row MAXL
+    int maxl = 0;                 // 0: tile engine; -1: lane groups; -2: BSR lane groups; else the short-row MAXL
     MatView<VM> m{};
     const WinDesc *win = nullptr; // operand windows (short-row engine, K <= 2)
     GroupView gv{};               // length-grouped rows (lane-group engine)
+    int bdim = 1;                 // BSR block size (maxl == -2)
 
     template <int MAXL>
     sla_status setup_rows(const sla_csr *A, cudaStream_t s)
@@ -356,8 +358,42 @@ struct TileLaunch {
         return SLA_SUCCESS;
     }
 
+    template <int B>
+    sla_status setup_bsr(const sla_csr *A, cudaStream_t s)
+    {
+        const GroupPart *gp;
+        SLA_TRY(ensure_groups(const_cast<sla_csr *>(A), s, &gp));
+        m = view<VM>(A, nullptr);
+        gv.rows = gp->d_rows;
+        for (int b = 0; b <= GBINS; ++b) {
+            gv.task0[b] = gp->task0[b];
+            gv.pos0[b] = gp->pos0[b];
+        }
+        gv.n_tasks = gp->n_tasks;
+        int per_sm = 0;
+        SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_bsr_group<K, VM, B, Op>,
+                                                                   BsrCfg<K, B, VM, Op>::T, 0));
+        per_sm = std::max(per_sm, 1);
+        const int per_block = BsrCfg<K, B, VM, Op>::T / 32;
+        grid = std::max(1, std::min((gp->n_tasks + per_block - 1) / per_block, per_sm * A->num_sms));
+        bdim = B;
+        maxl = -2;
+        return SLA_SUCCESS;
+    }
+
     sla_status setup(const sla_csr *A, cudaStream_t s)
     {
+        if (A->bdim > 1) {
+            if constexpr (LANE_GROUPS) {
+                switch (A->bdim) {
+                case 2: return setup_bsr<2>(A, s);
+                case 3: return setup_bsr<3>(A, s);
+                case 4: return setup_bsr<4>(A, s);
+                default: return fail(SLA_ERR_INVALID_ARG, "BSR block size must be 2, 3 or 4");
+                }
+            }
+            return fail(SLA_ERR_INVALID_ARG, "a BSR matrix takes at most 4 right-hand sides");
+        }
         if (A->max_row_len <= ROWS_MAXL) {
             if (A->max_row_len <= 4)
                 return setup_rows<4>(A, s);
@@ -398,7 +434,7 @@ struct TileLaunch {
     }
     void launch(cudaStream_t s, const Op &op, double *part, PcgState *st, int *err) const
     {
-        if (maxl == -1 ? gv.n_tasks == 0 : m.n_tiles == 0)
+        if (maxl < 0 ? gv.n_tasks == 0 : m.n_tiles == 0)
             return;
         // windows are bulk-copied from the gathered vectors: they need 16-byte alignment
         bool aligned = true;
@@ -413,6 +449,16 @@ struct TileLaunch {
         case -1:
             if constexpr (LANE_GROUPS)
                 k_rowgroup<K, VM, Op><<<grid, GroupCfg<K, Op>::T, 0, s>>>(m, gv, op, part, st);
+            break;
+        case -2:
+            if constexpr (LANE_GROUPS) {
+                if (bdim == 2)
+                    k_bsr_group<K, VM, 2, Op><<<grid, BsrCfg<K, 2, VM, Op>::T, 0, s>>>(m, gv, op, part, st);
+                else if (bdim == 3)
+                    k_bsr_group<K, VM, 3, Op><<<grid, BsrCfg<K, 3, VM, Op>::T, 0, s>>>(m, gv, op, part, st);
+                else if (bdim == 4)
+                    k_bsr_group<K, VM, 4, Op><<<grid, BsrCfg<K, 4, VM, Op>::T, 0, s>>>(m, gv, op, part, st);
+            }
             break;
         default:
             if constexpr (!LANE_GROUPS)
@@ -442,7 +488,7 @@ template <typename V, int K>
 static sla_status spmv_k(const sla_csr *A, int nc, const void *x, void *y, cudaStream_t s)
 {
     // short rows: CSR-direct product over the slice descriptors
-    if (A->n > 0 && A->batch == 1 && A->max_row_len <= 16 && K <= 4) {
+    if (A->n > 0 && A->batch == 1 && A->bdim == 1 && A->max_row_len <= 16 && K <= 4) {
         if (A->max_row_len <= 8)
             return spmv_slices_k<V, K, 8>(A, nc, x, y, s);
         return spmv_slices_k<V, K, 16>(A, nc, x, y, s);
@@ -460,6 +506,20 @@ template <typename VM, typename VV>
 static sla_status grad_v(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g,
                          cudaStream_t s)
 {
+    if (A->bdim > 1) {
+        const int64_t nbr = pattern_rows(A);
+        if (nbr == 0 || A->nnz == 0)
+            return SLA_SUCCESS;
+        const int grid = A->num_sms * 8;
+        if (A->bdim == 2)
+            k_bsr_grad<VM, VV, 2><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g);
+        else if (A->bdim == 3)
+            k_bsr_grad<VM, VV, 3><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g);
+        else
+            k_bsr_grad<VM, VV, 4><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g);
+        SLA_CUDA_TRY(cudaGetLastError());
+        return SLA_SUCCESS;
+    }
     const TilePart *tp;
     SLA_TRY(ensure_tiles(const_cast<sla_csr *>(A), GRAD_D, GRAD_D, s, &tp));
     if (tp->n_tiles == 0)
@@ -681,7 +741,7 @@ constexpr bool persist_compiled()
 template <typename VV, int K>
 static int persist_maxl(const sla_csr *A, const Plan *p)
 {
-    if (K > 8 || A->batch > 1 || A->n == 0 || A->nnz == 0)
+    if (K > 8 || A->batch > 1 || A->n == 0 || A->nnz == 0 || A->bdim > 1)
         return 0;
     int64_t L = A->max_row_len;
     if (p->kind == 2) {

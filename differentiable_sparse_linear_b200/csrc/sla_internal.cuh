@@ -31,6 +31,7 @@ sla_status cuda_fail(cudaError_t e, const char *what);
 
 // ------------------------------------------------------------------ limits
 constexpr int KMAX = 16;            // right-hand sides handled by one solve
+constexpr int BSR_KMAX = 4;         // ... with a BSR matrix
 constexpr int NPMAX = 2;            // dot products one kernel reduces per right-hand side
 
 // ------------------------------------------------------------------ device solver state
@@ -79,7 +80,8 @@ struct TilePart {
 
 // Rows of a long-row matrix grouped by length for the lane-group SpMV: a row of len entries
 // goes to a group of G lanes, G the smallest power of two with 4 G >= len (G = 1 up to 32;
-// rows longer than 128 entries get a whole warp).  The rows of one G form a bin; bins are
+// rows longer than 128 entries get a whole warp).  For a BSR matrix the rows are block rows,
+// len counts blocks and the factor is 2 (a lane takes two blocks per pass).  The rows of one G form a bin; bins are
 // ordered G = 32, 16, ..., 1, and a warp task is 32 / G consecutive rows of one bin.  In
 // the G = 32 bin rows are ordered by length, longest first, elsewhere by index.
 constexpr int GBINS = 6;
@@ -155,6 +157,9 @@ struct sla_csr {
     const int32_t *rp = nullptr;
     const int32_t *ci = nullptr;
     const void *val = nullptr;
+    // block sparse rows: rp / ci index bdim x bdim blocks (row-major values), n and nnz count
+    // scalar rows and values; 1 for CSR
+    int32_t bdim = 1;
     // owned arrays (used by the internal G^T handle)
     int32_t *own_rp = nullptr, *own_ci = nullptr;
     void *own_val = nullptr;
@@ -192,6 +197,10 @@ struct sla_precond {
 };
 
 namespace sla {
+
+// Rows and entries of the stored pattern (blocks for a BSR matrix).
+inline int64_t pattern_rows(const sla_csr *A) { return A->n / A->bdim; }
+inline int64_t pattern_nnz(const sla_csr *A) { return A->nnz / ((int64_t)A->bdim * A->bdim); }
 
 // Solve plan: workspace + captured graph for one (A, M, K) combination.
 struct Plan {

@@ -485,6 +485,24 @@ __device__ __forceinline__ void group_row_sum(const MatView<VM> &m, const Op &op
     }
 }
 
+// This lane's row position in task t (-1: none) and the task's bin.  Static indices only,
+// so the bin table stays in the parameter bank.
+__device__ __forceinline__ int group_locate(const GroupView &g, int t, int lane, int &bin)
+{
+    int b = 0, t0 = g.task0[0], p0 = g.pos0[0], p1 = g.pos0[1];
+#pragma unroll
+    for (int i = 1; i < GBINS; ++i)
+        if (t >= g.task0[i]) {
+            b = i;
+            t0 = g.task0[i];
+            p0 = g.pos0[i];
+            p1 = g.pos0[i + 1];
+        }
+    bin = b;
+    const int pos = p0 + ((t - t0) << b) + (lane >> (GBINS - 1 - b));
+    return pos < p1 ? pos : -1;
+}
+
 template <int K, typename VM, class Op>
 __global__ void __launch_bounds__(GroupCfg<K, Op>::T, GroupCfg<K, Op>::MINB)
 k_rowgroup(const MatView<VM> m, const GroupView g, const Op op, double *partials, PcgState *st)
@@ -511,22 +529,7 @@ k_rowgroup(const MatView<VM> m, const GroupView g, const Op op, double *partials
     for (int i = 0; i < (NPK > 0 ? NPK : 1); ++i)
         part[i] = 0.0;
 
-    // this lane's row position in task t (-1: none) and the task's bin
-    // (static indices only: the bin table stays in the parameter bank)
-    auto locate = [&](int t, int &bin) {
-        int b = 0, t0 = g.task0[0], p0 = g.pos0[0], p1 = g.pos0[1];
-#pragma unroll
-        for (int i = 1; i < GBINS; ++i)
-            if (t >= g.task0[i]) {
-                b = i;
-                t0 = g.task0[i];
-                p0 = g.pos0[i];
-                p1 = g.pos0[i + 1];
-            }
-        bin = b;
-        const int pos = p0 + ((t - t0) << b) + (lane >> (GBINS - 1 - b));
-        return pos < p1 ? pos : -1;
-    };
+    auto locate = [&](int t, int &bin) { return group_locate(g, t, lane, bin); };
     const int nw = gridDim.x * NW;
     int t = blockIdx.x * NW + (tid >> 5);
     int bin = 0, pos = t < g.n_tasks ? locate(t, bin) : -1;

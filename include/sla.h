@@ -149,6 +149,24 @@ SLA_API sla_status sla_csr_create_list(sla_csr **out, int32_t batch, const int64
                                int64_t nnz_total, const int32_t *d_row_ptr, const int32_t *d_col,
                                const void *d_val, sla_dtype dtype, uint32_t flags, void *stream);
 
+/* One square block sparse row (BSR) matrix: dense block_dim x block_dim blocks on a CSR
+ * pattern of blocks ([SM] "Efficient Sparse Matrix Algebra in Python for Mathematics", Key
+ * sparse formats and memory tradeoffs; Block sparse patterns and sharding strategies: one
+ * index per dense block).  block_dim is 2, 3 or 4 (SLA_ERR_INVALID_ARG otherwise; use
+ * sla_csr_create for 1).  d_row_ptr (n_block_rows+1) and d_col (nnzb) index blocks, with
+ * nnzb = row_ptr[n_block_rows]; d_val holds nnzb*block_dim^2 values of `dtype`, block k
+ * row-major at d_val[k*block_dim^2], so scalar entry (I*b + r, col[k]*b + c) is
+ * d_val[k*b*b + r*b + c].  The scalar system has n = n_block_rows*block_dim rows and
+ * nnz = nnzb*block_dim^2 stored values (what sla_csr_shape reports, and the length of a
+ * gradient on the pattern, aligned with d_val).  Borrowing, alignment, immutability of the
+ * pattern and SLA_VALIDATE (on the block pattern) are as for sla_csr_create.  The handle
+ * works with sla_spmv, sla_spmv_multi and the batched solves up to 4 right-hand sides,
+ * sla_precond_jacobi (the scalar diagonal) and as A of sla_precond_spai (G must be CSR),
+ * the solves and adjoints (graph engine), and sla_pattern_grad. */
+SLA_API sla_status sla_bsr_create(sla_csr **out, int64_t n_block_rows, int32_t block_dim, int64_t nnzb,
+                          const int32_t *d_row_ptr, const int32_t *d_col, const void *d_val,
+                          sla_dtype dtype, uint32_t flags, void *stream);
+
 SLA_API sla_status sla_csr_destroy(sla_csr *A);
 
 /* n_rows, nnz and batch (1 for a single matrix) of a handle; any output may be NULL. */

@@ -95,6 +95,10 @@ class BSR:
     def nnz(self) -> int:
         return self.nnzb * self.b * self.b
 
+    @property
+    def batch(self) -> int:
+        return 1
+
     sys_row_off = None
 
 
