@@ -180,14 +180,19 @@ def measured_peaks() -> tuple[float, str]:
         return 6650.0, "fallback"
 
 
-KERNEL_SOURCES = ("row_engine.cuh", "tile_engine.cuh", "pcg_ops.cuh", "persist.cuh", "sell.cuh", "pcg_impl.cuh")
+# The files that define each profiled kernel's code: its ncu traffic stays valid while they
+# are unchanged (other kernels' sources do not move it).
+KERNEL_SOURCES = {
+    "k_pcg_persistent": ("persist.cuh", "sell.cuh", "pcg_ops.cuh"),
+    "q_spmv": ("tile_engine.cuh", "pcg_ops.cuh"),
+}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the sources that define the SpMV/PCG kernels (ncu traffic is tied to it)."""
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources that define a kernel (its ncu traffic is tied to it)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differentiable_sparse_linear_b200", "csrc")
-    for fn in KERNEL_SOURCES:
+    for fn in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -200,7 +205,9 @@ def profiled_traffic(kernel: str, workload: str, units: float = 1.0) -> int | No
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    src = kernel_source_hash()
+    if kernel not in KERNEL_SOURCES:
+        return None
+    src = kernel_source_hash(kernel)
     for ln in open(path):
         parts = ln.split()
         if len(parts) >= 4 and not ln.startswith("#") and parts[0] == kernel and parts[1] == workload:
