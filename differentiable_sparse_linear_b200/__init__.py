@@ -389,6 +389,8 @@ class _Solve(torch.autograd.Function):
         need_A = ctx.needs_input_grad[0]
         dLdb, dLdA, info = sla_pcg_adjoint(ctx.A, ctx.M, x, gx.contiguous(), want_dA=need_A,
                                            rtol=ctx.rtol, maxit=ctx.maxit, vector_f64=ctx.vf64)
+        if dLdA is not None:
+            dLdA = dLdA.view(ctx.A.val.shape)       # BSR values are [nnzb, b, b]
         return dLdA, dLdb, None, None, None, None, None
 
 
