@@ -89,7 +89,7 @@ def test_determinism():
     assert np.array_equal(a.G.val, b.G.val) and np.array_equal(a.B, b.B)
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5, 6])
 def test_workload_recipes_small(cfg):
     w = W.workload(cfg, "small")
     assert w.A.val.dtype == w.dtype
@@ -98,3 +98,46 @@ def test_workload_recipes_small(cfg):
     assert (w.G is not None) == (w.precond == "spai")
     if cfg == 3:
         assert w.B.shape == (w.A.n_rows, 8)
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_elastic_bsr_structure(b):
+    """The block vector problem: 7-point block pattern (7N^3 - 6N^2 blocks), symmetric, SPD,
+    row-major blocks with -S off the diagonal and 6 S + shift I on it."""
+    from oracle_checks import dense_bsr
+    N = 4
+    A = W.elastic3d_bsr(N, b, 0.1, np.float64)
+    assert A.n_rows == N ** 3 * b and A.nnzb == 7 * N ** 3 - 6 * N ** 2
+    assert np.all(np.diff(A.row_ptr) >= 4)
+    for I in range(A.n_brows):
+        cols = A.col[A.row_ptr[I]:A.row_ptr[I + 1]]
+        assert np.all(np.diff(cols) > 0) and I in cols
+    S = W.coupling_block(b)
+    rows = np.repeat(np.arange(A.n_brows), np.diff(A.row_ptr))
+    diag = rows == A.col
+    assert np.allclose(A.val[~diag], -S) and np.allclose(A.val[diag], 6 * S + 0.1 * np.eye(b))
+    D = dense_bsr(A)
+    assert np.array_equal(D, D.T)
+    assert np.linalg.eigvalsh(D).min() > 0
+
+
+def test_random_bsr_lengths():
+    lens = np.array([0, 3, 1, 0, 6, 2])
+    A = W.random_bsr(6, 3, lens, 9, np.float32)
+    assert np.array_equal(np.diff(A.row_ptr), lens) and A.val.shape == (lens.sum(), 3, 3)
+    for I in range(6):
+        cols = A.col[A.row_ptr[I]:A.row_ptr[I + 1]]
+        assert np.all(np.diff(cols) > 0) and np.all((cols >= 0) & (cols < 6))
+
+
+def test_bench_stream_bytes():
+    """bench.py's matrix-stream byte count: CSR values + indices + row pointers; BSR one index
+    and b*b values per block + block row pointers."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    A = W.elastic3d_bsr(5, 3, 0.1, np.float32)
+    assert bench.stream_bytes(A, 4) == A.nnzb * (9 * 4 + 4) + (A.n_brows + 1) * 4
+    C = W.poisson2d(9, np.float32)
+    assert bench.stream_bytes(C, 4) == C.nnz * 8 + (C.n_rows + 1) * 4
