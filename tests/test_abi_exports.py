@@ -51,6 +51,24 @@ def test_host_only_calls(libsla):
     assert libsla.sla_csr_create(ctypes.byref(h), 4, 5, 0, None, None, None, 0, 0, None) == -1
 
 
+def test_bsr_argument_checks(libsla):
+    """sla_bsr_create refuses bad block sizes, shapes and pointers before any device work."""
+    f = libsla.sla_bsr_create
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_uint32, ctypes.c_void_p]
+    h = ctypes.c_void_p()
+    assert f(None, 4, 3, 0, None, None, None, 0, 0, None) == -1               # out is NULL
+    for bdim in (0, 1, 5):
+        assert f(ctypes.byref(h), 4, bdim, 0, 16, None, None, 0, 0, None) == -1
+    assert f(ctypes.byref(h), -1, 3, 0, 16, None, None, 0, 0, None) == -1     # negative size
+    assert f(ctypes.byref(h), 2 ** 30, 3, 0, 16, None, None, 0, 0, None) == -1  # int32 overflow
+    assert f(ctypes.byref(h), 4, 3, 0, 16, None, None, 7, 0, None) == -1      # bad dtype
+    assert f(ctypes.byref(h), 4, 3, 5, 16, None, None, 0, 0, None) == -1      # nnzb > 0, no col
+    assert f(ctypes.byref(h), 4, 3, 0, 24, None, None, 0, 0, None) == -1      # row_ptr not 16-aligned
+    assert h.value is None
+
+
 def test_no_cpu_fallback_in_binding():
     """The binding has no arithmetic path of its own: it never imports the oracle."""
     pkg = os.path.join(ROOT, "differentiable_sparse_linear_b200")
