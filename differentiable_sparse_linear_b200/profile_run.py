@@ -43,6 +43,8 @@ def main(argv=None) -> int:
 
     if w.A.sys_row_off is not None:
         Ad = sla.sla_csr_create_list(list(w.A.sys_row_off), dev(w.A.row_ptr), dev(w.A.col), dev(w.A.val))
+    elif isinstance(w.A, W.BSR):
+        Ad = sla.sla_bsr_create(dev(w.A.row_ptr), dev(w.A.col), dev(w.A.val))
     else:
         Ad = sla.sla_csr_create(dev(w.A.row_ptr), dev(w.A.col), dev(w.A.val))
     if w.precond == "spai":
