@@ -176,7 +176,8 @@ SLA_API sla_status sla_csr_shape(const sla_csr *A, int64_t *n_rows, int64_t *nnz
  * overlap.  Accumulates each row in fp64 and rounds once to the value type. */
 SLA_API sla_status sla_spmv(const sla_csr *A, const void *d_x, void *d_y, void *stream);
 
-/* Y = A X for nrhs right-hand sides in [n][nrhs] layout (1 <= nrhs <= 16). */
+/* Y = A X for nrhs right-hand sides in [n][nrhs] layout (1 <= nrhs <= 16; a BSR handle
+ * takes at most 4, SLA_ERR_INVALID_ARG above). */
 SLA_API sla_status sla_spmv_multi(const sla_csr *A, int32_t nrhs, const void *d_X, void *d_Y, void *stream);
 
 /* ---------------------------------------------------------------- preconditioners */
@@ -232,7 +233,8 @@ SLA_API sla_status sla_pcg_adjoint_batched(const sla_csr *A, const sla_precond *
 
 /* dL/dA_k = -sum_c lambda_c,row(k) * x_c,col(k) on A's pattern, for nrhs vectors in
  * [n][nrhs] layout ([TS] Methodology §2; with lambda = x = v it is the Hellmann-Feynman
- * eigenvalue gradient of the same section up to sign). */
+ * eigenvalue gradient of the same section up to sign).  For a BSR handle k runs over the
+ * stored scalar values in d_val order (nnzb*b*b of them). */
 SLA_API sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *d_lam, const void *d_x,
                             void *d_g, void *stream);
 
