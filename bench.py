@@ -2,10 +2,10 @@
 
 One step = the whole hot path on one batch of synthetic input: the forward PCG solve
 x = A^-1 b, the adjoint solve A lambda = w (w = dL/dx for L = w.x) and the pattern
-gradient dL/dA_ij = -lambda_i x_j.  The default workload is the SPAI-preconditioned 2D
-Poisson problem (1024 x 1024 grid, fp32 values and vectors, fp64 reductions,
-M^-1 = G G^T + 3e-3 I, tolerance 1e-6).  value = PCG iterations (forward + adjoint) per
-second over all ranks.
+gradient dL/dA_ij = -lambda_i x_j.  The default workload is the largest single-GPU one:
+the SPAI-preconditioned power-law SPD system (n = 4,194,304, 212.7M stored entries, fp32
+values and vectors, fp64 reductions, M^-1 = G G^T + 3e-3 I, tolerance 1e-6).  value = PCG
+iterations (forward + adjoint) per second over all ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..6]
 
@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--size", default="full", choices=["full", "small", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-reps", type=int, default=20)
@@ -216,28 +216,46 @@ def profiled_traffic(kernel: str, workload: str, units: float = 1.0) -> int | No
     return None
 
 
-def cpu_baseline(w, budget_s: float = 15.0) -> dict:
-    """The fp64 oracle (single-threaded C) on a bounded sample: fixed PCG iterations."""
-    import oracle
-    ora = oracle.get()
+def _oracle_problem(ora, w):
+    """(A, b, preconditioner) of the workload as the oracle takes them: system 0 of a list,
+    a BSR matrix as its scalar CSR; the preconditioner (and G^T) is built once, outside any
+    timed region."""
     B = w.B if w.B.ndim == 1 else w.B[:, 0]
-    A = w.A
-    A = oracle_matrix(ora, A)
+    A = oracle_matrix(ora, w.A)
     if A.sys_row_off is not None:
         A = ora.system(A, 0)
         B = B[: A.n_rows]
-    kw = dict(precond=w.precond, G=w.G, eps=w.eps)
+    P = ora._precond(A, w.precond, w.G, w.eps)
+    return A, B, P
+
+
+def _time_oracle(ora, A, B, P, budget_s: float) -> tuple[int, float]:
+    """Fixed PCG iterations of the forward solve for about budget_s seconds: (iters, s)."""
     t0 = time.perf_counter()
-    ora.pcg(A, B, fixed_iters=5, **kw)
-    per = (time.perf_counter() - t0) / 5
-    iters = int(max(5, min(5000, budget_s / max(per, 1e-9))))
+    ora.pcg(A, B, fixed_iters=2, _P=P)
+    per = (time.perf_counter() - t0) / 2
+    iters = int(max(2, min(5000, budget_s / max(per, 1e-9))))
     t0 = time.perf_counter()
-    r = ora.pcg(A, B, fixed_iters=iters, **kw)
-    dt = time.perf_counter() - t0
-    return {"value": r.iters / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{r.iters} fixed PCG iterations of the forward solve on the same "
-                      f"{'system 0 of the ' if w.A.sys_row_off is not None else ''}workload "
-                      f"({dt:.1f} s, one host thread)"}
+    r = ora.pcg(A, B, fixed_iters=iters, _P=P)
+    return r.iters, time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s: float = 10.0) -> dict:
+    """The fp64 oracle on a bounded sample (fixed PCG iterations of the forward solve), once
+    on one host thread and once in its OpenMP build on every host core (same source, same
+    bits; row-parallel products and vector updates, sequential dot products)."""
+    import oracle
+    seq, par = oracle.get(), oracle.get_omp()
+    A, B, P = _oracle_problem(seq, w)
+    it1, dt1 = _time_oracle(seq, A, B, P, budget_s)
+    itn, dtn = _time_oracle(par, A, B, P, budget_s)
+    cores = os.cpu_count() or 1
+    part = "system 0 of the " if w.A.sys_row_off is not None else ""
+    return {"value": itn / dtn, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "value_1_thread": it1 / dt1,
+            "sample": f"fixed PCG iterations of the forward solve on {part}the same workload: "
+                      f"{itn} on all {cores} host cores (OpenMP build, {dtn:.1f} s) and {it1} on one "
+                      f"thread ({dt1:.1f} s); preconditioner set-up outside the timed sample"}
 
 
 # ------------------------------------------------------------------------- ranks
@@ -264,34 +282,29 @@ def run_reference(args):
     import sla_workloads as W
     w = W.workload(args.config, args.size)
     import oracle
-    ora = oracle.get()
-    B = w.B if w.B.ndim == 1 else w.B[:, 0]
-    A = w.A
-    A = oracle_matrix(ora, A)
-    if A.sys_row_off is not None:
-        A = ora.system(A, 0)
-        B = B[: A.n_rows]
-    kw = dict(precond=w.precond, G=w.G, eps=w.eps)
+    ora = oracle.get_omp()
+    A, B, P = _oracle_problem(ora, w)
     t0 = time.perf_counter()
-    ora.pcg(A, B, fixed_iters=3, **kw)
-    per = (time.perf_counter() - t0) / 3
-    per_step = int(max(3, min(2000, 2.0 / max(per, 1e-9))))     # about 2 s of CPU per step
+    ora.pcg(A, B, fixed_iters=2, _P=P)
+    per = (time.perf_counter() - t0) / 2
+    per_step = int(max(2, min(2000, 2.0 / max(per, 1e-9))))     # about 2 s of CPU per step
     for _ in range(args.warmup):
-        ora.pcg(A, B, fixed_iters=per_step, **kw)
+        ora.pcg(A, B, fixed_iters=per_step, _P=P)
     t0 = time.perf_counter()
     total = 0
     for _ in range(args.steps):
-        total += ora.pcg(A, B, fixed_iters=per_step, **kw).iters
+        total += ora.pcg(A, B, fixed_iters=per_step, _P=P).iters
     dt = time.perf_counter() - t0
     value = total / dt
-    sample = (f"{per_step} fixed forward PCG iterations per step of the fp64 oracle on "
-              f"{w.name} (one host thread)")
+    cores = os.cpu_count() or 1
+    sample = (f"{per_step} fixed forward PCG iterations per step of the fp64 oracle (OpenMP build, "
+              f"all {cores} host cores) on {w.name}; preconditioner set-up outside the timed steps")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": w.name, "n": int(A.n_rows), "nnz": int(A.nnz)},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -363,9 +376,19 @@ def run_ours(args):
     lam_buf = torch.empty_like(b)
     g_buf = torch.empty(A.nnz, dtype=va.dtype, device=dev)
 
-    def step(bv, wv, x_out):
+    fwd_events = []                 # (start, end) CUDA events around each forward solve
+    fwd_iters = []                  # its iterations (single systems)
+
+    def step(bv, wv, x_out, record=False):
+        if record:
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            fwd_events.append((f0, f1))
+            f0.record()
         if multi:
             x, inf = sla.sla_pcg_solve_batched(Ad, M, bv, x_out, rtol=w.tol, engine=args.engine)
+            if record:
+                fwd_events[-1][1].record()
             lam, g, ainf = sla.sla_pcg_adjoint_batched(Ad, M, x, wv, rtol=w.tol, engine=args.engine,
                                                        dLdB=lam_buf, dLdA=g_buf)
             engines_seen.update(i.engine for i in inf + ainf)
@@ -375,6 +398,9 @@ def run_ours(args):
             return (sum(i.iters for i in inf) + sum(i.iters for i in ainf),
                     launches(it[0], inf[0].engine) + launches(it[1], ainf[0].engine) + 1, x, lam)
         x, inf = sla.sla_pcg_solve(Ad, M, bv, x_out, rtol=w.tol, engine=args.engine)
+        if record:
+            fwd_events[-1][1].record()
+        fwd_iters.append(inf.iters)
         lam, g, ainf = sla.sla_pcg_adjoint(Ad, M, x, wv, rtol=w.tol, engine=args.engine, dLdb=lam_buf, dLdA=g_buf)
         engines_seen.update((inf.engine, ainf.engine))
         if inf.status != 0 or ainf.status != 0:
@@ -382,13 +408,24 @@ def run_ours(args):
         return (inf.iters + ainf.iters, launches(inf.iters, inf.engine) + launches(ainf.iters, ainf.engine) + 1,
                 x, lam)
 
-    # L2 flush between timed launches: write 512 MiB (evicts every line of ours), then read
-    # 256 MiB so the lines the write dirtied are back in HBM before the next timed launch
-    # (otherwise that launch would pay their write-back)
+    # Between timed steps the L2 (126 MB) must not hold this step's inputs.  Workloads whose
+    # matrices stream well over the L2's size per product evict it themselves; the others
+    # are flushed: write 512 MiB (evicts every line of ours), then read 256 MiB so the lines
+    # the write dirtied are back in HBM before the next timed launch (otherwise that launch
+    # would pay their write-back).  The flush runs inside the timed step; its two kernels
+    # are torch's, not counted in gpu_launches.
+    L2_BYTES = 126 << 20
+    big = stream_bytes(A, vbytes(w.dtype)) > 4 * L2_BYTES
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     drain = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+    l2_note = (f"no flush: inputs larger than L2 (the matrix streams "
+               f"{stream_bytes(A, vbytes(w.dtype)) / 1e9:.2f} GB per product, L2 is 126 MB)" if big else
+               "flushed between steps inside the timed step (512 MiB write, then a 256 MiB read that "
+               "writes the dirtied lines back; 2 torch kernels per step, not in gpu_launches)")
 
-    def flush_l2():
+    def flush_l2(force=False):
+        if big and not force:
+            return
         flush.zero_()
         drain.sum()
 
@@ -419,9 +456,10 @@ def run_ours(args):
     gc.disable()            # no collector pause inside the timed region
     t_begin = clocks.mark()
     ev0.record()
+    fwd_iters.clear()
     for k in range(args.steps):
         flush_l2()
-        it, nl, _, _ = step(b, wl, X)
+        it, nl, _, _ = step(b, wl, X, record=True)
         evs[k].record()
         total_iters += it
         total_launch += nl
@@ -545,6 +583,9 @@ def run_ours(args):
                             "nnz_s*(s_v+4) + (n_s+1)*4 + 13*n_s*s_v (streaming form; the kernel keeps "
                             "each system's vectors in shared memory)"}
     elif not is_list:
+        # graph engine: every kernel of one iteration launched alone in loop order, each
+        # bracketed by CUDA events on the launching stream (the loop itself runs inside a
+        # graph, where events cannot bracket single kernels)
         kt = sla.sla_pcg_kernel_times(Ad, M, nrhs, reps=args.kernel_reps)
         names = list(kernel_bytes(w))
         kb = kernel_bytes(w)
@@ -556,6 +597,24 @@ def run_ours(args):
         roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
                     "frac": ach / peak, "traffic": tr, "peak_source": peak_kind,
                     "algorithmic_bytes": kb[dom], "ms_per_launch": kernels[dom]["ms"]}
+    iteration = None
+    if not is_list and fwd_events:
+        # the full PCG iteration, measured live: the forward solves of the timed steps (CUDA
+        # events on the solve stream around each solve call, which also holds the solve's
+        # small set-up and copy-out kernels) against the algorithmic bytes of the iterations
+        # they ran -- one product with A, and with SPAI one with G^T and one with G, plus 16
+        # vector passes (SPAI) or 13 (Jacobi) of n x nrhs elements
+        fwd_ms = sum(a.elapsed_time(b_) for a, b_ in fwd_events)
+        sv = vbytes(w.dtype)
+        per_iter = stream_bytes(A, sv) + (16 if spai else 13) * A.n_rows * nrhs * sv
+        if spai:
+            per_iter += 2 * matrix_bytes(A.n_rows, w.G.nnz, sv)
+        its = sum(fwd_iters)
+        ach_i = per_iter * its / (fwd_ms * 1e6)
+        iteration = {"bound": "hbm", "achieved": ach_i, "peak": peak, "unit": "GB/s", "frac": ach_i / peak,
+                     "bytes_per_iteration": per_iter, "iterations": its, "ms": fwd_ms,
+                     "ms_per_iteration": fwd_ms / max(its, 1), "peak_source": peak_kind,
+                     "timing": "forward solves inside the timed steps, CUDA events on the solve stream"}
     if not is_list:
         # standalone SpMV y = A x, L2 flushed before each launch
         xs = torch.randn(A.n_rows * nrhs, dtype=va.dtype, device=dev).reshape(b.shape)
@@ -563,7 +622,7 @@ def run_ours(args):
         tot = 0.0
         reps = 20
         for r in range(reps + 2):
-            flush_l2()
+            flush_l2(force=True)
             s0 = torch.cuda.Event(enable_timing=True)
             s1 = torch.cuda.Event(enable_timing=True)
             s0.record()
@@ -597,11 +656,11 @@ def run_ours(args):
                        "iters_per_step": iters_per_step,
                        "step": "forward PCG solve + adjoint PCG solve + pattern gradient",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed between steps (512 MiB write, then a 256 MiB read that writes the dirtied lines back)", "setup_s": setup_s,
+                       "l2": l2_note, "setup_s": setup_s,
                        "engine": "+".join(sorted(engines_seen))},
             "step_ms": {"min": min(step_ms), "median": float(np.median(step_ms)), "max": max(step_ms),
                         "argmax": int(np.argmax(step_ms))},
-            "roofline": roofline, "spmv": spmv, "kernels": kernels,
+            "roofline": roofline, "iteration_roofline": iteration, "spmv": spmv, "kernels": kernels,
             "gpu_launches": total_launch, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -28,7 +28,7 @@ __all__ = [
     "sla_version", "sla_csr_create", "sla_bsr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
-    "sla_pcg_solve_batched_noalloc",
+    "sla_pcg_solve_batched_noalloc", "sla_eigen_grad", "sla_csr_add_diagonal", "sla_nonlinear_adjoint",
     "sla_workspace_bytes", "sla_pcg_kernel_times", "sla_pcg_phase_times", "solve",
     "ENGINES",
 ]
@@ -345,6 +345,45 @@ def sla_pattern_grad(A: Matrix, lam: torch.Tensor, x: torch.Tensor, g: Optional[
     _check(lib().sla_pattern_grad(A.handle, nrhs, _ptr(lam), _ptr(x), _ptr(g), _stream(stream)),
            "sla_pattern_grad")
     return g
+
+
+def sla_eigen_grad(A: Matrix, V: torch.Tensor, g: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """d mu / d A_k = v_row(k) v_col(k) on A's pattern for unit eigenvector(s) V ([n] or
+    [n, nvec]; summed over the columns)."""
+    nvec = 1 if V.dim() == 1 else V.shape[1]
+    _check_vec(A, V, False)
+    g = torch.empty(A.nnz, dtype=A.dtype, device=V.device) if g is None else g
+    _check(lib().sla_eigen_grad(A.handle, nvec, _ptr(V), _ptr(g), _stream(stream)), "sla_eigen_grad")
+    return g
+
+
+def sla_csr_add_diagonal(A: Matrix, c: torch.Tensor, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Values of A + diag(c) on A's pattern (e.g. a Jacobian J = A + diag(N'(u)))."""
+    _check_vec(A, c, False)
+    out = torch.empty_like(A.val.reshape(-1)) if out is None else out
+    _check(lib().sla_csr_add_diagonal(A.handle, _ptr(c), _ptr(out), _stream(stream)), "sla_csr_add_diagonal")
+    return out
+
+
+def sla_nonlinear_adjoint(J: Matrix, M: Optional[Preconditioner], A: Optional[Matrix], u: torch.Tensor,
+                          dLdu: torch.Tensor, *, want_dA: bool = True, rtol: float = 0.0, maxit: int = 0,
+                          vector_f64: bool = False, engine: str = "auto", lam: Optional[torch.Tensor] = None,
+                          dLdA: Optional[torch.Tensor] = None, stream=None):
+    """Backward pass of F(u) = A u + N(u) - b = 0 at its solution u: solves J^T lambda = dL/du
+    (J = A + diag(N'(u)), SPD) and returns (lambda = dL/db, dL/dA on A's pattern or None, info)."""
+    _check_vec(J, dLdu, vector_f64)
+    lam = torch.empty_like(dLdu) if lam is None else lam
+    if want_dA and A is not None and dLdA is None:
+        dLdA = torch.empty(A.nnz, dtype=A.dtype, device=dLdu.device)
+    elif not want_dA or A is None:
+        dLdA = None
+    info = _lib.sla_pcg_info()
+    opts = _opts(rtol, maxit, vector_f64, engine)
+    _check(lib().sla_nonlinear_adjoint(J.handle, _mh(M), None if A is None else A.handle, _ptr(u), _ptr(dLdu),
+                                       _ptr(lam), _ptr(dLdA), C.byref(opts), C.byref(info), _stream(stream)),
+           "sla_nonlinear_adjoint")
+    return lam, dLdA, _infos([info])[0]
 
 
 def sla_pcg_kernel_times(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1, reps: int = 20,

@@ -65,6 +65,10 @@ SIGNATURES = {
     "sla_pcg_adjoint_batched": (_st, [_vp, _vp, C.c_int32, _vp, _vp, _vp, _vp,
                                       C.POINTER(sla_pcg_opts), C.POINTER(sla_pcg_info), _vp]),
     "sla_pattern_grad": (_st, [_vp, C.c_int32, _vp, _vp, _vp, _vp]),
+    "sla_eigen_grad": (_st, [_vp, C.c_int32, _vp, _vp, _vp]),
+    "sla_csr_add_diagonal": (_st, [_vp, _vp, _vp, _vp]),
+    "sla_nonlinear_adjoint": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, C.POINTER(sla_pcg_opts),
+                                    C.POINTER(sla_pcg_info), _vp]),
     "sla_pcg_solve_batched_noalloc": (_st, [_vp, _vp, _vp, _vp, C.POINTER(sla_pcg_opts),
                                             C.POINTER(sla_pcg_info), _vp]),
     "sla_pcg_kernel_times": (_st, [_vp, _vp, C.c_int32, C.c_int32, C.c_int32, C.POINTER(C.c_double), _vp]),

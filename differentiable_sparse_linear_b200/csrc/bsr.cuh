@@ -130,7 +130,8 @@ k_bsr_group(const MatView<VM> m, const GroupView g, const Op op, double *partial
 // in storage order (coalesced writes of g).
 template <typename VM, typename VV, int B>
 __global__ void __launch_bounds__(256)
-k_bsr_grad(int64_t nbr, const int32_t *rp, const int32_t *ci, int nrhs, const VV *lam, const VV *x, VM *g)
+k_bsr_grad(int64_t nbr, const int32_t *rp, const int32_t *ci, int nrhs, const VV *lam, const VV *x, VM *g,
+           double scale)
 {
     constexpr int BB = B * B;
     const int lane = threadIdx.x & 31;
@@ -145,7 +146,7 @@ k_bsr_grad(int64_t nbr, const int32_t *rp, const int32_t *ci, int nrhs, const VV
             double s = 0.0;
             for (int q = 0; q < nrhs; ++q)
                 s = __fma_rn((double)lam[i * nrhs + q], (double)x[j * nrhs + q], s);
-            g[k0 * BB + t] = (VM)(-s);
+            g[k0 * BB + t] = (VM)(scale * s);
         }
     }
 }

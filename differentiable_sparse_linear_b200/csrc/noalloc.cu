@@ -9,14 +9,14 @@
 //
 // The array is a file-scope __device__ array of NOALLOC_MAX_SYSTEMS results (1.5 MiB); every
 // GPU that loads the library holds it until the process exits.  Host code only holds a
-// stand-in for its name, so its device address is looked up once per device with
-// cudaGetSymbolAddress, on that device's first call.  Every call on a device shares the
-// array: calls that overlap on the GPU (different streams, or different host threads) race
-// on it and must be serialised by the caller.
+// stand-in for its name, so every call looks its device address up with
+// cudaGetSymbolAddress on the current device.  The address is not cached: a context that is
+// torn down and created again (cudaDeviceReset) can place the array elsewhere.  Every call
+// on a device shares the array: calls that overlap on the GPU (different streams, or
+// different host threads) race on it and must be serialised by the caller.
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "sla.h"
 #include "sla_internal.cuh"
@@ -29,29 +29,16 @@ sla_status launch_list_kernel(const sla_csr *A, const sla_precond *M, const void
 namespace {
 
 constexpr int NOALLOC_MAX_SYSTEMS = 65536;
-constexpr int NOALLOC_MAX_DEVICES = 64;
-
 static __device__ __align__(256) sla_pcg_info g_noalloc_info[NOALLOC_MAX_SYSTEMS];
 
-std::mutex g_lock;
-sla_pcg_info *g_info_addr[NOALLOC_MAX_DEVICES] = {};
-
-// Device address of g_noalloc_info on the current device (looked up on first use).
+// Device address of g_noalloc_info in the current device's context (a host-side lookup).
 sla_status noalloc_scratch(sla_pcg_info **out)
 {
-    int dev = 0;
-    SLA_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES)
-        return fail(SLA_ERR_UNSUPPORTED, "device ordinal beyond the no-allocation entry point's table");
-    std::lock_guard<std::mutex> g(g_lock);
-    if (!g_info_addr[dev]) {
-        void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_info);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaGetSymbolAddress of the fixed result array");
-        g_info_addr[dev] = (sla_pcg_info *)p;
-    }
-    *out = g_info_addr[dev];
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_info);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetSymbolAddress of the fixed result array");
+    *out = (sla_pcg_info *)p;
     return SLA_SUCCESS;
 }
 
@@ -79,14 +66,19 @@ extern "C" sla_status sla_pcg_solve_batched_noalloc(const sla_csr *A, const sla_
     cudaStream_t s = (cudaStream_t)stream;
     sla_pcg_info *d_info = nullptr;
     SLA_TRY(noalloc_scratch(&d_info));
-    // the array keeps the previous call's results: clear this call's slots first
-    SLA_CUDA_TRY(cudaMemsetAsync(d_info, 0, sizeof(sla_pcg_info) * (size_t)A->batch, s));
+    // the array keeps the previous call's results: fill this call's slots with a value that
+    // is no solver outcome (status -1), so a slot the kernel left unwritten cannot pass for
+    // a converged solve
+    SLA_CUDA_TRY(cudaMemsetAsync(d_info, 0xFF, sizeof(sla_pcg_info) * (size_t)A->batch, s));
     SLA_TRY(launch_list_kernel(A, M, d_B, d_X, opts, d_info, s));
     SLA_CUDA_TRY(cudaMemcpyAsync(h_info, d_info, sizeof(sla_pcg_info) * (size_t)A->batch,
                                  cudaMemcpyDeviceToHost, s));
     SLA_CUDA_TRY(cudaStreamSynchronize(s));
     sla_status worst = SLA_SUCCESS;
-    for (int i = 0; i < A->batch; ++i)
+    for (int i = 0; i < A->batch; ++i) {
+        if (h_info[i].status < 0)
+            return fail(SLA_ERR_CUDA, "the list solve left a system's result unwritten");
         worst = std::max(worst, (sla_status)h_info[i].status);
+    }
     return worst;
 }

@@ -126,11 +126,11 @@ sla_status launch_spmv(const sla_csr *A, int K, const void *x, void *y, cudaStre
 }
 
 sla_status launch_pattern_grad(const sla_csr *A, int nrhs, int vec64, const void *lam, const void *x,
-                               void *g, cudaStream_t s)
+                               void *g, cudaStream_t s, double scale)
 {
     if (A->dtype == SLA_F64)
-        return grad_dd(A, nrhs, lam, x, g, s);
-    return vec64 ? grad_fd(A, nrhs, lam, x, g, s) : grad_ff(A, nrhs, lam, x, g, s);
+        return grad_dd(A, nrhs, lam, x, g, scale, s);
+    return vec64 ? grad_fd(A, nrhs, lam, x, g, scale, s) : grad_ff(A, nrhs, lam, x, g, scale, s);
 }
 
 sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s)

@@ -26,9 +26,10 @@ sla_status run_ff(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double 
     SLA_DISPATCH_K(p->K, run_k, A, p, nrhs, B, X, tol, maxit, engine, s)
 }
 
-sla_status grad_ff(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g, cudaStream_t s)
+sla_status grad_ff(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g, double scale,
+                   cudaStream_t s)
 {
-    return grad_v<float, float>(A, nrhs, lam, x, g, s);
+    return grad_v<float, float>(A, nrhs, lam, x, g, scale, s);
 }
 
 static int pad_k(int nrhs)

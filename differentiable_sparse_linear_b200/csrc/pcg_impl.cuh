@@ -232,7 +232,7 @@ constexpr int GRAD_D = 2048;
 
 template <typename VM, typename VV>
 __global__ void __launch_bounds__(GRAD_T)
-k_pattern_grad(const MatView<VM> m, int nrhs, const VV *lam, const VV *x, VM *g)
+k_pattern_grad(const MatView<VM> m, int nrhs, const VV *lam, const VV *x, VM *g, double scale)
 {
     __shared__ int32_t s_rp[GRAD_D];
     for (int t = blockIdx.x; t < m.n_tiles; t += gridDim.x) {
@@ -264,7 +264,7 @@ k_pattern_grad(const MatView<VM> m, int nrhs, const VV *lam, const VV *x, VM *g)
             double s = 0.0;
             for (int c = 0; c < nrhs; ++c)
                 s = __fma_rn((double)lam[i * nrhs + c], (double)x[j * nrhs + c], s);
-            g[k0 + e] = (VM)(-s);
+            g[k0 + e] = (VM)(scale * s);
         }
         __syncthreads();
     }
@@ -504,7 +504,7 @@ static sla_status spmv_k(const sla_csr *A, int nc, const void *x, void *y, cudaS
 
 template <typename VM, typename VV>
 static sla_status grad_v(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g,
-                         cudaStream_t s)
+                         double scale, cudaStream_t s)
 {
     if (A->bdim > 1) {
         const int64_t nbr = pattern_rows(A);
@@ -512,11 +512,11 @@ static sla_status grad_v(const sla_csr *A, int nrhs, const void *lam, const void
             return SLA_SUCCESS;
         const int grid = A->num_sms * 8;
         if (A->bdim == 2)
-            k_bsr_grad<VM, VV, 2><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g);
+            k_bsr_grad<VM, VV, 2><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g, scale);
         else if (A->bdim == 3)
-            k_bsr_grad<VM, VV, 3><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g);
+            k_bsr_grad<VM, VV, 3><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g, scale);
         else
-            k_bsr_grad<VM, VV, 4><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g);
+            k_bsr_grad<VM, VV, 4><<<grid, 256, 0, s>>>(nbr, A->rp, A->ci, nrhs, (const VV *)lam, (const VV *)x, (VM *)g, scale);
         SLA_CUDA_TRY(cudaGetLastError());
         return SLA_SUCCESS;
     }
@@ -528,7 +528,7 @@ static sla_status grad_v(const sla_csr *A, int nrhs, const void *lam, const void
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_pattern_grad<VM, VV>, GRAD_T, 0);
     const int grid = std::max(1, std::min(tp->n_tiles, std::max(per_sm, 1) * A->num_sms));
     k_pattern_grad<VM, VV><<<grid, GRAD_T, 0, s>>>(view<VM>(A, tp), nrhs, (const VV *)lam,
-                                                   (const VV *)x, (VM *)g);
+                                                   (const VV *)x, (VM *)g, scale);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
 }

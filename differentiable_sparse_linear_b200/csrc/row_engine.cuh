@@ -410,6 +410,10 @@ k_rows_tma(const MatView<VM> m, const WinDesc *win, const Op op, double *partial
         int2 n0 = make_int2(0, 0), n1 = make_int2(0, 0);
         WinDesc nw;
         nw.nseg = 0;
+        int issued_phase[NST];             // phase parity of each stage's last issued copies
+#pragma unroll
+        for (int s = 0; s < NST; ++s)
+            issued_phase[s] = -1;
         if (blockIdx.x < m.n_tiles) {
             n0 = m.desc[blockIdx.x];
             n1 = m.desc[blockIdx.x + 1];
@@ -428,13 +432,20 @@ k_rows_tma(const MatView<VM> m, const WinDesc *win, const Op op, double *partial
             }
             mbar_wait_bounded(&empty_bar[rp.stage], rp.phase ^ 1u, err);
             E::issue(m, op, d0, d1, wd, smem + (size_t)rp.stage * PITCH, &full_bar[rp.stage], gate);
+            issued_phase[rp.stage] = (int)rp.phase;
             rp.next<NST>();
         }
-        // every copy has landed and been read before the block exits
+        // every copy has landed and been read before the block exits: the consumers release
+        // each stage after its copies landed; if a consumer's wait ran out instead, the
+        // stage's last copies may still be in flight, so wait (bounded) for their completion
+        // too -- no bulk copy may still write this block's shared memory after it exits
         for (int s = 0; s < NST; ++s) {
             mbar_wait_bounded(&empty_bar[rp.stage], rp.phase ^ 1u, err);
             rp.next<NST>();
         }
+        for (int s = 0; s < NST; ++s)
+            if (issued_phase[s] >= 0)
+                mbar_wait_bounded(&full_bar[s], (uint32_t)issued_phase[s], err);
         return;
     }
 

@@ -239,8 +239,10 @@ void destroy_plan(Plan *p);
 
 // launchers implemented in the .cu files
 sla_status launch_spmv(const sla_csr *A, int K, const void *x, void *y, cudaStream_t s);
+// g_k = scale * sum_c lam[row(k)][c] x[col(k)][c] on A's pattern (scale -1: the adjoint's
+// dL/dA; +1: the eigenvalue gradient).
 sla_status launch_pattern_grad(const sla_csr *A, int K, int vec64, const void *lam, const void *x,
-                               void *g, cudaStream_t s);
+                               void *g, cudaStream_t s, double scale = -1.0);
 sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s);
 sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv64, void *dinv32, int *d_err, cudaStream_t s);
 sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t *d_perm,
@@ -261,7 +263,7 @@ sla_status kernel_times(sla_csr *A, Plan *p, int nrhs, int reps, double *h_ms, c
     sla_status run_##T(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, double tol,            \
                        long long maxit, int engine, cudaStream_t s);                                \
     sla_status grad_##T(const sla_csr *A, int nrhs, const void *lam, const void *x, void *g,         \
-                        cudaStream_t s);
+                        double scale, cudaStream_t s);
 SLA_COMBO_DECL(ff)
 SLA_COMBO_DECL(dd)
 SLA_COMBO_DECL(fd)

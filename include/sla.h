@@ -238,6 +238,37 @@ SLA_API sla_status sla_pcg_adjoint_batched(const sla_csr *A, const sla_precond *
 SLA_API sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *d_lam, const void *d_x,
                             void *d_g, void *stream);
 
+/* Eigenvalue gradient by the Hellmann-Feynman theorem ([TS] Methodology §2, Eigenvalue
+ * Problems): for a simple eigenvalue mu of a symmetric A with unit eigenvector v,
+ * d mu / d A_ij = v_i v_j, formed on A's pattern only.  d_V holds nvec (>= 1) unit
+ * eigenvectors in [n][nvec] layout, A's dtype; d_g (nnz, aligned with A's values) receives
+ * g_k = sum_c V[row(k)][c] V[col(k)][c], the gradient of the sum of those eigenvalues.  The
+ * eigenvectors come from the caller (this library has no eigensolver).  Same kernel as
+ * sla_pattern_grad with the opposite sign; BSR handles give g in d_val order. */
+SLA_API sla_status sla_eigen_grad(const sla_csr *A, int32_t nvec, const void *d_V, void *d_g, void *stream);
+
+/* d_val_out = the values of A + diag(d_c) on A's pattern ([TS] Methodology §2, Nonlinear
+ * Systems: the Jacobian J = dF/du of F(u) = A u + N(u) - b with an elementwise N is
+ * A + diag(N'(u))).  d_c: n values of A's dtype; d_val_out: nnz values (caller-owned, not A's
+ * own array), usually the value array of a handle J created once on A's pattern arrays.
+ * Every row must store its diagonal (SLA_ERR_INVALID_ARG otherwise); CSR and list handles
+ * (SLA_ERR_UNSUPPORTED for BSR).  Synchronises `stream`.  A Jacobi preconditioner built on
+ * J must be refreshed (sla_precond_refresh) after J's values change. */
+SLA_API sla_status sla_csr_add_diagonal(const sla_csr *A, const void *d_c, void *d_val_out, void *stream);
+
+/* Backward pass of a nonlinear system F(u, theta) = 0 solved by the caller ([TS] Methodology
+ * §2, Nonlinear Systems): one adjoint solve J^T lambda = dL/du with the Jacobian J = dF/du at
+ * the solution u (J SPD, so the same PCG as sla_pcg_solve, with M built on J), then the
+ * vector-Jacobian product for F = A u + N(u) - b: dL/dA_k = -lambda_row(k) u_col(k) on A's
+ * pattern (A's values are the parameters) and dL/db = lambda.  d_lambda (n) receives lambda;
+ * A and d_dLdA may be NULL to skip the product; A must match J's size, dtype and batch (J
+ * may share A's pattern arrays).  The work does not depend on how many nonlinear iterations
+ * the forward solve took.  Single systems; vector types as sla_pcg_solve (opts->vector_f64). */
+SLA_API sla_status sla_nonlinear_adjoint(const sla_csr *J, const sla_precond *M, const sla_csr *A,
+                                         const void *d_u, const void *d_dLdu, void *d_lambda,
+                                         void *d_dLdA, const sla_pcg_opts *opts, sla_pcg_info *info,
+                                         void *stream);
+
 /* The list solve of sla_pcg_solve_batched (list handle, nrhs = 1, Jacobi or no
  * preconditioner) for callers that cannot allocate device memory while they solve --
  * code under a memory pool or budget that owns the device's memory, hosts that forbid
@@ -245,9 +276,12 @@ SLA_API sla_status sla_pattern_grad(const sla_csr *A, int32_t nrhs, const void *
  * free can bring.  This call allocates nothing: the per-system results pass through a
  * fixed array in the library's own device memory (1.5 MiB, held by every GPU that loads
  * the library until the process exits), and at most 65536 systems are accepted per call
- * (SLA_ERR_INVALID_ARG beyond that).  The first call on a device looks up that array's
- * device address, so make it before any stream capture.  All calls on a device share the
- * array: calls that overlap on the GPU race on it.  The matrix and preconditioner handles
+ * (SLA_ERR_INVALID_ARG beyond that).  Every call looks up that array's device address in
+ * the current context (cudaGetSymbolAddress, a host-side lookup; on a device's first call it
+ * can load the library's device code, so make that first call before any stream capture
+ * begins), fills this call's slots with status -1 and synchronises `stream` to read the
+ * results back into h_info.  All calls on a device share the array: calls that overlap on
+ * the GPU race on it.  The matrix and preconditioner handles
  * are created beforehand with the usual calls.  There is no counterpart on the pages this
  * library follows: it is an interface variant, not a different method. */
 SLA_API sla_status sla_pcg_solve_batched_noalloc(const sla_csr *A, const sla_precond *M,

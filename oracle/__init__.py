@@ -85,8 +85,16 @@ class Oracle:
                                 C.c_double, C.c_int64, C.c_int64, C.POINTER(C.c_int64),
                                 C.POINTER(C.c_double), C.c_void_p]
         lib.ora_pcg.restype = C.c_int
+        lib.ora_pcg_ex.argtypes = [C.c_int64, _i32p, _i32p, _f64p, C.POINTER(_Precond), _f64p, _f64p,
+                                   C.c_double, C.c_int64, C.c_int64, C.c_int32, C.POINTER(C.c_int64),
+                                   C.POINTER(C.c_double), C.c_void_p]
+        lib.ora_pcg_ex.restype = C.c_int
         lib.ora_pattern_grad.argtypes = [C.c_int64, _i32p, _i32p, _f64p, _f64p, _f64p]
         lib.ora_pattern_grad.restype = None
+        lib.ora_eigen_grad.argtypes = [C.c_int64, _i32p, _i32p, _f64p, _f64p]
+        lib.ora_eigen_grad.restype = None
+        lib.ora_add_diagonal.argtypes = [C.c_int64, _i32p, _i32p, _f64p, _f64p, _f64p]
+        lib.ora_add_diagonal.restype = C.c_int
         lib.ora_bsr_spmv.argtypes = [C.c_int64, C.c_int32, _i32p, _i32p, _f64p, _f64p, _f64p]
         lib.ora_bsr_spmv.restype = None
         lib.ora_bsr_to_csr.argtypes = [C.c_int64, C.c_int32, _i32p, _i32p, _f64p, _i32p, _i32p, _f64p,
@@ -129,6 +137,19 @@ class Oracle:
         self.lib.ora_pattern_grad(A.n_rows, _i32(A.row_ptr), _i32(A.col), _f64(lam), _f64(x), g)
         return g
 
+    def eigen_grad(self, A, v) -> np.ndarray:
+        """d mu / dA_ij = v_i v_j on A's stored entries (v a unit eigenvector of symmetric A)."""
+        g = np.empty(A.nnz, dtype=np.float64)
+        self.lib.ora_eigen_grad(A.n_rows, _i32(A.row_ptr), _i32(A.col), _f64(v), g)
+        return g
+
+    def add_diagonal(self, A, c):
+        """A + diag(c) on A's pattern (same class as A, fp64 values)."""
+        out = np.empty(A.nnz, dtype=np.float64)
+        if self.lib.ora_add_diagonal(A.n_rows, _i32(A.row_ptr), _i32(A.col), _f64(A.val), _f64(c), out) != 0:
+            raise ValueError("a row stores no diagonal entry")
+        return type(A)(A.n_rows, A.n_cols, _i32(A.row_ptr), _i32(A.col), out)
+
     # ---------------------------------------------------------------- preconditioners
     def _precond(self, A, kind: str, G=None, eps: float = 0.0):
         keep = []
@@ -165,8 +186,12 @@ class Oracle:
     # ---------------------------------------------------------------- solves
     def pcg(self, A, b, precond: str = "jacobi", G=None, eps: float = 0.0, tol: float = 1e-10,
             maxit: Optional[int] = None, fixed_iters: int = 0, history: bool = False,
-            _P=None) -> SolveResult:
-        """PCG from x0 = 0; maxit defaults to 10 * n."""
+            store_f32: bool = False, _P=None) -> SolveResult:
+        """PCG from x0 = 0; maxit defaults to 10 * n.
+
+        store_f32: the same recurrence with every vector it keeps rounded to binary32 when
+        formed (fp64 dot products and scalars) -- the arithmetic of fp32 vector storage, for
+        comparing iteration counts with a solver that stores its vectors in fp32."""
         n = A.n_rows
         maxit = 10 * max(n, 1) if maxit is None else int(maxit)
         P, keep = _P if _P is not None else self._precond(A, precond, G, eps)
@@ -176,15 +201,15 @@ class Oracle:
         rel = C.c_double(0.0)
         hlen = (fixed_iters if fixed_iters > 0 else maxit) + 1
         hist = np.zeros(hlen, dtype=np.float64) if history else None
-        st = self.lib.ora_pcg(n, _i32(A.row_ptr), _i32(A.col), _f64(A.val), C.byref(P), b, x,
-                              float(tol), maxit, int(fixed_iters), C.byref(it), C.byref(rel),
-                              hist.ctypes.data if history else None)
+        st = self.lib.ora_pcg_ex(n, _i32(A.row_ptr), _i32(A.col), _f64(A.val), C.byref(P), b, x,
+                                 float(tol), maxit, int(fixed_iters), 1 if store_f32 else 0,
+                                 C.byref(it), C.byref(rel), hist.ctypes.data if history else None)
         if history:
             hist = hist[: it.value + 1]
         return SolveResult(x, int(it.value), float(rel.value), int(st), hist)
 
     def adjoint(self, A, x, w, precond: str = "jacobi", G=None, eps: float = 0.0,
-                tol: float = 1e-10, maxit: Optional[int] = None) -> AdjointResult:
+                tol: float = 1e-10, maxit: Optional[int] = None, store_f32: bool = False) -> AdjointResult:
         """Solve A^T lam = w (w = dL/dx) by PCG; return dL/db = lam and dL/dA on the pattern.
 
         The transpose is formed explicitly, as the definition states it; M is the same
@@ -192,8 +217,21 @@ class Oracle:
         """
         At = self.transpose(A)
         P, keep = self._precond(A, precond, G, eps)
-        res = self.pcg(At, w, tol=tol, maxit=maxit, _P=(P, keep))
+        res = self.pcg(At, w, tol=tol, maxit=maxit, store_f32=store_f32, _P=(P, keep))
         g = self.grad(A, res.x, x)
+        return AdjointResult(res.x, g, res.iters, res.relres, res.status)
+
+    def nonlinear_adjoint(self, J, A, u, dLdu, precond: str = "jacobi", G=None, eps: float = 0.0,
+                          tol: float = 1e-10, maxit: Optional[int] = None, store_f32: bool = False):
+        """Backward pass of F(u) = A u + N(u) - b = 0 at its solution u ([TS] Methodology §2,
+        Nonlinear Systems): lambda solves J^T lambda = dL/du with the Jacobian J = dF/du
+        (PCG on the explicit transpose, preconditioner built on J), then the vector-Jacobian
+        product dL/dA_ij = -lambda_i u_j (A's values are parameters) and dL/db = lambda.
+        Returns AdjointResult(lam, grad on A's pattern, ...)."""
+        Jt = self.transpose(J)
+        P, keep = self._precond(J, precond, G, eps)
+        res = self.pcg(Jt, dLdu, tol=tol, maxit=maxit, store_f32=store_f32, _P=(P, keep))
+        g = self.grad(A, res.x, u)
         return AdjointResult(res.x, g, res.iters, res.relres, res.status)
 
     # ---------------------------------------------------------------- batches
@@ -299,3 +337,16 @@ def get() -> Oracle:
     if _default is None:
         _default = Oracle()
     return _default
+
+
+_omp: Optional[Oracle] = None
+
+
+def get_omp() -> Oracle:
+    """The same source built with OpenMP: independent row / element loops on every host
+    core, dot products sequential, results bit-identical to get()'s.  Only the benchmark's
+    CPU baseline uses it."""
+    global _omp
+    if _omp is None:
+        _omp = Oracle(_build.build_omp())
+    return _omp

@@ -22,6 +22,11 @@
  *  - Breakdown: p.q <= 0 or not finite, or r.z <= 0 or not finite for a residual that has
  *    not met the tolerance (A or M not SPD).
  *  - Every pin of these functions lives in the tests; none is "parity unpinned".
+ *
+ * Threads: build.py also compiles this same source with OpenMP (liboracle_omp.so), used
+ * only to time the CPU baseline on every host core.  The pragmas below split loops whose
+ * iterations are independent (rows of a product, elements of a vector update) over
+ * threads; dot products and norms stay sequential, so both builds give identical bits.
  */
 #include <math.h>
 #include <stdint.h>
@@ -36,6 +41,7 @@
 void ora_spmv(int64_t n_rows, const int32_t *row_ptr, const int32_t *col, const double *val,
               const double *x, double *y)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n_rows; ++i) {
         double s = 0.0;
         for (int64_t k = row_ptr[i]; k < row_ptr[i + 1]; ++k)
@@ -113,20 +119,41 @@ typedef struct {
     double eps;
 } ora_precond;
 
-void ora_precond_apply(int64_t n, const ora_precond *M, const double *r, double *z, double *work)
+/* Round every entry of v to the nearest binary32 value (kept in a double).  Used only by
+ * the fp32-storage mode of the solve below. */
+static void ora_round_f32(int64_t n, double *v)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        v[i] = (double)(float)v[i];
+}
+
+static void precond_apply(int64_t n, const ora_precond *M, const double *r, double *z, double *work,
+                          int store_f32)
 {
     if (M == NULL || M->kind == 0) {
         for (int64_t i = 0; i < n; ++i)
             z[i] = r[i];
     } else if (M->kind == 1) {
+#pragma omp parallel for schedule(static)
         for (int64_t i = 0; i < n; ++i)
             z[i] = r[i] / M->diag[i];
     } else {
         ora_spmv(n, M->gt_rp, M->gt_ci, M->gt_v, r, work);   /* y = G^T r */
+        if (store_f32)
+            ora_round_f32(n, work);
         ora_spmv(n, M->g_rp, M->g_ci, M->g_v, work, z);      /* z = G y   */
+#pragma omp parallel for schedule(static)
         for (int64_t i = 0; i < n; ++i)
             z[i] = z[i] + M->eps * r[i];                     /* + eps r   */
     }
+    if (store_f32)
+        ora_round_f32(n, z);
+}
+
+void ora_precond_apply(int64_t n, const ora_precond *M, const double *r, double *z, double *work)
+{
+    precond_apply(n, M, r, z, work, 0);
 }
 
 static int ora_finite(double a) { return a == a && a - a == 0.0; }
@@ -141,10 +168,17 @@ static int ora_finite(double a) { return a == a && a - a == 0.0; }
  * fixed_iters > 0 runs exactly that many iterations and ignores tol (lockstep checks).
  * hist (optional, maxit+1 or fixed_iters+1 doubles) receives ||r_k||/||b|| for k = 0.. .
  * Returns ORA_CONVERGED, ORA_NOT_CONVERGED or ORA_BREAKDOWN; *iters and *relres report
- * the last iteration and its relative recursive residual. */
-int ora_pcg(int64_t n, const int32_t *rp, const int32_t *ci, const double *v,
-            const ora_precond *M, const double *b, double *x, double tol, int64_t maxit,
-            int64_t fixed_iters, int64_t *iters, double *relres, double *hist)
+ * the last iteration and its relative recursive residual.
+ *
+ * store_f32 != 0 is the same recurrence with single-precision vector storage: every vector
+ * the iteration keeps (q, x, r, the SPAI intermediate y = G^T r, z and p) is rounded to the
+ * nearest binary32 value right after it is formed in fp64; dot products, norms and the
+ * scalars stay fp64.  It is the arithmetic of a solver that stores its vectors in fp32 with
+ * fp64 reductions, so the stopping decision (an integer: the iteration count) can be taken
+ * in that storage precision too. */
+int ora_pcg_ex(int64_t n, const int32_t *rp, const int32_t *ci, const double *v,
+               const ora_precond *M, const double *b, double *x, double tol, int64_t maxit,
+               int64_t fixed_iters, int32_t store_f32, int64_t *iters, double *relres, double *hist)
 {
     double *r = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
     double *z = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
@@ -160,7 +194,9 @@ int ora_pcg(int64_t n, const int32_t *rp, const int32_t *ci, const double *v,
         x[i] = 0.0;
         r[i] = b[i];
     }
-    bnorm = sqrt(ora_dot(n, b, b));
+    if (store_f32)
+        ora_round_f32(n, r);
+    bnorm = sqrt(ora_dot(n, r, r));
     *relres = 0.0;
     if (hist)
         hist[0] = bnorm > 0.0 ? 1.0 : 0.0;
@@ -169,7 +205,7 @@ int ora_pcg(int64_t n, const int32_t *rp, const int32_t *ci, const double *v,
         goto done;
     }
     *relres = 1.0;
-    ora_precond_apply(n, M, r, z, w);
+    precond_apply(n, M, r, z, w, store_f32);
     for (int64_t i = 0; i < n; ++i)
         p[i] = z[i];
     rho = ora_dot(n, r, z);
@@ -180,15 +216,22 @@ int ora_pcg(int64_t n, const int32_t *rp, const int32_t *ci, const double *v,
     while (k < limit) {
         k += 1;
         ora_spmv(n, rp, ci, v, p, q);
+        if (store_f32)
+            ora_round_f32(n, q);
         pq = ora_dot(n, p, q);
         if (!(pq > 0.0) || !ora_finite(pq)) {
             status = ORA_BREAKDOWN;
             break;
         }
         alpha = rho / pq;
+#pragma omp parallel for schedule(static)
         for (int64_t i = 0; i < n; ++i) {
             x[i] = x[i] + alpha * p[i];
             r[i] = r[i] - alpha * q[i];
+        }
+        if (store_f32) {
+            ora_round_f32(n, x);
+            ora_round_f32(n, r);
         }
         rnorm = sqrt(ora_dot(n, r, r));
         *relres = rnorm / bnorm;
@@ -202,15 +245,18 @@ int ora_pcg(int64_t n, const int32_t *rp, const int32_t *ci, const double *v,
             status = ORA_CONVERGED;
             break;
         }
-        ora_precond_apply(n, M, r, z, w);
+        precond_apply(n, M, r, z, w, store_f32);
         rho_new = ora_dot(n, r, z);
         if (!(rho_new > 0.0) || !ora_finite(rho_new)) {
             status = ORA_BREAKDOWN;
             break;
         }
         beta = rho_new / rho;
+#pragma omp parallel for schedule(static)
         for (int64_t i = 0; i < n; ++i)
             p[i] = z[i] + beta * p[i];
+        if (store_f32)
+            ora_round_f32(n, p);
         rho = rho_new;
     }
 done:
@@ -223,6 +269,14 @@ done:
     return status;
 }
 
+/* The fp64 solve (no rounding of the stored vectors). */
+int ora_pcg(int64_t n, const int32_t *rp, const int32_t *ci, const double *v,
+            const ora_precond *M, const double *b, double *x, double tol, int64_t maxit,
+            int64_t fixed_iters, int64_t *iters, double *relres, double *hist)
+{
+    return ora_pcg_ex(n, rp, ci, v, M, b, x, tol, maxit, fixed_iters, 0, iters, relres, hist);
+}
+
 /* Gradient of L with respect to the stored entries of A ([TS] Methodology §2, Linear
  * Systems): for every stored (i, j), dL/dA_ij = -lambda_i * x_j, where A^T lambda = dL/dx.
  * g is aligned with A's value array. */
@@ -232,6 +286,37 @@ void ora_pattern_grad(int64_t n_rows, const int32_t *rp, const int32_t *ci, cons
     for (int64_t i = 0; i < n_rows; ++i)
         for (int64_t k = rp[i]; k < rp[i + 1]; ++k)
             g[k] = -lam[i] * x[ci[k]];
+}
+
+/* Eigenvalue gradient ([TS] Methodology §2, Eigenvalue Problems, Hellmann-Feynman): for a
+ * simple eigenvalue mu of a symmetric A with unit eigenvector v, d mu / d A_ij = v_i v_j,
+ * evaluated on every stored (i, j); g is aligned with A's value array. */
+void ora_eigen_grad(int64_t n_rows, const int32_t *rp, const int32_t *ci, const double *v, double *g)
+{
+    for (int64_t i = 0; i < n_rows; ++i)
+        for (int64_t k = rp[i]; k < rp[i + 1]; ++k)
+            g[k] = v[i] * v[ci[k]];
+}
+
+/* out = the values of A + diag(c) on A's pattern (the Jacobian A + diag(N'(u)) of
+ * F(u) = A u + N(u) - b, [TS] Methodology §2, Nonlinear Systems).  Returns -1 if a row stores
+ * no diagonal entry. */
+int ora_add_diagonal(int64_t n_rows, const int32_t *rp, const int32_t *ci, const double *v,
+                     const double *c, double *out)
+{
+    for (int64_t i = 0; i < n_rows; ++i) {
+        int found = 0;
+        for (int64_t k = rp[i]; k < rp[i + 1]; ++k) {
+            out[k] = v[k];
+            if (ci[k] == i) {
+                out[k] = v[k] + c[i];
+                found = 1;
+            }
+        }
+        if (!found)
+            return -1;
+    }
+    return 0;
 }
 
 /* Block sparse row (BSR) storage -- [SM] "Efficient Sparse Matrix Algebra in Python for

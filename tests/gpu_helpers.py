@@ -44,6 +44,17 @@ def rel(a, b) -> float:
     return float(np.linalg.norm(a - b) / (d if d > 0 else 1.0))
 
 
+def relmax(a, b) -> float:
+    """Largest element error relative to the largest reference element (catches a single
+    wrong row that a 2-norm over millions of rows can hide)."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    if b.size == 0:
+        return 0.0
+    d = float(np.max(np.abs(b)))
+    return float(np.max(np.abs(a - b)) / (d if d > 0 else 1.0))
+
+
 def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy().astype(np.float64)
 

@@ -17,6 +17,14 @@ What pins what:
   * SPAI apply -- the dense product (G G^T + eps I) r.
   * adjoint    -- A lam = w; w.x = lam.b; sum A_ij g_ij = -L; central finite differences
                   of L = w.A^-1 b (dense LU) in single stored entries and in b.
+  * fp32 storage -- a hand-worked 2 x 2 case in which binary32 storage of q ends CG one
+                  step early with x exact; bit-exact agreement where every vector is exact
+                  in binary32; returned iterates are binary32 values and track the fp64
+                  recurrence to rounding for the first steps.
+  * eigenvalue gradient -- the closed-form 2D Poisson eigenpairs (v_i v_j and
+                  sum A_k g_k = mu) and central differences of a dense eigenvalue.
+  * nonlinear adjoint -- central differences of L = w.u for A u + u^3 = b solved by dense
+                  Newton, in single stored entries and in b; A + diag(c) against dense.
   * BSR        -- a dense matrix assembled block by block (numpy) for the block SpMV and the
                   scalar CSR expansion; closed-form eigenpairs of L (x) S + shift I (the
                   block vector problem) for the SpMV and one-step PCG; central finite
@@ -386,10 +394,152 @@ def check_bsr_grad_fd(ora):
         assert abs(adj.grad[k, r, c] - fd) <= 1e-7 * max(1.0, abs(fd)), f"BSR dL/dA block {k} ({r},{c})"
 
 
+# ------------------------------------------------------------------ fp32-storage mode
+def check_store_f32_worked_2x2(ora):
+    """A hand-worked case where binary32 storage of q = A p changes the iteration count.
+
+    A = diag(1, 1 + d) with d = 1e-9 (below half an fp32 ulp of 1), b = (1, 1), plain CG,
+    tol 1e-12.  fp64: q = (1, 1 + d), alpha = 2 / (2 + d), the residual after one step is
+    about d / 2 > tol, and CG ends at step 2 (two distinct eigenvalues).  fp32 storage: q
+    rounds to (1, 1), so alpha = 1, r = 0 and the solve ends after ONE step with x = (1, 1)
+    exactly."""
+    d = 1e-9
+    A = csr_from_dense(np.diag([1.0, 1.0 + d]))
+    b = np.array([1.0, 1.0])
+    r64 = ora.pcg(A, b, precond="none", tol=1e-12)
+    r32 = ora.pcg(A, b, precond="none", tol=1e-12, store_f32=True)
+    assert r64.status == 0 and r64.iters == 2, (r64.status, r64.iters)
+    assert abs(r64.x[1] - 1.0 / (1.0 + d)) <= 1e-15
+    assert r32.status == 0 and r32.iters == 1, (r32.status, r32.iters)
+    assert r32.x[0] == 1.0 and r32.x[1] == 1.0 and r32.relres == 0.0
+
+
+def check_store_f32_exact_case(ora):
+    """Where every stored vector is exact in binary32 the two modes agree bit for bit:
+    Jacobi on a diagonal matrix with power-of-two entries and small-integer b converges in
+    one step to x = b / diag, exactly."""
+    diag = np.array([1.0, 2.0, 4.0, 8.0, 0.5, 16.0])
+    A = csr_from_dense(np.diag(diag))
+    b = np.array([3.0, -2.0, 5.0, 1.0, -7.0, 12.0])
+    r64 = ora.pcg(A, b, precond="jacobi", tol=1e-12)
+    r32 = ora.pcg(A, b, precond="jacobi", tol=1e-12, store_f32=True)
+    assert r64.iters == r32.iters == 1
+    assert np.array_equal(r32.x, b / diag) and np.array_equal(r64.x, r32.x)
+
+
+def check_store_f32_rounds_and_tracks(ora):
+    """On the power-law SPAI recipe: every iterate the fp32-storage mode returns is a binary32
+    value (the fp64 mode's are not), and for the first steps its iterates stay within fp32
+    rounding distance of the fp64 recurrence's (the same method, only the storage differs)."""
+    w = W.workload(5, "tiny")
+    kw = dict(precond="spai", G=w.G, eps=w.eps)
+    for k in (1, 2, 3, 5):
+        x64 = ora.pcg(w.A, w.B, fixed_iters=k, **kw).x
+        x32 = ora.pcg(w.A, w.B, fixed_iters=k, store_f32=True, **kw).x
+        assert np.array_equal(x32, x32.astype(np.float32).astype(np.float64))
+        assert not np.array_equal(x64, x64.astype(np.float32).astype(np.float64))
+        d = np.linalg.norm(x32 - x64) / np.linalg.norm(x64)
+        assert 0.0 < d <= 1e-5 * k, (k, d)
+    # converged: the same solution to the fp32 tolerance
+    a = ora.pcg(w.A, w.B, tol=w.tol, **kw)
+    b = ora.pcg(w.A, w.B, tol=w.tol, store_f32=True, **kw)
+    assert a.status == b.status == 0
+    assert np.linalg.norm(a.x - b.x) / np.linalg.norm(a.x) <= 1e-5
+
+
+# ------------------------------------------------------------------ eigenvalue gradient
+def check_eigen_grad_closed_form(ora):
+    """2D Poisson eigenpair in closed form: g_k = v_i v_j for the unit eigenvector, and by
+    homogeneity of the eigenvalue in A, sum_k A_k g_k = v^T A v = mu."""
+    N = 17
+    A = W.poisson2d(N)
+    for j, k in ((1, 1), (4, 9), (17, 3)):
+        vj, lj = lap_eig_1d(N, j)
+        vk, lk = lap_eig_1d(N, k)
+        v = np.outer(vj, vk).ravel()
+        v /= np.linalg.norm(v)
+        g = ora.eigen_grad(A, v)
+        rows = A.rows_of_entries()
+        assert np.allclose(g, v[rows] * v[A.col.astype(np.int64)], rtol=0, atol=1e-16)
+        mu = lj + lk
+        assert abs(float(A.val.astype(np.float64) @ g) - mu) <= 1e-12 * mu, "sum A_k g_k = mu"
+
+
+def check_eigen_grad_fd(ora):
+    """Central differences of a simple eigenvalue of a random SPD matrix in single stored
+    entries (each perturbation breaks the symmetry; the eigenvalue of the perturbed matrix
+    comes from a dense non-symmetric eigensolver)."""
+    rng = np.random.default_rng(29)
+    A = random_spd(14, 707)
+    Ad = dense(A)
+    mus, vecs = np.linalg.eigh(Ad)
+    m = 6
+    assert min(mus[m] - mus[m - 1], mus[m + 1] - mus[m]) > 1e-3
+    v = vecs[:, m]
+    g = ora.eigen_grad(A, v)
+    rows = A.rows_of_entries()
+    for kk in rng.choice(A.nnz, size=14, replace=False):
+        i, j = int(rows[kk]), int(A.col[kk])
+        h = 1e-6
+        Ap = Ad.copy(); Ap[i, j] += h
+        Am = Ad.copy(); Am[i, j] -= h
+        ep = np.linalg.eigvals(Ap); em = np.linalg.eigvals(Am)
+        fp = float(np.real(ep[np.argmin(np.abs(ep - mus[m]))]))
+        fm = float(np.real(em[np.argmin(np.abs(em - mus[m]))]))
+        fd = (fp - fm) / (2 * h)
+        assert abs(g[kk] - fd) <= 1e-7, f"d mu / dA[{i},{j}]: {g[kk]} vs {fd}"
+
+
+# ------------------------------------------------------------------ nonlinear adjoint
+def _newton_cubic(Ad, b, iters=60):
+    """Solve A u + u^3 = b by dense Newton to machine precision."""
+    u = np.linalg.solve(Ad, b)
+    for _ in range(iters):
+        F = Ad @ u + u ** 3 - b
+        du = np.linalg.solve(Ad + np.diag(3 * u ** 2), F)
+        u = u - du
+        if np.max(np.abs(du)) <= 1e-16 * max(1.0, np.max(np.abs(u))):
+            break
+    return u
+
+
+def check_nonlinear_adjoint_fd(ora):
+    """F(u) = A u + u^3 - b = 0, L = w.u: the adjoint through J = A + diag(3 u^2) gives
+    dL/db = lambda and dL/dA_ij = -lambda_i u_j; central differences of L (dense Newton
+    solves) in single stored entries and in b."""
+    rng = np.random.default_rng(31)
+    A = random_spd(12, 808)
+    Ad = dense(A)
+    b = rng.uniform(-1, 1, 12)
+    w = rng.uniform(-1, 1, 12)
+    u = _newton_cubic(Ad, b)
+    J = ora.add_diagonal(A, 3 * u ** 2)
+    assert np.allclose(dense(J), Ad + np.diag(3 * u ** 2), rtol=0, atol=1e-15)
+    res = ora.nonlinear_adjoint(J, A, u, w, precond="jacobi", tol=1e-14)
+    assert res.status == 0
+    L = lambda Ax, bx: float(w @ _newton_cubic(Ax, bx))
+    rows = A.rows_of_entries()
+    for kk in rng.choice(A.nnz, size=10, replace=False):
+        i, j = int(rows[kk]), int(A.col[kk])
+        h = 1e-6
+        Ap = Ad.copy(); Ap[i, j] += h
+        Am = Ad.copy(); Am[i, j] -= h
+        fd = (L(Ap, b) - L(Am, b)) / (2 * h)
+        assert abs(res.grad[kk] - fd) <= 1e-7 * max(1.0, abs(fd)), f"dL/dA[{i},{j}]"
+    for i in rng.choice(12, size=5, replace=False):
+        h = 1e-6
+        bp = b.copy(); bp[i] += h
+        bm = b.copy(); bm[i] -= h
+        fd = (L(Ad, bp) - L(Ad, bm)) / (2 * h)
+        assert abs(res.lam[i] - fd) <= 1e-7 * max(1.0, abs(fd)), f"dL/db[{i}]"
+
+
 ALL_CHECKS = [
     check_spmv_closed_form, check_spmv_dense, check_transpose, check_spai_apply,
     check_pcg_krylov_optimal, check_pcg_eigvec_one_step, check_pcg_m_distinct,
     check_pcg_dense_solve, check_pcg_scaling, check_pcg_status, check_adjoint_identities,
     check_grad_fd, check_grad_fd_symmetric, check_list_blocks,
     check_bsr_spmv_dense, check_bsr_closed_form, check_bsr_grad_fd,
+    check_store_f32_worked_2x2, check_store_f32_exact_case, check_store_f32_rounds_and_tracks,
+    check_eigen_grad_closed_form, check_eigen_grad_fd, check_nonlinear_adjoint_fd,
 ]

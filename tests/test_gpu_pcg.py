@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import sla_workloads as W
-from gpu_helpers import SOL_TOL, dev, host, iters_close, matrix, precond, rel, tol_key
+from gpu_helpers import SOL_TOL, dev, host, iters_close, matrix, precond, rel, relmax, tol_key
 
 pytestmark = pytest.mark.gpu
 
@@ -23,21 +23,18 @@ def _ora_kw(w):
 
 # (config, size, fp64 vectors with an fp32 matrix)
 SINGLE = [(1, "tiny", False), (1, "small", False), (2, "tiny", False), (2, "small", False),
-          (2, "small", True), (5, "tiny", True), (5, "small", True)]
+          (2, "small", True), (5, "tiny", False), (5, "small", False), (5, "tiny", True),
+          (5, "small", True)]
 
 
 def _vecs(w, vf64):
     return np.float64 if vf64 else w.dtype
 
 
-def _iters_ok(gpu, ora_it, w, vf64):
-    """Within 2 % of the oracle.  With fp32 vectors on the power-law SPAI system the Krylov
-    vectors' fp32 storage itself delays convergence by 2-3 % (an fp32-storage emulation of
-    the same recurrence gives the same counts), so that mode is held to 5 %; the fp64-vector
-    mode meets 2 %."""
-    if w.dtype == np.float32 and not vf64 and w.precond == "spai" and w.A.nnz > 20 * w.A.n_rows:
-        return abs(gpu - ora_it) <= max(1, 0.05 * ora_it)
-    return iters_close(gpu, ora_it)
+def _store_f32(w, vf64):
+    """fp32 vectors: the oracle's count reference is its fp32-storage mode, so the stopping
+    decision is taken in the precision the solver stores its vectors in."""
+    return w.dtype == np.float32 and not vf64
 
 
 @pytest.mark.parametrize("engine", ["auto", "graph"])
@@ -52,11 +49,14 @@ def test_forward_parity(ora, cfg, size, vf64, engine):
     if engine == "graph":
         assert info.engine == "graph"
     ref = ora.pcg(w.A, w.B, **_ora_kw(w))
-    assert info.status == 0 and ref.status == 0
-    assert _iters_ok(info.iters, ref.iters, w, vf64), (info.iters, ref.iters)
+    cnt = ora.pcg(w.A, w.B, store_f32=True, **_ora_kw(w)) if _store_f32(w, vf64) else ref
+    assert info.status == 0 and ref.status == 0 and cnt.status == 0
+    assert iters_close(info.iters, cnt.iters), (info.iters, cnt.iters, ref.iters)
     assert info.relres <= w.tol
     tol_sol = SOL_TOL[np.float64 if (vf64 or w.dtype == np.float64) else np.float32]
-    assert rel(host(x), ref.x) <= max(tol_sol, 10 * w.tol if vf64 else 0)
+    tol_sol = max(tol_sol, 10 * w.tol if vf64 else 0)
+    assert rel(host(x), ref.x) <= tol_sol
+    assert relmax(host(x), ref.x) <= 10 * tol_sol
     # the true residual of the GPU solution, computed by the oracle's SpMV
     true = np.linalg.norm(w.B.astype(np.float64) - ora.spmv(w.A, host(x))) / np.linalg.norm(w.B)
     assert true <= (10 * w.tol if w.dtype == np.float64 else 1e-3)
@@ -74,11 +74,18 @@ def test_adjoint_parity(ora, cfg, size, vf64, engine):
                                        engine=engine)
     xo = ora.pcg(w.A, w.B, **_ora_kw(w)).x
     ref = ora.adjoint(w.A, xo, w.W, **_ora_kw(w))
+    if _store_f32(w, vf64):
+        x32 = ora.pcg(w.A, w.B, store_f32=True, **_ora_kw(w)).x
+        cnt = ora.adjoint(w.A, x32, w.W, store_f32=True, **_ora_kw(w))
+    else:
+        cnt = ref
     assert info.status == 0
-    assert _iters_ok(info.iters, ref.iters, w, vf64), (info.iters, ref.iters)
+    assert iters_close(info.iters, cnt.iters), (info.iters, cnt.iters, ref.iters)
     t = SOL_TOL[tol_key(w.dtype)]
     assert rel(host(lam), ref.lam) <= t
     assert rel(host(g), ref.grad) <= t
+    assert relmax(host(lam), ref.lam) <= 10 * t
+    assert relmax(host(g), ref.grad) <= 10 * t
     # the gradient is -lam_i x_j of the GPU's own lam and x, rounded once to A's type
     g2 = ora.grad(w.A, host(lam), host(x))
     assert rel(host(g), g2) <= (1e-15 if w.dtype == np.float64 else 1e-7)

@@ -22,6 +22,8 @@ MUTANTS = {
     "spai_drops_eps": ("z[i] = z[i] + M->eps * r[i];", "z[i] = z[i];"),
     "spai_transposed_order": (
         "ora_spmv(n, M->gt_rp, M->gt_ci, M->gt_v, r, work);   /* y = G^T r */\n"
+        "        if (store_f32)\n"
+        "            ora_round_f32(n, work);\n"
         "        ora_spmv(n, M->g_rp, M->g_ci, M->g_v, work, z);      /* z = G y   */",
         "ora_spmv(n, M->g_rp, M->g_ci, M->g_v, r, work);\n"
         "        ora_spmv(n, M->gt_rp, M->gt_ci, M->gt_v, work, z);"),
@@ -39,6 +41,12 @@ MUTANTS = {
                         "s += val[k * b * b + (int64_t)r * b + c] * x[(int64_t)ci[k] * b + r];"),
     "bsr_expansion_position": ("const int64_t p = k * b * b + (int64_t)r * b + c;",
                                "const int64_t p = k * b * b + (int64_t)c * b + r;"),
+    "store_f32_keeps_q": ("        if (store_f32)\n            ora_round_f32(n, q);\n", ""),
+    "store_f32_keeps_x": ("            ora_round_f32(n, x);\n", ""),
+    "eigen_grad_sign": ("g[k] = v[i] * v[ci[k]];", "g[k] = -v[i] * v[ci[k]];"),
+    "eigen_grad_row_only": ("g[k] = v[i] * v[ci[k]];", "g[k] = v[i] * v[i];"),
+    "add_diagonal_first_entry": ("            if (ci[k] == i) {\n                out[k] = v[k] + c[i];",
+                                 "            if (k == rp[i]) {\n                out[k] = v[k] + c[i];"),
     "bsr_expansion_column": ("out_ci[e] = (int32_t)((int64_t)ci[k] * b + c);",
                              "out_ci[e] = (int32_t)((int64_t)ci[k] + c);"),
 }
