@@ -29,6 +29,7 @@ __all__ = [
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
     "sla_pcg_solve_batched_noalloc", "sla_eigen_grad", "sla_csr_add_diagonal", "sla_nonlinear_adjoint",
+    "sla_vec_dot", "sla_pcg_update", "sla_pcg_direction", "sla_vec_gather", "sla_vec_scatter_add",
     "sla_workspace_bytes", "sla_pcg_kernel_times", "sla_pcg_phase_times", "solve",
     "ENGINES",
 ]
@@ -384,6 +385,52 @@ def sla_nonlinear_adjoint(J: Matrix, M: Optional[Preconditioner], A: Optional[Ma
                                        _ptr(lam), _ptr(dLdA), C.byref(opts), C.byref(info), _stream(stream)),
            "sla_nonlinear_adjoint")
     return lam, dLdA, _infos([info])[0]
+
+
+def sla_vec_dot(x: torch.Tensor, y: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[0] = x . y in fp64 (device tensor; no host synchronisation)."""
+    out = torch.empty(1, dtype=torch.float64, device=x.device) if out is None else out
+    _check(lib().sla_vec_dot(_dtype_code(x.dtype), x.numel(), _ptr(x), _ptr(y), _ptr(out), _stream(stream)),
+           "sla_vec_dot")
+    return out
+
+
+def sla_pcg_update(alpha: float, p: torch.Tensor, q: torch.Tensor, x: torch.Tensor, r: torch.Tensor,
+                   dinv: Optional[torch.Tensor], z: torch.Tensor, out2: Optional[torch.Tensor] = None,
+                   n: Optional[int] = None, stream=None) -> torch.Tensor:
+    """x += alpha p, r -= alpha q, z = dinv * r; returns the device tensor [r.r, r.z] (fp64).
+    n: number of leading elements to update (default: all of r)."""
+    out2 = torch.empty(2, dtype=torch.float64, device=r.device) if out2 is None else out2
+    n = r.numel() if n is None else int(n)
+    _check(lib().sla_pcg_update(_dtype_code(r.dtype), n, float(alpha), _ptr(p), _ptr(q), _ptr(x), _ptr(r),
+                                _ptr(dinv), _ptr(z), _ptr(out2), _stream(stream)), "sla_pcg_update")
+    return out2
+
+
+def sla_pcg_direction(beta: float, z: torch.Tensor, p: torch.Tensor, n: Optional[int] = None, stream=None):
+    """p = z + beta p on the leading n elements (default: all)."""
+    n = p.numel() if n is None else int(n)
+    _check(lib().sla_pcg_direction(_dtype_code(p.dtype), n, float(beta), _ptr(z), _ptr(p), _stream(stream)),
+           "sla_pcg_direction")
+    return p
+
+
+def sla_vec_gather(idx: torch.Tensor, src: torch.Tensor, dst: torch.Tensor, stream=None) -> torch.Tensor:
+    """dst[k] = src[idx[k]] (idx int32)."""
+    if idx.dtype != torch.int32:
+        raise ValueError("idx must be int32")
+    _check(lib().sla_vec_gather(_dtype_code(src.dtype), idx.numel(), _ptr(idx), _ptr(src), _ptr(dst),
+                                _stream(stream)), "sla_vec_gather")
+    return dst
+
+
+def sla_vec_scatter_add(idx: torch.Tensor, src: torch.Tensor, dst: torch.Tensor, stream=None) -> torch.Tensor:
+    """dst[idx[k]] += src[k] (idx int32, distinct)."""
+    if idx.dtype != torch.int32:
+        raise ValueError("idx must be int32")
+    _check(lib().sla_vec_scatter_add(_dtype_code(dst.dtype), idx.numel(), _ptr(idx), _ptr(src), _ptr(dst),
+                                     _stream(stream)), "sla_vec_scatter_add")
+    return dst
 
 
 def sla_pcg_kernel_times(A: Matrix, M: Optional[Preconditioner] = None, nrhs: int = 1, reps: int = 20,

@@ -69,6 +69,11 @@ SIGNATURES = {
     "sla_csr_add_diagonal": (_st, [_vp, _vp, _vp, _vp]),
     "sla_nonlinear_adjoint": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, C.POINTER(sla_pcg_opts),
                                     C.POINTER(sla_pcg_info), _vp]),
+    "sla_vec_dot": (_st, [C.c_int32, C.c_int64, _vp, _vp, _vp, _vp]),
+    "sla_pcg_update": (_st, [C.c_int32, C.c_int64, C.c_double, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "sla_pcg_direction": (_st, [C.c_int32, C.c_int64, C.c_double, _vp, _vp, _vp]),
+    "sla_vec_gather": (_st, [C.c_int32, C.c_int64, _vp, _vp, _vp, _vp]),
+    "sla_vec_scatter_add": (_st, [C.c_int32, C.c_int64, _vp, _vp, _vp, _vp]),
     "sla_pcg_solve_batched_noalloc": (_st, [_vp, _vp, _vp, _vp, C.POINTER(sla_pcg_opts),
                                             C.POINTER(sla_pcg_info), _vp]),
     "sla_pcg_kernel_times": (_st, [_vp, _vp, C.c_int32, C.c_int32, C.c_int32, C.POINTER(C.c_double), _vp]),

@@ -269,6 +269,42 @@ SLA_API sla_status sla_nonlinear_adjoint(const sla_csr *J, const sla_precond *M,
                                          void *d_dLdA, const sla_pcg_opts *opts, sla_pcg_info *info,
                                          void *stream);
 
+/* ---------------------------------------------------------------- iteration steps
+ * The vector steps of one PCG iteration as separate calls, for solvers that drive the
+ * iteration from the host between collectives: the row-block distributed PCG of [TS]
+ * Methodology §3 (each rank owns a contiguous block of rows, exchanges halo values before
+ * each product and all-reduces the scalars).  dtype is the vectors' type (SLA_F32 or
+ * SLA_F64); all vectors are device arrays of n elements; reductions are fp64, summed in a
+ * fixed order (deterministic) and written to DEVICE memory, so they can feed a collective
+ * without a host round trip.  fp32 updates round the scalar to fp32 once and use one fused
+ * multiply-add, as the single-GPU solve engines do.  None synchronises `stream`. */
+
+/* d_out[0] = sum_i x_i y_i (fp64). */
+SLA_API sla_status sla_vec_dot(int32_t dtype, int64_t n, const void *d_x, const void *d_y, double *d_out,
+                               void *stream);
+
+/* The update after q = A p ([TS] Methodology §1 CG step): x += alpha p, r -= alpha q,
+ * z = D^-1 r (d_dinv: n values of 1/A_ii in the vector type; NULL: z = r), and
+ * d_out2[0] = r.r, d_out2[1] = r.z of the updated r (fp64). */
+SLA_API sla_status sla_pcg_update(int32_t dtype, int64_t n, double alpha, const void *d_p, const void *d_q,
+                                  void *d_x, void *d_r, const void *d_dinv, void *d_z, double *d_out2,
+                                  void *stream);
+
+/* p = z + beta p. */
+SLA_API sla_status sla_pcg_direction(int32_t dtype, int64_t n, double beta, const void *d_z, void *d_p,
+                                     void *stream);
+
+/* d_dst[k] = d_src[d_idx[k]] for k < n (packing the values a neighbour needs; indices must
+ * lie inside d_src). */
+SLA_API sla_status sla_vec_gather(int32_t dtype, int64_t n, const int32_t *d_idx, const void *d_src,
+                                  void *d_dst, void *stream);
+
+/* d_dst[d_idx[k]] += d_src[k] for k < n (summing received halo contributions into their
+ * owner's entries); the indices of one call must be distinct (no atomics: the result is
+ * deterministic), and lie inside d_dst. */
+SLA_API sla_status sla_vec_scatter_add(int32_t dtype, int64_t n, const int32_t *d_idx, const void *d_src,
+                                       void *d_dst, void *stream);
+
 /* The list solve of sla_pcg_solve_batched (list handle, nrhs = 1, Jacobi or no
  * preconditioner) for callers that cannot allocate device memory while they solve --
  * code under a memory pool or budget that owns the device's memory, hosts that forbid
