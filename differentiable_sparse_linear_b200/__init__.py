@@ -21,11 +21,11 @@ import torch
 from . import _lib
 from ._lib import (SLA_BREAKDOWN, SLA_ERR_CUDA, SLA_ERR_INVALID_ARG, SLA_ERR_INVALID_CSR,
                    SLA_ERR_OOM, SLA_ERR_UNSUPPORTED, SLA_F32, SLA_F64, SLA_NOT_CONVERGED,
-                   SLA_SPD, SLA_SUCCESS, SLA_VALIDATE)
+                   SLA_SPD, SLA_STATIC_VALUES, SLA_SUCCESS, SLA_VALIDATE)
 
 __all__ = [
     "SlaError", "Matrix", "Preconditioner", "PcgInfo", "lib",
-    "sla_version", "sla_csr_create", "sla_bsr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
+    "sla_version", "sla_csr_create", "sla_csr_values_changed", "sla_bsr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
     "sla_pcg_solve_batched_noalloc", "sla_eigen_grad", "sla_csr_add_diagonal", "sla_nonlinear_adjoint",
@@ -189,16 +189,24 @@ def _check_vec(A: Matrix, v: torch.Tensor, vector_f64: bool):
 
 
 def sla_csr_create(row_ptr: torch.Tensor, col: torch.Tensor, val: torch.Tensor, *,
-                   validate: bool = True, spd: bool = True, stream=None) -> Matrix:
-    """sla_csr_create: one square CSR matrix (n = row_ptr.numel() - 1)."""
+                   validate: bool = True, spd: bool = True, static_values: bool = False,
+                   stream=None) -> Matrix:
+    """sla_csr_create: one square CSR matrix (n = row_ptr.numel() - 1).  static_values: the
+    caller changes the values only with sla_csr_values_changed (SLA_STATIC_VALUES)."""
     n = row_ptr.numel() - 1
     if row_ptr.dtype != torch.int32 or col.dtype != torch.int32:
         raise ValueError("row_ptr and col must be int32")
     h = C.c_void_p()
-    flags = (SLA_VALIDATE if validate else 0) | (SLA_SPD if spd else 0)
+    flags = ((SLA_VALIDATE if validate else 0) | (SLA_SPD if spd else 0)
+             | (SLA_STATIC_VALUES if static_values else 0))
     _check(lib().sla_csr_create(C.byref(h), n, n, col.numel(), _ptr(row_ptr), _ptr(col), _ptr(val),
                                 _dtype_code(val.dtype), flags, _stream(stream)), "sla_csr_create")
     return Matrix(h.value, row_ptr, col, val)
+
+
+def sla_csr_values_changed(A: Matrix, stream=None) -> None:
+    """The values of a SLA_STATIC_VALUES handle were changed in place."""
+    _check(lib().sla_csr_values_changed(A.handle, _stream(stream)), "sla_csr_values_changed")
 
 
 def sla_bsr_create(row_ptr: torch.Tensor, col: torch.Tensor, val: torch.Tensor, *,

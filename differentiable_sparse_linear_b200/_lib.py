@@ -19,6 +19,7 @@ SLA_F32 = 0
 SLA_F64 = 1
 SLA_SPD = 1
 SLA_VALIDATE = 2
+SLA_STATIC_VALUES = 4
 SLA_ENGINE_AUTO = 0
 SLA_ENGINE_GRAPH = 1
 SLA_ENGINE_PERSISTENT = 2
@@ -50,6 +51,7 @@ SIGNATURES = {
     "sla_bsr_create": (_st, [C.POINTER(_vp), C.c_int64, C.c_int32, C.c_int64, _vp, _vp, _vp,
                              C.c_int, C.c_uint32, _vp]),
     "sla_csr_destroy": (_st, [_vp]),
+    "sla_csr_values_changed": (_st, [_vp, _vp]),
     "sla_csr_shape": (_st, [_vp, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int32)]),
     "sla_spmv": (_st, [_vp, _vp, _vp, _vp]),
     "sla_spmv_multi": (_st, [_vp, C.c_int32, _vp, _vp, _vp]),

@@ -575,6 +575,12 @@ static void free_csr(sla_csr *A)
         delete A->sell;
         A->sell = nullptr;
     }
+    if (A->groups) {
+        cudaFree(A->groups->d_rows);
+        delete A->groups;
+        A->groups = nullptr;
+    }
+    free_csb(A);
     if (A->d_err)
         cudaFree(A->d_err);
     if (A->d_sys_off)

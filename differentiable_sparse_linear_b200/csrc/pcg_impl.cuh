@@ -15,6 +15,7 @@
 #include "row_engine.cuh"
 #include "tile_engine.cuh"
 #include "bsr.cuh"
+#include "csb.cuh"
 
 namespace sla {
 
@@ -331,10 +332,13 @@ struct TileLaunch {
     // sides; above that, block-owned tiles (a lane's gathers would not fit its registers)
     static constexpr bool LANE_GROUPS = K <= 4;
     int grid = 0;
-    int maxl = 0;                 // 0: tile engine; -1: lane groups; -2: BSR lane groups; else the short-row MAXL
+    int maxl = 0;                 // 0: tile engine; -1: lane groups; -2: BSR lane groups;
+                                  // -3: column-sorted segments; else the short-row MAXL
     MatView<VM> m{};
     const WinDesc *win = nullptr; // operand windows (short-row engine, K <= 2)
     GroupView gv{};               // length-grouped rows (lane-group engine)
+    CsbView<VM> cv{};             // column-sorted segments
+    size_t csb_smem = 0;
     int bdim = 1;                 // BSR block size (maxl == -2)
 
     template <int MAXL>
@@ -404,6 +408,31 @@ struct TileLaunch {
             return setup_rows<16>(A, s);
         }
         int per_sm = 0;
+        // one right-hand side, one gathered vector: the column-sorted segments, for the
+        // solver's operations (solves gather the values first) and for the caller-facing
+        // product when the handle's values are declared static (otherwise that product reads
+        // the CSR values, which may change between calls)
+        if constexpr (K == 1 && Op::NG == 1) {
+            if (A->batch == 1 && (!any_ld<Op>::value || (A->flags & SLA_STATIC_VALUES))) {
+                const CsbPart *cp;
+                SLA_TRY(ensure_csb(const_cast<sla_csr *>(A), s, &cp));
+                cv.seg_row0 = cp->d_seg_row0;
+                cv.seg_ch0 = cp->d_seg_ch0;
+                cv.cbase = cp->d_cbase;
+                cv.pk = cp->d_pk;
+                cv.val = (const VM *)cp->d_val;
+                cv.n_seg = cp->n_seg;
+                csb_smem = (size_t)std::max(cp->rmax, 1) * sizeof(double);
+                auto kern = k_csb<VM, Op>;
+                SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csb_smem));
+                SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, CsbCfg::T, csb_smem));
+                per_sm = std::max(per_sm, 1);
+                grid = std::max(1, std::min(cp->n_seg, per_sm * A->num_sms));
+                m = view<VM>(A, nullptr);
+                maxl = -3;
+                return SLA_SUCCESS;
+            }
+        }
         if constexpr (LANE_GROUPS) {
             const GroupPart *gp;
             SLA_TRY(ensure_groups(const_cast<sla_csr *>(A), s, &gp));
@@ -434,6 +463,12 @@ struct TileLaunch {
     }
     void launch(cudaStream_t s, const Op &op, double *part, PcgState *st, int *err) const
     {
+        if (maxl == -3) {
+            if constexpr (K == 1 && Op::NG == 1)
+                if (cv.n_seg > 0)
+                    k_csb<VM, Op><<<grid, CsbCfg::T, csb_smem, s>>>(cv, op, part, st);
+            return;
+        }
         if (maxl < 0 ? gv.n_tasks == 0 : m.n_tiles == 0)
             return;
         // windows are bulk-copied from the gathered vectors: they need 16-byte alignment
@@ -497,6 +532,8 @@ static sla_status spmv_k(const sla_csr *A, int nc, const void *x, void *y, cudaS
     Op op{(const V *)x, (V *)y, nc, nc};
     TileLaunch<K, V, Op> L;
     SLA_TRY(L.setup(A, s));
+    if (L.maxl == -3 && !A->csb_vals_current)     // static values: the copy, refreshed on demand
+        SLA_TRY(launch_csb_values(A, s));
     L.launch(s, op, nullptr, nullptr, A->d_err);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
@@ -842,6 +879,13 @@ static sla_status run_k(sla_csr *A, Plan *p, int nrhs, const void *B, void *X, d
         if constexpr (persist_compiled<VV, K, 16>())
             SLA_TRY((persist_launch<VM, VV, K, 16>(A, p, s)));
     } else {
+        // column-sorted copies of long-row matrices: values gathered from the CSR arrays
+        // before every solve (they may have changed since the last one)
+        SLA_TRY(launch_csb_values(A, s));
+        if (p->kind == 2) {
+            SLA_TRY(launch_csb_values(p->M->G, s));
+            SLA_TRY(launch_csb_values(p->M->GT, s));
+        }
         SLA_CUDA_TRY(cudaGraphLaunch(p->exec, s));
     }
     k_copy_out<VV, K><<<gv, 256, 0, s>>>(n, nrhs, (const VV *)p->x, (VV *)X);

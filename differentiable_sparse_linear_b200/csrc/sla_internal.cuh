@@ -133,6 +133,23 @@ struct SellPart {
     void *d_val = nullptr;               // the matrix's type
 };
 
+// Column-sorted row segments of a long-row matrix (csb.cuh): segment s holds rows
+// [seg_row0[s], seg_row0[s+1]) (at most CSB_RMAX) and chunks [seg_ch0[s], seg_ch0[s+1]) of
+// 32 entry slots, its entries in ascending (column, row) order; per chunk the smallest
+// column, per slot (column - base) << 16 | local row (0xFFFF: padding), the CSR position of
+// the entry (-1: padding) and its value (gathered from the CSR values before each solve).
+struct CsbPart {
+    int n_seg = 0;
+    int rmax = 0;                        // rows of the largest segment
+    int64_t n_chunks = 0;
+    int32_t *d_seg_row0 = nullptr;
+    int32_t *d_seg_ch0 = nullptr;
+    int32_t *d_cbase = nullptr;
+    uint32_t *d_pk = nullptr;
+    int32_t *d_perm = nullptr;
+    void *d_val = nullptr;               // the matrix's type
+};
+
 // Read-only view of a CSR matrix passed to kernels.
 template <typename V>
 struct MatView {
@@ -175,6 +192,8 @@ struct sla_csr {
     std::map<int, sla::TilePart> tiles;    // by item budget D
     sla::SellPart *sell = nullptr;         // sliced ELL copy (persistent solver)
     sla::GroupPart *groups = nullptr;      // rows grouped by length (long-row matrices)
+    sla::CsbPart *csb = nullptr;           // column-sorted row segments (long-row matrices)
+    int csb_vals_current = 0;              // csb's value copy matches the CSR values
     int device = 0;
     int num_sms = 148;
     std::vector<sla::Plan *> plans;
@@ -233,6 +252,11 @@ sla_status ensure_sell(sla_csr *A, cudaStream_t s, const SellPart **out);
 // Build (once) the length-grouped row list of a matrix.
 sla_status ensure_groups(sla_csr *A, cudaStream_t s, const GroupPart **out);
 sla_status launch_sell_values(const sla_csr *A, const SellPart *sp, cudaStream_t s);
+// Build (once) the column-sorted segments of a long-row CSR matrix; gather their values
+// from the CSR values (every solve); free them.
+sla_status ensure_csb(sla_csr *A, cudaStream_t s, const CsbPart **out);
+sla_status launch_csb_values(const sla_csr *A, cudaStream_t s);
+void free_csb(sla_csr *A);
 size_t plan_bytes(const sla_csr *A, const sla_precond *M, int K, int vec64);
 sla_status get_plan(sla_csr *A, const sla_precond *M, int K, int vec64, Plan **out);
 void destroy_plan(Plan *p);

@@ -73,6 +73,10 @@ typedef enum { SLA_F32 = 0, SLA_F64 = 1 } sla_dtype;
 #define SLA_VALIDATE 2u   /* check the pattern on the device: row_ptr[0] = 0, row_ptr non-  */
                           /* decreasing, row_ptr[n] = nnz, columns in range, strictly        */
                           /* ascending in each row (so duplicates are rejected, not summed)  */
+#define SLA_STATIC_VALUES 4u /* the caller does not change the values after creation, or    */
+                          /* calls sla_csr_values_changed after it does: single-vector       */
+                          /* products (sla_spmv) may then read a copy of the values kept in  */
+                          /* the library's own layout (solves re-read the values anyway)     */
 
 typedef struct sla_csr sla_csr;
 typedef struct sla_precond sla_precond;
@@ -168,6 +172,11 @@ SLA_API sla_status sla_bsr_create(sla_csr **out, int64_t n_block_rows, int32_t b
                           sla_dtype dtype, uint32_t flags, void *stream);
 
 SLA_API sla_status sla_csr_destroy(sla_csr *A);
+
+/* For a handle created with SLA_STATIC_VALUES: the caller changed the values in place, so
+ * copies of them held in the library's layouts must be refreshed before the next product
+ * (done lazily, on `stream`, by that product).  Harmless on other handles. */
+SLA_API sla_status sla_csr_values_changed(sla_csr *A, void *stream);
 
 /* n_rows, nnz and batch (1 for a single matrix) of a handle; any output may be NULL. */
 SLA_API sla_status sla_csr_shape(const sla_csr *A, int64_t *n_rows, int64_t *nnz, int32_t *batch);

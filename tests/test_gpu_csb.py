@@ -1,0 +1,104 @@
+"""The column-sorted segment engine (the long-row SpMV of single-right-hand-side solves) on
+patterns made to reach its edge cases: columns 70000 apart inside one segment (chunks cut
+early: the in-chunk column offset is 16 bits), a hub row of 3000 entries, empty-neighbour
+rows, many segments with a ragged last one, fp32 and fp64.  Lockstep iterates after k
+steps, then a converged solve and adjoint, against the oracle."""
+import numpy as np
+import pytest
+
+import sla_workloads as W
+from gpu_helpers import SOL_TOL, dev, host, iters_close, matrix, rel, relmax
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ora():
+    import oracle
+    return oracle.get()
+
+
+def _wide_spd(n, dtype):
+    rng = np.random.default_rng(91)
+    jump = 70001 if n > 140002 else n // 2         # columns further apart than 16 bits reach
+    i = np.arange(n - 1, dtype=np.int64)
+    lo = [i, i[: n - jump]]                        # chain and a wide jump
+    hi = [i + 1, i[: n - jump] + jump]
+    hub = 12345
+    others = rng.choice(np.setdiff1d(np.arange(n), [hub]), size=3000, replace=False).astype(np.int64)
+    lo.append(np.minimum(others, hub))
+    hi.append(np.maximum(others, hub))
+    a = rng.integers(0, n, 20000)
+    b = rng.integers(0, n, 20000)
+    keep = a != b
+    lo.append(np.minimum(a, b)[keep])
+    hi.append(np.maximum(a, b)[keep])
+    key = np.unique(np.concatenate(lo) * n + np.concatenate(hi))
+    A = W._assemble_symmetric(key // n, key % n, n, 17, 0.5, dtype)
+    assert np.diff(A.row_ptr).max() > 3000
+    return A
+
+
+@pytest.mark.parametrize("dtype", [np.float32, np.float64])
+def test_csb_lockstep_and_solve(ora, dtype):
+    import differentiable_sparse_linear_b200 as sla
+    n = 150001
+    A = _wide_spd(n, dtype)
+    Ad = matrix(A)
+    M = sla.sla_precond_jacobi(Ad)
+    b = W.rhs_normal(92, n, dtype)
+    w = W.rhs_uniform(93, n, dtype=dtype)
+    tight = 1e-11 if dtype == np.float64 else 1e-5
+    for k in (1, 4, 9):
+        x, info = sla.sla_pcg_solve(Ad, M, dev(b), rtol=1e-300, maxit=k, engine="graph")
+        assert info.iters == k and info.status == sla.SLA_NOT_CONVERGED
+        ref = ora.pcg(A, b, precond="jacobi", fixed_iters=k)
+        assert rel(host(x), ref.x) <= tight, (k, rel(host(x), ref.x))
+        assert relmax(host(x), ref.x) <= 10 * tight
+    tol = 1e-10 if dtype == np.float64 else 1e-6
+    x, info = sla.sla_pcg_solve(Ad, M, dev(b), rtol=tol)
+    ref = ora.pcg(A, b, precond="jacobi", tol=tol)
+    cnt = ora.pcg(A, b, precond="jacobi", tol=tol, store_f32=True) if dtype == np.float32 else ref
+    assert info.status == 0 and iters_close(info.iters, cnt.iters), (info.iters, cnt.iters, ref.iters)
+    assert rel(host(x), ref.x) <= SOL_TOL[dtype]
+    lam, g, ainfo = sla.sla_pcg_adjoint(Ad, M, x, dev(w), rtol=tol)
+    adj = ora.adjoint(A, ref.x, w, precond="jacobi", tol=tol)
+    assert ainfo.status == 0
+    assert rel(host(lam), adj.lam) <= SOL_TOL[dtype] and rel(host(g), adj.grad) <= SOL_TOL[dtype]
+
+
+def test_csb_values_follow_in_place_changes(ora):
+    """The sorted copy's values are gathered from the CSR values at every solve."""
+    import differentiable_sparse_linear_b200 as sla
+    A = _wide_spd(150001, np.float64)
+    val = dev(A.val)
+    Ad = sla.sla_csr_create(dev(A.row_ptr), dev(A.col), val)
+    M = sla.sla_precond_jacobi(Ad)
+    b = W.rhs_normal(94, A.n_rows, np.float64)
+    x1, _ = sla.sla_pcg_solve(Ad, M, dev(b), rtol=1e-10)
+    val.mul_(2.0)                                    # A -> 2A in place: x -> x / 2
+    M.refresh()
+    x2, _ = sla.sla_pcg_solve(Ad, M, dev(b), rtol=1e-10)
+    assert rel(host(x2), host(x1) / 2.0) <= 1e-8
+
+
+@pytest.mark.parametrize("cfg,size", [(5, "small"), (5, "tiny")])
+def test_static_values_spmv(ora, cfg, size):
+    """sla_spmv of a SLA_STATIC_VALUES handle reads the column-sorted value copy; after the
+    values change in place, sla_csr_values_changed makes the next product use the new ones."""
+    import differentiable_sparse_linear_b200 as sla
+    from gpu_helpers import SPMV_TOL
+    w = W.workload(cfg, size)
+    A = w.A
+    val = dev(A.val)
+    As = sla.sla_csr_create(dev(A.row_ptr), dev(A.col), val, static_values=True)
+    Ad = sla.sla_csr_create(dev(A.row_ptr), dev(A.col), val)
+    x = W.rhs_normal(95, A.n_rows, w.dtype)
+    ref = ora.spmv(A, x)
+    ys = host(sla.sla_spmv(As, dev(x)))
+    yd = host(sla.sla_spmv(Ad, dev(x)))
+    assert rel(ys, ref) <= SPMV_TOL[w.dtype] and rel(yd, ref) <= SPMV_TOL[w.dtype]
+    val.mul_(-0.5)
+    sla.sla_csr_values_changed(As)
+    ys2 = host(sla.sla_spmv(As, dev(x)))
+    assert rel(ys2, -0.5 * ref) <= SPMV_TOL[w.dtype]

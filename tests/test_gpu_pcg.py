@@ -117,14 +117,16 @@ def test_multi_rhs_parity(ora, size):
     M, _ = precond(w, Ad)
     X, infos = sla.sla_pcg_solve_batched(Ad, M, dev(w.B), rtol=w.tol)
     Xo, outs = ora.pcg_multi(w.A, w.B, **_ora_kw(w))
+    X32, c32 = ora.pcg_multi(w.A, w.B, store_f32=True, **_ora_kw(w))   # fp32 vectors: counts in fp32 storage
     for c in range(w.nrhs):
         assert infos[c].status == 0
-        assert iters_close(infos[c].iters, outs[c].iters), (c, infos[c].iters, outs[c].iters)
+        assert iters_close(infos[c].iters, c32[c].iters), (c, infos[c].iters, c32[c].iters, outs[c].iters)
         assert rel(host(X)[:, c], Xo[:, c]) <= SOL_TOL[np.float32]
     Lam, G, ainf = sla.sla_pcg_adjoint_batched(Ad, M, X, dev(w.W), rtol=w.tol)
     Lo, go, aouts = ora.adjoint_multi(w.A, Xo, w.W, **_ora_kw(w))
+    _, _, a32 = ora.adjoint_multi(w.A, X32, w.W, store_f32=True, **_ora_kw(w))
     for c in range(w.nrhs):
-        assert iters_close(ainf[c].iters, aouts[c].iters)
+        assert iters_close(ainf[c].iters, a32[c].iters), (c, ainf[c].iters, a32[c].iters, aouts[c].iters)
     assert rel(host(Lam), Lo) <= SOL_TOL[np.float32]
     assert rel(host(G), go) <= SOL_TOL[np.float32]
 
