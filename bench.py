@@ -400,7 +400,7 @@ def run_ours(args):
         x, inf = sla.sla_pcg_solve(Ad, M, bv, x_out, rtol=w.tol, engine=args.engine)
         if record:
             fwd_events[-1][1].record()
-        fwd_iters.append(inf.iters)
+            fwd_iters.append(inf.iters)
         lam, g, ainf = sla.sla_pcg_adjoint(Ad, M, x, wv, rtol=w.tol, engine=args.engine, dLdb=lam_buf, dLdA=g_buf)
         engines_seen.update((inf.engine, ainf.engine))
         if inf.status != 0 or ainf.status != 0:
