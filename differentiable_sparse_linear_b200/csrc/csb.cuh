@@ -35,6 +35,9 @@ constexpr int CSB_RMAX = 16384;                // rows per segment (fp64 sums in
 #ifndef SLA_CSB_TMA
 #define SLA_CSB_TMA 0
 #endif
+#ifndef SLA_CSB_PAIR
+#define SLA_CSB_PAIR 0
+#endif
 constexpr bool CSB_TMA = SLA_CSB_TMA != 0;     // matrix stream by bulk copies (k_csb_tma)
 constexpr uint32_t CSB_PAD = 0xFFFFu;
 
@@ -46,6 +49,53 @@ struct CsbView {
     const uint32_t *pk;                        // per entry slot
     const VM *val;                             // per entry slot
     int n_seg;
+    int rmax;                                  // rows of the largest segment
+};
+
+// A segment's row sums in shared memory (8 bytes per row).  fp32 values with fp32 vectors:
+// a pair of fp32 sums per row -- hi takes each product rounded to fp32 with an atomic add
+// that returns the old value, and lo takes that addition's exact rounding error (recovered
+// from the old value and the addend by the two-sum identity) plus the product's own fp32
+// rounding error -- so the row sum hi + lo carries about 48 bits, where a plain fp32 sum in
+// arbitrary order would move the solver's iteration counts.  Otherwise fp64 atomic adds.
+constexpr bool CSB_PAIR = SLA_CSB_PAIR != 0;
+template <typename VM, typename VV>
+struct CsbSums {
+    static constexpr bool PAIR = CSB_PAIR && sizeof(VM) == 4 && sizeof(VV) == 4;
+    double *d;
+    float *hi, *lo;
+    __device__ __forceinline__ CsbSums(void *base, int rmax)
+        : d((double *)base), hi((float *)base), lo((float *)base + rmax) {}
+    __device__ __forceinline__ void zero(int i)
+    {
+        if constexpr (PAIR) {
+            hi[i] = 0.f;
+            lo[i] = 0.f;
+        } else {
+            d[i] = 0.0;
+        }
+    }
+    __device__ __forceinline__ void add(int r, double p)
+    {
+        if constexpr (PAIR) {
+            const float ph = __double2float_rn(p);
+            const float pl = __double2float_rn(p - (double)ph);
+            const float old = atomicAdd(&hi[r], ph);
+            const float sm = __fadd_rn(old, ph);
+            const float bb = __fsub_rn(sm, old);
+            const float err = __fadd_rn(__fsub_rn(old, __fsub_rn(sm, bb)), __fsub_rn(ph, bb));
+            atomicAdd(&lo[r], __fadd_rn(err, pl));
+        } else {
+            atomicAdd(&d[r], p);
+        }
+    }
+    __device__ __forceinline__ double get(int i) const
+    {
+        if constexpr (PAIR)
+            return (double)hi[i] + (double)lo[i];
+        else
+            return d[i];
+    }
 };
 
 struct CsbCfg {
@@ -106,6 +156,7 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
         op.stage(s_scal);
     __syncthreads();
     GlobalRows<Op, 1> rv{op};
+    CsbSums<VM, VV> sums(s_y, c.rmax);
     double part[NR];
 #pragma unroll
     for (int i = 0; i < NR; ++i)
@@ -119,7 +170,7 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
         CsbRound<VM, U> cur;
         cur.load(c, ch, ch1, lane);
         for (int i = tid; i < R; i += T)
-            s_y[i] = 0.0;
+            sums.zero(i);
         __syncthreads();
         for (; ch < ch1; ch += U * NW) {
             CsbRound<VM, U> nxt;
@@ -132,12 +183,12 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
 #pragma unroll
             for (int u = 0; u < U; ++u)
                 if ((cur.w[u] & 0xFFFFu) != CSB_PAD)
-                    atomicAdd(&s_y[cur.w[u] & 0xFFFFu], (double)cur.a[u] * (double)g[u]);
+                    sums.add((int)(cur.w[u] & 0xFFFFu), (double)cur.a[u] * (double)g[u]);
             cur = nxt;
         }
         __syncthreads();
         for (int i = tid; i < R; i += T) {
-            const double acc[1] = {s_y[i]};
+            const double acc[1] = {sums.get(i)};
             op.emit((int64_t)(r0 + i), acc, part, s_scal, rv);
         }
         __syncthreads();
@@ -157,7 +208,7 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
 // wait is bounded in time (a wait that runs out sets *err and the abort flag; the kernel
 // then runs to its end without further copies, its results flagged invalid by the host).
 struct CsbTmaCfg {
-    static constexpr int NCW = 32;             // consumer warps
+    static constexpr int NCW = 31;             // consumer warps (+1 producer: 1024 threads)
     static constexpr int TC = NCW * 32;        // consumer threads
     static constexpr int T = TC + 32;          // + the producer warp
     static constexpr int SC = NCW;             // chunks per stage
@@ -186,7 +237,7 @@ k_csb_tma(const CsbView<VM> c, const Op op, double *partials, PcgState *st, int 
     static_assert(Op::NG == 1, "the column-sorted engine gathers one vector");
 
     extern __shared__ __align__(128) unsigned char smem[];
-    double *s_y = (double *)(smem + L::RING);
+    CsbSums<VM, VV> sums(smem + L::RING, c.rmax);
     __shared__ __align__(8) uint64_t full_bar[NST];
     __shared__ __align__(8) uint64_t empty_bar[NST];
     __shared__ int s_abort;
@@ -256,7 +307,7 @@ k_csb_tma(const CsbView<VM> c, const Op op, double *partials, PcgState *st, int 
         const int c0 = c.seg_ch0[s], c1 = c.seg_ch0[s + 1];
         const int ngroups = (c1 - c0 + Cfg::SC - 1) / Cfg::SC;
         for (int i = tid; i < R; i += Cfg::TC)
-            s_y[i] = 0.0;
+            sums.zero(i);
         csync();
         for (int gb = 0; gb < ngroups; gb += U) {
             int base[U];
@@ -292,11 +343,11 @@ k_csb_tma(const CsbView<VM> c, const Op op, double *partials, PcgState *st, int 
 #pragma unroll
             for (int u = 0; u < U; ++u)
                 if ((w[u] & 0xFFFFu) != CSB_PAD)
-                    atomicAdd(&s_y[w[u] & 0xFFFFu], (double)a[u] * (double)g[u]);
+                    sums.add((int)(w[u] & 0xFFFFu), (double)a[u] * (double)g[u]);
         }
         csync();
         for (int i = tid; i < R; i += Cfg::TC) {
-            const double acc[1] = {s_y[i]};
+            const double acc[1] = {sums.get(i)};
             op.emit((int64_t)(r0 + i), acc, part, s_scal, rv);
         }
         csync();

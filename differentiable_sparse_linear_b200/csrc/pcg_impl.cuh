@@ -422,6 +422,7 @@ struct TileLaunch {
                 cv.pk = cp->d_pk;
                 cv.val = (const VM *)cp->d_val;
                 cv.n_seg = cp->n_seg;
+                cv.rmax = std::max(cp->rmax, 1);
                 csb_smem = (size_t)std::max(cp->rmax, 1) * sizeof(double) + (CSB_TMA ? CsbTmaLayout<VM>::RING : 0);
                 const void *kern = CSB_TMA ? (const void *)k_csb_tma<VM, Op> : (const void *)k_csb<VM, Op>;
                 SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csb_smem));
