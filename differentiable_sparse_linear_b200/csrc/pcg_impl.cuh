@@ -423,11 +423,10 @@ struct TileLaunch {
                 cv.val = (const VM *)cp->d_val;
                 cv.n_seg = cp->n_seg;
                 cv.rmax = std::max(cp->rmax, 1);
-                csb_smem = (size_t)std::max(cp->rmax, 1) * sizeof(double) + (CSB_TMA ? CsbTmaLayout<VM>::RING : 0);
-                const void *kern = CSB_TMA ? (const void *)k_csb_tma<VM, Op> : (const void *)k_csb<VM, Op>;
+                csb_smem = (size_t)std::max(cp->rmax, 1) * sizeof(double);
+                auto kern = k_csb<VM, Op>;
                 SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csb_smem));
-                SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &per_sm, kern, CSB_TMA ? CsbTmaCfg::T : CsbCfg::T, csb_smem));
+                SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, CsbCfg::T, csb_smem));
                 per_sm = std::max(per_sm, 1);
                 grid = std::max(1, std::min(cp->n_seg, per_sm * A->num_sms));
                 m = view<VM>(A, nullptr);
@@ -467,12 +466,8 @@ struct TileLaunch {
     {
         if (maxl == -3) {
             if constexpr (K == 1 && Op::NG == 1)
-                if (cv.n_seg > 0) {
-                    if (CSB_TMA)
-                        k_csb_tma<VM, Op><<<grid, CsbTmaCfg::T, csb_smem, s>>>(cv, op, part, st, err);
-                    else
-                        k_csb<VM, Op><<<grid, CsbCfg::T, csb_smem, s>>>(cv, op, part, st);
-                }
+                if (cv.n_seg > 0)
+                    k_csb<VM, Op><<<grid, CsbCfg::T, csb_smem, s>>>(cv, op, part, st);
             return;
         }
         if (maxl < 0 ? gv.n_tasks == 0 : m.n_tiles == 0)
