@@ -345,6 +345,7 @@ sla_status ensure_sell(sla_csr *A, cudaStream_t s, const SellPart **out)
         A->sell = nullptr;
     }
     SellPart *sp = new SellPart();
+    A->sell_vals_current = 0;
     sp->n_slices = nsl;
     sp->n_slots = slots;
     sp->rel16 = rel16 ? 1 : 0;

@@ -229,5 +229,6 @@ extern "C" sla_status sla_csr_values_changed(sla_csr *A, void *stream)
     if (!A)
         return fail(SLA_ERR_INVALID_ARG, "NULL handle");
     A->csb_vals_current = 0;
+    A->sell_vals_current = 0;
     return SLA_SUCCESS;
 }

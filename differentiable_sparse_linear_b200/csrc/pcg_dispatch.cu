@@ -206,6 +206,7 @@ sla_status launch_sell_values(const sla_csr *A, const SellPart *sp, cudaStream_t
         k_pack_values<double><<<grid, 256, 0, s>>>(sp->n_slots, sp->d_perm, (const double *)A->val,
                                                    (double *)sp->d_val);
     SLA_CUDA_TRY(cudaGetLastError());
+    const_cast<sla_csr *>(A)->sell_vals_current = 1;
     return SLA_SUCCESS;
 }
 

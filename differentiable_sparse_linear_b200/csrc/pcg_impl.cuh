@@ -520,11 +520,48 @@ static sla_status spmv_slices_k(const sla_csr *A, int nc, const void *x, void *y
     return SLA_SUCCESS;
 }
 
+// Short rows, values declared static: the product over the sliced copy (values refreshed
+// when stale), whole-row operand accesses where the layout and alignment allow them.
+template <typename V, int K, int MAXL>
+static sla_status spmv_sell_k(const sla_csr *A, int nc, const void *x, void *y, cudaStream_t s)
+{
+    const SellPart *sp;
+    SLA_TRY(ensure_sell(const_cast<sla_csr *>(A), s, &sp));
+    if (!A->sell_vals_current)
+        SLA_TRY(launch_sell_values(A, sp, s));
+    SellView<V> v;
+    v.desc = sp->d_desc;
+    v.offs = sp->d_offs;
+    v.lens = sp->d_lens;
+    v.idx16 = sp->rel16 ? (const int16_t *)sp->d_idx : nullptr;
+    v.idx32 = sp->rel16 ? nullptr : (const int32_t *)sp->d_idx;
+    v.val = (const V *)sp->d_val;
+    v.n = A->n;
+    v.n_slices = sp->n_slices;
+    OpSpmv<V, K> op{(const V *)x, (V *)y, nc, nc};
+    const uintptr_t wbytes = (uintptr_t)RowIO<V, K>::W;
+    op.rows = nc == K && ((uintptr_t)x % wbytes) == 0 && ((uintptr_t)y % wbytes) == 0;
+    auto kern = k_spmv_sell<V, K, MAXL>;
+    int per_sm = 0;
+    SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, SPS_T, 0));
+    const int64_t want = (sp->n_slices + 2 * (SPS_T / 32) - 1) / (2 * (SPS_T / 32));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)std::max(per_sm, 1) * A->num_sms));
+    kern<<<grid, SPS_T, 0, s>>>(v, op);
+    SLA_CUDA_TRY(cudaGetLastError());
+    return SLA_SUCCESS;
+}
+
 template <typename V, int K>
 static sla_status spmv_k(const sla_csr *A, int nc, const void *x, void *y, cudaStream_t s)
 {
-    // short rows: CSR-direct product over the slice descriptors
-    if (A->n > 0 && A->batch == 1 && A->bdim == 1 && A->max_row_len <= 16 && K <= 4) {
+    // short rows: the sliced copy when the values are static, else the CSR-direct product
+    // over the slice descriptors
+    if (A->n > 0 && A->batch == 1 && A->bdim == 1 && A->max_row_len <= 16 && K <= 8) {
+        if (A->flags & SLA_STATIC_VALUES) {
+            if (A->max_row_len <= 8)
+                return spmv_sell_k<V, K, 8>(A, nc, x, y, s);
+            return spmv_sell_k<V, K, 16>(A, nc, x, y, s);
+        }
         if (A->max_row_len <= 8)
             return spmv_slices_k<V, K, 8>(A, nc, x, y, s);
         return spmv_slices_k<V, K, 16>(A, nc, x, y, s);

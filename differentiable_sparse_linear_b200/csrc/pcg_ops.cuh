@@ -193,6 +193,9 @@ struct OpSpmv {
     const V *x;
     V *y;
     int ld, nc;
+    // whole-row vector accesses: set by the host only when ld == nc == K and x, y are
+    // aligned to the row width the access uses (RowIO)
+    bool rows = false;
     __device__ const V *row_vec(int) const { return nullptr; }
     __host__ __device__ const V *gvec(int) const { return x; }
     __host__ __device__ int gstride() const { return ld; }
@@ -207,9 +210,14 @@ struct OpSpmv {
     {
         return c < nc ? __ldg(&x[j * ld + c]) : (V)0;
     }
-    // caller vectors: any leading dimension, so element by element
+    // caller vectors: any leading dimension, so element by element (whole rows when the
+    // host found the layout and alignment allow it)
     __device__ __forceinline__ void operand_row(int64_t j, V (&o)[K], const double *s) const
     {
+        if (rows) {
+            RowIO<V, K>::load(x + j * K, o);
+            return;
+        }
 #pragma unroll
         for (int c = 0; c < K; ++c)
             o[c] = operand(j, c, s);
@@ -224,6 +232,14 @@ struct OpSpmv {
     __device__ __forceinline__ void emit(int64_t i, const double (&acc)[K], double (&)[N], const double *,
                                          const RV &) const
     {
+        if (rows) {
+            V v[K];
+#pragma unroll
+            for (int c = 0; c < K; ++c)
+                v[c] = (V)acc[c];
+            RowIO<V, K>::store(y + i * K, v);
+            return;
+        }
 #pragma unroll
         for (int c = 0; c < K; ++c)
             if (c < nc)

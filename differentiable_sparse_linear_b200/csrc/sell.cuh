@@ -205,4 +205,17 @@ k_spmv_slices(int64_t n, int64_t n_slices, const uint2 *__restrict__ desc, const
     }
 }
 
+// y = A x from the sliced copy of a short-row matrix whose values are declared static
+// (SLA_STATIC_VALUES; the copy is refreshed when the caller reports a change): every slot row
+// of a slice is one coalesced 128-byte access of values, diagonal slices read no column
+// indices, and [n][K] operands move as whole rows.  The persistent solver's phase code, with
+// the plain product as its row epilogue.
+template <typename V, int K, int MAXL>
+__global__ void __launch_bounds__(SPS_T)
+k_spmv_sell(const SellView<V> m, const OpSpmv<V, K> op)
+{
+    double part[1] = {0.0};
+    sell_phase<K, V, MAXL, SPS_T, (K <= 2 ? 2 : 1)>(m, op, part, nullptr);
+}
+
 }  // namespace sla

@@ -194,6 +194,7 @@ struct sla_csr {
     sla::GroupPart *groups = nullptr;      // rows grouped by length (long-row matrices)
     sla::CsbPart *csb = nullptr;           // column-sorted row segments (long-row matrices)
     int csb_vals_current = 0;              // csb's value copy matches the CSR values
+    int sell_vals_current = 0;             // sell's value copy matches the CSR values
     int device = 0;
     int num_sms = 148;
     std::vector<sla::Plan *> plans;

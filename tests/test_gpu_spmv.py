@@ -117,3 +117,24 @@ def test_invalid_patterns_rejected():
         with pytest.raises(sla.SlaError) as e:
             sla.sla_csr_create(*mk(rp, ci))
         assert e.value.status == sla.SLA_ERR_INVALID_CSR
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("cfg,size", [(1, "small"), (2, "small"), (3, "small"), (2, "tiny"), (5, "small")])
+def test_spmv_static_values(ora, cfg, size, k):
+    """Handles with SLA_STATIC_VALUES: short rows read the sliced copy (whole-row operand
+    accesses when the block is [n][k] with k a power of two), long rows the column-sorted
+    copy (one column); a change of the values is picked up after sla_csr_values_changed."""
+    import differentiable_sparse_linear_b200 as sla
+    w = W.workload(cfg, size)
+    A = w.A
+    val = dev(A.val)
+    As = sla.sla_csr_create(dev(A.row_ptr), dev(A.col), val, static_values=True)
+    X = _x(A.n_rows, k, w.dtype, 30 + k)
+    Y = sla.sla_spmv(As, dev(X)) if k == 1 else sla.sla_spmv_multi(As, dev(X))
+    ref = _ref(ora, A, X)
+    assert rel(host(Y), ref) <= SPMV_TOL[tol_key(w.dtype)]
+    val.mul_(3.0)
+    sla.sla_csr_values_changed(As)
+    Y = sla.sla_spmv(As, dev(X)) if k == 1 else sla.sla_spmv_multi(As, dev(X))
+    assert rel(host(Y), 3.0 * ref) <= SPMV_TOL[tol_key(w.dtype)]
