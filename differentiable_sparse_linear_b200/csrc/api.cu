@@ -949,6 +949,8 @@ sla_status sla_precond_spai(sla_precond **out, const sla_csr *A, const sla_csr *
         return fail(SLA_ERR_INVALID_ARG, "G must be a CSR matrix (A may be BSR)");
     if (!(eps >= 0.0))
         return fail(SLA_ERR_INVALID_ARG, "eps must be >= 0");
+    if (A->d_sys_off)       // a list: the list kernel reads G's columns as local indices
+        SLA_TRY(check_list_blocks(A, G, (cudaStream_t)stream));
     sla_precond *M = new sla_precond();
     M->kind = 2;
     M->A = A;

@@ -3,8 +3,13 @@
 // Solvers and Sparse Tensor Parallelism for PyTorch", Methodology §1), forward and adjoint.
 //
 // One block owns one system for its whole solve: the system's vectors (x, r, p, q, z,
-// D^-1, and for the adjoint the forward x) live in shared memory, so the only HBM traffic
-// is the system's matrix (re-read from L2 after the first iteration), b, and the results.
+// D^-1, for the adjoint the forward x, and with SPAI y = G^T r) live in shared memory, so the
+// only HBM traffic is the system's matrix (re-read from L2 after the first iteration), b,
+// and the results.  Systems too large for shared memory keep the same vectors in a device
+// workspace (nv values per row of the batch), with the same code and order of operations.
+// Preconditioners: Jacobi, none, or SPAI z = G (G^T r) + eps r ([SPAI] "Learning Sparse
+// Approximate Inverse Preconditioners for Conjugate Gradient Solvers on GPUs", Approach)
+// with G block-diagonal on the list's systems (checked when the preconditioner is made).
 // Dot products are block reductions in fp64 with a fixed order; each system has its own
 // stopping test, iteration count and status.  There is no grid-wide dependency, so the
 // whole batch is one launch and needs no graph.
@@ -48,8 +53,9 @@ __device__ __forceinline__ void list_sum2(double &a, double &b, double *s_red)
 }
 
 // q = A p on one system (rows [0, ns), local columns = global - o0), S lanes per row;
-// returns this thread's share of p.q (only the first lane of each row group contributes).
-template <typename V, int S>
+// returns this thread's share of p.q (only the first lane of each row group contributes;
+// 0 without DOT).
+template <typename V, int S, bool DOT = true>
 __device__ __forceinline__ double list_spmv(int ns, int64_t o0, const int32_t *rp, const int32_t *ci,
                                             const V *val, const V *p, V *q)
 {
@@ -68,17 +74,50 @@ __device__ __forceinline__ double list_spmv(int ns, int64_t o0, const int32_t *r
         if (lane == 0) {
             const V qv = (V)acc;
             q[i] = qv;
-            part += (double)p[i] * (double)qv;
+            if (DOT)
+                part += (double)p[i] * (double)qv;
         }
     }
     return part;
 }
 
+// The SPAI factor of a list (block-diagonal G and its explicit transpose) for the kernel.
+template <typename V>
+struct ListSpai {
+    const int32_t *g_rp, *g_ci;
+    const V *g_val;
+    const int32_t *gt_rp, *gt_ci;
+    const V *gt_val;
+    double eps;
+};
+
+// z = G (G^T r) + eps r on one system; returns this thread's share of r.z.  Ends with the
+// block synchronised.
+template <typename V, int S>
+__device__ __forceinline__ double list_spai_apply(int ns, int64_t o0, const ListSpai<V> &m, const V *r, V *y,
+                                                  V *z)
+{
+    list_spmv<V, S, false>(ns, o0, m.gt_rp, m.gt_ci, m.gt_val, r, y);
+    __syncthreads();
+    list_spmv<V, S, false>(ns, o0, m.g_rp, m.g_ci, m.g_val, y, z);
+    __syncthreads();
+    double rz = 0.0;
+    for (int i = threadIdx.x; i < ns; i += LIST_T) {
+        const V zi = (V)__fma_rn(m.eps, (double)r[i], (double)z[i]);
+        z[i] = zi;
+        rz += (double)r[i] * (double)zi;
+    }
+    return rz;
+}
+
+// Vectors of one system per row of the batch: x, r, p, q, z, D^-1, forward x, y (SPAI).
+constexpr int LIST_NV = 8;
+
 template <typename V, int S>
 __global__ void __launch_bounds__(LIST_T)
 k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sys_off, int batch,
            const V *B, V *X, const V *dinv, const V *Xf, V *Gout, double tol, long long maxit_opt,
-           sla_pcg_info *info)
+           sla_pcg_info *info, const ListSpai<V> spai, int use_spai, V *ws)
 {
     extern __shared__ __align__(16) unsigned char s_raw[];
     __shared__ double s_red[2 * (LIST_T / 32) + 2];
@@ -86,13 +125,14 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
     for (int s = blockIdx.x; s < batch; s += gridDim.x) {
         const int64_t o0 = sys_off[s];
         const int ns = (int)(sys_off[s + 1] - o0);
-        V *x = (V *)s_raw;
+        V *x = ws ? ws + (int64_t)LIST_NV * o0 : (V *)s_raw;
         V *r = x + ns;
         V *p = r + ns;
         V *q = p + ns;
         V *z = q + ns;
         V *dv = z + ns;
         V *xf = dv + ns;
+        V *y = xf + ns;
         const long long maxit = maxit_opt > 0 ? maxit_opt : 10LL * (ns > 0 ? ns : 1);
 
         double bb = 0.0, rz = 0.0;
@@ -103,12 +143,20 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
             x[i] = (V)0;
             r[i] = bi;
             dv[i] = di;
-            z[i] = zi;
-            p[i] = zi;
+            if (!use_spai) {
+                z[i] = zi;
+                p[i] = zi;
+                rz += (double)bi * (double)zi;
+            }
             if (Xf)
                 xf[i] = Xf[o0 + i];
             bb += (double)bi * (double)bi;
-            rz += (double)bi * (double)zi;
+        }
+        if (use_spai) {
+            __syncthreads();
+            rz = list_spai_apply<V, S>(ns, o0, spai, r, y, z);
+            for (int i = tid; i < ns; i += LIST_T)
+                p[i] = z[i];
         }
         list_sum2(bb, rz, s_red);
         const double bnorm = sqrt(bb);
@@ -137,12 +185,26 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
                     x[i] = (V)__fma_rn(alpha, (double)p[i], (double)x[i]);
                     const V rn = (V)__fma_rn(-alpha, (double)q[i], (double)r[i]);
                     r[i] = rn;
-                    const V zn = (V)((double)rn * (double)dv[i]);
-                    z[i] = zn;
                     rr += (double)rn * (double)rn;
-                    rzn += (double)rn * (double)zn;
+                    if (!use_spai) {
+                        const V zn = (V)((double)rn * (double)dv[i]);
+                        z[i] = zn;
+                        rzn += (double)rn * (double)zn;
+                    }
                 }
-                list_sum2(rr, rzn, s_red);
+                if (use_spai) {
+                    // stopping test first (on r.r), then z = M^-1 r: the apply is skipped on
+                    // the last iteration, as in the single-system solvers
+                    double dummy = 0.0;
+                    list_sum2(rr, dummy, s_red);
+                    relres = sqrt(rr) / bnorm;
+                    if (isfinite(relres) && relres > tol) {
+                        rzn = list_spai_apply<V, S>(ns, o0, spai, r, y, z);
+                        list_sum2(rzn, dummy, s_red);
+                    }
+                } else {
+                    list_sum2(rr, rzn, s_red);
+                }
                 relres = sqrt(rr) / bnorm;
                 if (!isfinite(relres)) {
                     status = SLA_BREAKDOWN;
@@ -185,12 +247,20 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
     }
 }
 
-template <typename V, int S>
-static sla_status list_launch(const sla_csr *A, const V *dinv, const void *B, void *X, const void *Xf,
-                              void *G, double tol, long long maxit, sla_pcg_info *d_info,
-                              cudaStream_t s)
+// Shared memory a system's vectors take; above LIST_SMEM_MAX they live in a workspace.
+constexpr size_t LIST_SMEM_MAX = 200 * 1024;
+
+static size_t list_smem(const sla_csr *A, int nv)
 {
-    const size_t shm = (size_t)7 * (size_t)A->max_sys_n * sizeof(V);
+    return (size_t)nv * (size_t)A->max_sys_n * (A->dtype == SLA_F32 ? 4 : 8);
+}
+
+template <typename V, int S>
+static sla_status list_launch(const sla_csr *A, const V *dinv, const ListSpai<V> &spai, int use_spai, V *ws,
+                              const void *B, void *X, const void *Xf, void *G, double tol, long long maxit,
+                              sla_pcg_info *d_info, cudaStream_t s)
+{
+    const size_t shm = ws ? 0 : (size_t)LIST_NV * (size_t)A->max_sys_n * sizeof(V);
     auto kern = k_list_pcg<V, S>;
     SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm));
     int per_sm = 0;
@@ -200,23 +270,40 @@ static sla_status list_launch(const sla_csr *A, const V *dinv, const void *B, vo
     const int grid = std::min<int64_t>(A->batch, (int64_t)per_sm * A->num_sms);
     kern<<<grid, LIST_T, shm, s>>>(A->rp, A->ci, (const V *)A->val, A->d_sys_off, A->batch,
                                    (const V *)B, (V *)X, dinv, (const V *)Xf, (V *)G, tol, maxit,
-                                   d_info);
+                                   d_info, spai, use_spai, ws);
     SLA_CUDA_TRY(cudaGetLastError());
     return SLA_SUCCESS;
 }
 
 template <typename V>
-static sla_status list_v(const sla_csr *A, const V *dinv, const void *B, void *X, const void *Xf,
+static sla_status list_v(const sla_csr *A, const sla_precond *M, V *ws, const void *B, void *X, const void *Xf,
                          void *G, double tol, long long maxit, sla_pcg_info *d_info, cudaStream_t s)
 {
+    const V *dinv = nullptr;
+    ListSpai<V> sp{};
+    int use_spai = 0;
+    if (M && M->kind == 1) {
+        dinv = (const V *)(sizeof(V) == 4 ? M->d_dinv : M->d_dinv64);
+    } else if (M && M->kind == 2) {
+        sp = ListSpai<V>{M->G->rp, M->G->ci, (const V *)M->G->val, M->GT->rp, M->GT->ci, (const V *)M->GT->val,
+                         M->eps};
+        use_spai = 1;
+    }
     const double mean = A->n > 0 ? (double)A->nnz / (double)A->n : 0.0;
     if (mean <= 6.0)
-        return list_launch<V, 4>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
+        return list_launch<V, 4>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
     if (mean <= 24.0)
-        return list_launch<V, 8>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
+        return list_launch<V, 8>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
     if (mean <= 64.0)
-        return list_launch<V, 16>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
-    return list_launch<V, 32>(A, dinv, B, X, Xf, G, tol, maxit, d_info, s);
+        return list_launch<V, 16>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
+    return list_launch<V, 32>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
+}
+
+static sla_status list_check_precond(const sla_precond *M)
+{
+    if (M && M->kind == 2 && (!M->G || !M->GT))
+        return fail(SLA_ERR_INVALID_ARG, "the SPAI preconditioner's G was destroyed");
+    return SLA_SUCCESS;
 }
 
 // Forward (Xf == nullptr) or adjoint (Xf = forward solution, B = dL/dx, X = dL/db,
@@ -225,19 +312,25 @@ sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B,
                           const void *Xf, void *G, const sla_pcg_opts *opts, sla_pcg_info *info,
                           cudaStream_t s)
 {
-    if (M && M->kind != 1)
-        return fail(SLA_ERR_UNSUPPORTED, "list solves support the Jacobi preconditioner or none");
-    if ((size_t)7 * A->max_sys_n * (A->dtype == SLA_F32 ? 4 : 8) > 200 * 1024)
-        return fail(SLA_ERR_UNSUPPORTED, "list solve: largest system exceeds the shared-memory size");
+    SLA_TRY(list_check_precond(M));
     const double tol = (opts && opts->rtol > 0) ? opts->rtol : (A->dtype == SLA_F32 ? 1e-6 : 1e-10);
     const long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 0;
     sla_pcg_info *d_info = nullptr;
     SLA_CUDA_TRY(cudaMallocAsync((void **)&d_info, sizeof(sla_pcg_info) * (size_t)A->batch, s));
+    // systems whose vectors do not fit in shared memory: a workspace of LIST_NV values per row
+    void *ws = nullptr;
+    cudaError_t we = cudaSuccess;
+    if (list_smem(A, LIST_NV) > LIST_SMEM_MAX && A->n > 0)
+        we = cudaMallocAsync(&ws, (size_t)LIST_NV * (size_t)A->n * (A->dtype == SLA_F32 ? 4 : 8), s);
     sla_status st;
-    if (A->dtype == SLA_F32)
-        st = list_v<float>(A, M ? (const float *)M->d_dinv : nullptr, B, X, Xf, G, tol, maxit, d_info, s);
+    if (we != cudaSuccess)
+        st = fail(SLA_ERR_OOM, "list solve: workspace allocation");
+    else if (A->dtype == SLA_F32)
+        st = list_v<float>(A, M, (float *)ws, B, X, Xf, G, tol, maxit, d_info, s);
     else
-        st = list_v<double>(A, M ? (const double *)M->d_dinv64 : nullptr, B, X, Xf, G, tol, maxit, d_info, s);
+        st = list_v<double>(A, M, (double *)ws, B, X, Xf, G, tol, maxit, d_info, s);
+    if (ws)
+        cudaFreeAsync(ws, s);
     if (st == SLA_SUCCESS) {
         cudaError_t e = cudaMemcpyAsync(info, d_info, sizeof(sla_pcg_info) * (size_t)A->batch,
                                         cudaMemcpyDeviceToHost, s);
@@ -255,6 +348,55 @@ sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B,
     return worst;
 }
 
+// *err = 1 if a row of M stores a column outside its system's range (block-diagonal check
+// of a list's SPAI factor against the list's system offsets).
+__global__ void k_check_blocks(int64_t n, const int32_t *rp, const int32_t *ci, const int64_t *sys_off,
+                               int batch, int *err)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        int lo = 0, hi = batch - 1;                 // the system holding row i
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sys_off[mid] <= i)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int64_t a = sys_off[lo], b = sys_off[lo + 1];
+        for (int64_t k = rp[i]; k < rp[i + 1]; ++k)
+            if (ci[k] < a || ci[k] >= b)
+                atomicOr(err, 1);
+    }
+}
+
+sla_status check_list_blocks(const sla_csr *A, const sla_csr *M, cudaStream_t s)
+{
+    if (M->n != A->n)
+        return fail(SLA_ERR_INVALID_ARG, "the factor must have the list's size");
+    if (A->n == 0)
+        return SLA_SUCCESS;
+    int *d_err = nullptr;
+    SLA_CUDA_TRY(cudaMallocAsync((void **)&d_err, sizeof(int), s));
+    cudaError_t e = cudaMemsetAsync(d_err, 0, sizeof(int), s);
+    const int grid = (int)std::min<int64_t>((A->n + 255) / 256, (int64_t)A->num_sms * 8);
+    if (e == cudaSuccess) {
+        k_check_blocks<<<grid, 256, 0, s>>>(M->n, M->rp, M->ci, A->d_sys_off, A->batch, d_err);
+        e = cudaGetLastError();
+    }
+    int h = 0;
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&h, d_err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    cudaFreeAsync(d_err, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "block-diagonal check of the SPAI factor");
+    if (h)
+        return fail(SLA_ERR_INVALID_ARG, "for a list handle, G must be block-diagonal on the list's systems");
+    return SLA_SUCCESS;
+}
+
 }  // namespace sla
 
 namespace sla {
@@ -264,17 +406,15 @@ namespace sla {
 sla_status launch_list_kernel(const sla_csr *A, const sla_precond *M, const void *B, void *X,
                               const sla_pcg_opts *opts, sla_pcg_info *d_info, cudaStream_t s)
 {
-    if (M && M->kind != 1)
-        return fail(SLA_ERR_UNSUPPORTED, "list solves support the Jacobi preconditioner or none");
-    if ((size_t)7 * A->max_sys_n * (A->dtype == SLA_F32 ? 4 : 8) > 200 * 1024)
-        return fail(SLA_ERR_UNSUPPORTED, "list solve: largest system exceeds the shared-memory size");
+    SLA_TRY(list_check_precond(M));
+    // this path allocates nothing: every system's vectors must fit in shared memory
+    if (list_smem(A, LIST_NV) > LIST_SMEM_MAX)
+        return fail(SLA_ERR_UNSUPPORTED, "list solve without allocation: largest system exceeds the shared-memory size");
     const double tol = (opts && opts->rtol > 0) ? opts->rtol : (A->dtype == SLA_F32 ? 1e-6 : 1e-10);
     const long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 0;
     if (A->dtype == SLA_F32)
-        return list_v<float>(A, M ? (const float *)M->d_dinv : nullptr, B, X, nullptr, nullptr, tol, maxit,
-                             d_info, s);
-    return list_v<double>(A, M ? (const double *)M->d_dinv64 : nullptr, B, X, nullptr, nullptr, tol, maxit,
-                          d_info, s);
+        return list_v<float>(A, M, (float *)nullptr, B, X, nullptr, nullptr, tol, maxit, d_info, s);
+    return list_v<double>(A, M, (double *)nullptr, B, X, nullptr, nullptr, tol, maxit, d_info, s);
 }
 
 }  // namespace sla

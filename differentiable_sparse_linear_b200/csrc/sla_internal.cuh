@@ -295,6 +295,8 @@ SLA_COMBO_DECL(fd)
 #undef SLA_COMBO_DECL
 sla_status spmv_ff(const sla_csr *A, int nrhs, const void *x, void *y, cudaStream_t s);
 sla_status spmv_dd(const sla_csr *A, int nrhs, const void *x, void *y, cudaStream_t s);
+// Fails unless every row of M keeps its columns inside its system of the list handle A.
+sla_status check_list_blocks(const sla_csr *A, const sla_csr *M, cudaStream_t s);
 sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B, void *X,
                           const void *Xfwd, void *G, const sla_pcg_opts *opts, sla_pcg_info *info,
                           cudaStream_t s);

@@ -148,7 +148,9 @@ SLA_API sla_status sla_csr_create(sla_csr **out, int64_t n_rows, int64_t n_cols,
  * h_sys_row_off[0] = 0, last = n_total) is copied.  Column indices are global and must lie in
  * the owning system's range (checked by SLA_VALIDATE).  sla_spmv works on the whole block
  * matrix; sla_pcg_solve_batched / sla_pcg_adjoint_batched solve every system on its own,
- * each with its own stopping test and info entry. */
+ * each with its own stopping test and info entry (one block per system: its vectors in
+ * shared memory, or in a workspace the call allocates when the largest system's do not fit;
+ * Jacobi, SPAI or no preconditioner). */
 SLA_API sla_status sla_csr_create_list(sla_csr **out, int32_t batch, const int64_t *h_sys_row_off,
                                int64_t nnz_total, const int32_t *d_row_ptr, const int32_t *d_col,
                                const void *d_val, sla_dtype dtype, uint32_t flags, void *stream);
@@ -198,7 +200,8 @@ SLA_API sla_status sla_precond_jacobi(sla_precond **out, const sla_csr *A, void 
 /* SPAI: M^-1 = G G^T + eps I ([SPAI] Approach).  G is a square CSR of A's size (it normally
  * carries A's lower-triangular pattern; any pattern is accepted), borrowed like A; the
  * library forms and owns G^T explicitly so each apply is two plain SpMVs.  For a list
- * handle A, G must be block-diagonal with the same blocks. */
+ * handle A, G must be block-diagonal with the same blocks (checked on the device:
+ * SLA_ERR_INVALID_ARG otherwise). */
 SLA_API sla_status sla_precond_spai(sla_precond **out, const sla_csr *A, const sla_csr *G, double eps,
                             void *stream);
 
@@ -314,8 +317,10 @@ SLA_API sla_status sla_vec_gather(int32_t dtype, int64_t n, const int32_t *d_idx
 SLA_API sla_status sla_vec_scatter_add(int32_t dtype, int64_t n, const int32_t *d_idx, const void *d_src,
                                        void *d_dst, void *stream);
 
-/* The list solve of sla_pcg_solve_batched (list handle, nrhs = 1, Jacobi or no
- * preconditioner) for callers that cannot allocate device memory while they solve --
+/* The list solve of sla_pcg_solve_batched (list handle, nrhs = 1; every system's vectors
+ * must fit in shared memory -- SLA_ERR_UNSUPPORTED otherwise, since the workspace the
+ * regular call would take is an allocation) for callers that cannot allocate device memory
+ * while they solve --
  * code under a memory pool or budget that owns the device's memory, hosts that forbid
  * allocation after start-up, or code that must avoid the synchronisation an allocation or
  * free can bring.  This call allocates nothing: the per-system results pass through a

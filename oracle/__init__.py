@@ -294,13 +294,22 @@ class Oracle:
         return r
 
     @staticmethod
-    def system(A, s: int):
-        """System s of a block-diagonal list as its own CSR (local column indices)."""
-        o0, o1 = int(A.sys_row_off[s]), int(A.sys_row_off[s + 1])
+    def system(A, s: int, sys_row_off=None):
+        """System s of a block-diagonal list as its own CSR (local column indices).  A matrix
+        without its own offsets (a list's SPAI factor) takes the list's `sys_row_off`."""
+        off = A.sys_row_off if sys_row_off is None else sys_row_off
+        o0, o1 = int(off[s]), int(off[s + 1])
         k0, k1 = int(A.row_ptr[o0]), int(A.row_ptr[o1])
         rp = (A.row_ptr[o0:o1 + 1].astype(np.int64) - k0).astype(np.int32)
         ci = (A.col[k0:k1].astype(np.int64) - o0).astype(np.int32)
         return type(A)(o1 - o0, o1 - o0, rp, ci, np.asarray(A.val[k0:k1]))
+
+    def _system_kw(self, A, s, kw):
+        """The solver options for system s: a list's SPAI factor G cut to the system's block."""
+        if kw.get("G") is not None:
+            kw = dict(kw)
+            kw["G"] = self.system(kw["G"], s, A.sys_row_off)
+        return kw
 
     def pcg_list(self, A, b, **kw):
         """Distinct-pattern batch: one PCG per diagonal block; b and x concatenated."""
@@ -308,7 +317,7 @@ class Oracle:
         out = []
         for s in range(A.batch):
             o0, o1 = int(A.sys_row_off[s]), int(A.sys_row_off[s + 1])
-            r = self.pcg(self.system(A, s), np.asarray(b)[o0:o1], **kw)
+            r = self.pcg(self.system(A, s), np.asarray(b)[o0:o1], **self._system_kw(A, s, kw))
             x[o0:o1] = r.x
             out.append(r)
         return x, out
@@ -321,7 +330,8 @@ class Oracle:
         for s in range(A.batch):
             o0, o1 = int(A.sys_row_off[s]), int(A.sys_row_off[s + 1])
             k0, k1 = int(A.row_ptr[o0]), int(A.row_ptr[o1])
-            r = self.adjoint(self.system(A, s), np.asarray(x)[o0:o1], np.asarray(w)[o0:o1], **kw)
+            r = self.adjoint(self.system(A, s), np.asarray(x)[o0:o1], np.asarray(w)[o0:o1],
+                             **self._system_kw(A, s, kw))
             lam[o0:o1] = r.lam
             g[k0:k1] = r.grad
             out.append(r)

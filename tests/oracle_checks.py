@@ -322,6 +322,16 @@ def check_list_blocks(ora):
     x, out = ora.pcg_list(A, b, precond="jacobi", tol=1e-13)
     assert all(r.status == 0 for r in out)
     assert rel(x, np.linalg.solve(Ad, b)) < 1e-10, "block-diagonal list vs dense solve"
+    # with a block-diagonal SPAI factor, cut to each system: the same solution, and every
+    # system's iterates are those of its own SPAI solve
+    A.sys_row_off = np.asarray(A.sys_row_off)
+    G = W.spai_factor_G(A, seed=23)
+    xs, outs = ora.pcg_list(A, b, precond="spai", G=G, eps=3e-3, tol=1e-13)
+    assert all(r.status == 0 for r in outs)
+    assert rel(xs, np.linalg.solve(Ad, b)) < 1e-10, "SPAI list vs dense solve"
+    o0, o1 = int(A.sys_row_off[2]), int(A.sys_row_off[3])
+    Gs = ora.system(G, 2, A.sys_row_off)
+    assert np.allclose(dense(Gs), dense(G)[o0:o1, o0:o1], rtol=0, atol=0)
 
 
 # ------------------------------------------------------------------------------ BSR
