@@ -400,6 +400,8 @@ def run_ours(args):
             x, inf = sla.sla_pcg_solve_batched(Ad, M, bv, x_out, rtol=w.tol, engine=args.engine)
             if record:
                 fwd_events[-1][1].record()
+                if not is_list:     # one iteration advances every right-hand side
+                    fwd_iters.append(max(i.iters for i in inf))
             lam, g, ainf = sla.sla_pcg_adjoint_batched(Ad, M, x, wv, rtol=w.tol, engine=args.engine,
                                                        dLdB=lam_buf, dLdA=g_buf)
             engines_seen.update(i.engine for i in inf + ainf)
