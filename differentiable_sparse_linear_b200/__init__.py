@@ -28,7 +28,7 @@ __all__ = [
     "sla_version", "sla_csr_create", "sla_csr_values_changed", "sla_bsr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
-    "sla_pcg_solve_batched_noalloc", "sla_eigen_grad", "sla_csr_add_diagonal", "sla_nonlinear_adjoint",
+    "sla_pcg_solve_batched_noalloc", "sla_list_kernel_ms", "sla_eigen_grad", "sla_csr_add_diagonal", "sla_nonlinear_adjoint",
     "sla_vec_dot", "sla_pcg_update", "sla_pcg_direction", "sla_vec_gather", "sla_vec_scatter_add",
     "sla_workspace_bytes", "sla_pcg_kernel_times", "sla_pcg_phase_times", "solve",
     "ENGINES",
@@ -311,6 +311,13 @@ def sla_pcg_solve_batched(A: Matrix, M: Optional[Preconditioner], B: torch.Tenso
     _check(lib().sla_pcg_solve_batched(A.handle, _mh(M), nrhs, _ptr(B), _ptr(X), C.byref(opts),
                                        infos, _stream(stream)), "sla_pcg_solve_batched")
     return X, _infos(infos)
+
+
+def sla_list_kernel_ms(A: Matrix) -> float:
+    """Device ms of the list kernel of the last (regular) list solve on list handle A."""
+    ms = C.c_double(0.0)
+    _check(lib().sla_list_kernel_ms(A.handle, C.byref(ms)), "sla_list_kernel_ms")
+    return ms.value
 
 
 def sla_pcg_solve_batched_noalloc(A: Matrix, M: Optional[Preconditioner], B: torch.Tensor,

@@ -76,6 +76,7 @@ SIGNATURES = {
     "sla_pcg_direction": (_st, [C.c_int32, C.c_int64, C.c_double, _vp, _vp, _vp]),
     "sla_vec_gather": (_st, [C.c_int32, C.c_int64, _vp, _vp, _vp, _vp]),
     "sla_vec_scatter_add": (_st, [C.c_int32, C.c_int64, _vp, _vp, _vp, _vp]),
+    "sla_list_kernel_ms": (_st, [_vp, C.POINTER(C.c_double)]),
     "sla_pcg_solve_batched_noalloc": (_st, [_vp, _vp, _vp, _vp, C.POINTER(sla_pcg_opts),
                                             C.POINTER(sla_pcg_info), _vp]),
     "sla_pcg_kernel_times": (_st, [_vp, _vp, C.c_int32, C.c_int32, C.c_int32, C.POINTER(C.c_double), _vp]),

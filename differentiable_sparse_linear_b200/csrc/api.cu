@@ -558,6 +558,11 @@ static void free_csr(sla_csr *A)
             M->G = nullptr;   // a SPAI preconditioner without G refuses further use
     }
     A->dependents.clear();
+    for (cudaEvent_t &ev : A->list_ev)
+        if (ev) {
+            cudaEventDestroy(ev);
+            ev = nullptr;
+        }
     for (Plan *p : A->plans)
         destroy_plan(p);
     A->plans.clear();

@@ -2,10 +2,10 @@
 // SparseTensorList batch of "torch-sla: Differentiable Sparse Linear Algebra with Adjoint
 // Solvers and Sparse Tensor Parallelism for PyTorch", Methodology §1), forward and adjoint.
 //
-// One block owns one system for its whole solve: the system's vectors (x, r, p, q, z,
-// D^-1, for the adjoint the forward x, and with SPAI y = G^T r) live in shared memory, so the
-// only HBM traffic is the system's matrix (re-read from L2 after the first iteration), b,
-// and the results.  Systems too large for shared memory keep the same vectors in a device
+// One block owns one system for its whole solve: the system's vectors (x, r, p, q, D^-1,
+// for the adjoint the forward x, and with SPAI z and y = G^T r) and its row offsets live in
+// shared memory, so the only HBM traffic is the system's matrix (re-read from L2 after the
+// first iteration), b, and the results.  Systems too large for shared memory keep the same vectors in a device
 // workspace (nv values per row of the batch), with the same code and order of operations.
 // Preconditioners: Jacobi, none, or SPAI z = G (G^T r) + eps r ([SPAI] "Learning Sparse
 // Approximate Inverse Preconditioners for Conjugate Gradient Solvers on GPUs", Approach)
@@ -53,29 +53,67 @@ __device__ __forceinline__ void list_sum2(double &a, double &b, double *s_red)
 }
 
 // q = A p on one system (rows [0, ns), local columns = global - o0), S lanes per row;
-// returns this thread's share of p.q (only the first lane of each row group contributes;
-// 0 without DOT).
+// `rpl` holds the system's row offsets (rpl[i] = first entry of local row i).  Each lane
+// group takes LIST_RU rows at once, so every lane has that many independent loads in
+// flight; a row's terms are still summed in entry order.  The trip count is the same for
+// every lane of a warp (the shuffles need the whole warp).  Returns this thread's share of
+// p.q (only the first lane of each row group contributes; 0 without DOT).
+constexpr int LIST_RU = 4;
+
 template <typename V, int S, bool DOT = true>
-__device__ __forceinline__ double list_spmv(int ns, int64_t o0, const int32_t *rp, const int32_t *ci,
+__device__ __forceinline__ double list_spmv(int ns, int64_t o0, const int32_t *rpl, const int32_t *ci,
                                             const V *val, const V *p, V *q)
 {
+    constexpr int NG = LIST_T / S;
     const int lane = threadIdx.x & (S - 1);
     const int grp = threadIdx.x / S;
-    constexpr int NG = LIST_T / S;
+    const int gw = grp & ~(32 / S - 1);            // first row group of this warp
     double part = 0.0;
-    for (int i = grp; i < ns; i += NG) {
-        const int64_t k0 = rp[o0 + i], k1 = rp[o0 + i + 1];
-        double acc = 0.0;
-        for (int64_t k = k0 + lane; k < k1; k += S)
-            acc = __fma_rn((double)val[k], (double)p[ci[k] - o0], acc);
+    for (int t0 = 0; gw + t0 < ns; t0 += NG * LIST_RU) {
+        uint32_t k[LIST_RU], k1[LIST_RU];          // entry offsets (< 2^31, so k + S cannot wrap)
+        double acc[LIST_RU];
 #pragma unroll
-        for (int off = S / 2; off > 0; off >>= 1)
-            acc += __shfl_xor_sync(0xffffffffu, acc, off, S);
+        for (int u = 0; u < LIST_RU; ++u) {
+            const int i = grp + t0 + u * NG;
+            k[u] = i < ns ? (uint32_t)rpl[i] + lane : 0u;
+            k1[u] = i < ns ? (uint32_t)rpl[i + 1] : 0u;
+            acc[u] = 0.0;
+        }
+        bool more = true;
+        while (more) {
+            V a[LIST_RU];
+            int32_t c[LIST_RU];
+#pragma unroll
+            for (int u = 0; u < LIST_RU; ++u) {
+                const bool in = k[u] < k1[u];
+                a[u] = in ? val[k[u]] : (V)0;
+                c[u] = in ? ci[k[u]] : -1;
+            }
+            more = false;
+#pragma unroll
+            for (int u = 0; u < LIST_RU; ++u) {
+                if (c[u] >= 0)
+                    acc[u] = __fma_rn((double)a[u], (double)p[c[u] - o0], acc[u]);
+                k[u] += S;
+                more |= k[u] < k1[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < LIST_RU; ++u)
+#pragma unroll
+            for (int off = S / 2; off > 0; off >>= 1)
+                acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off, S);
         if (lane == 0) {
-            const V qv = (V)acc;
-            q[i] = qv;
-            if (DOT)
-                part += (double)p[i] * (double)qv;
+#pragma unroll
+            for (int u = 0; u < LIST_RU; ++u) {
+                const int i = grp + t0 + u * NG;
+                if (i < ns) {
+                    const V qv = (V)acc[u];
+                    q[i] = qv;
+                    if (DOT)
+                        part += (double)p[i] * (double)qv;
+                }
+            }
         }
     }
     return part;
@@ -97,9 +135,9 @@ template <typename V, int S>
 __device__ __forceinline__ double list_spai_apply(int ns, int64_t o0, const ListSpai<V> &m, const V *r, V *y,
                                                   V *z)
 {
-    list_spmv<V, S, false>(ns, o0, m.gt_rp, m.gt_ci, m.gt_val, r, y);
+    list_spmv<V, S, false>(ns, o0, m.gt_rp + o0, m.gt_ci, m.gt_val, r, y);
     __syncthreads();
-    list_spmv<V, S, false>(ns, o0, m.g_rp, m.g_ci, m.g_val, y, z);
+    list_spmv<V, S, false>(ns, o0, m.g_rp + o0, m.g_ci, m.g_val, y, z);
     __syncthreads();
     double rz = 0.0;
     for (int i = threadIdx.x; i < ns; i += LIST_T) {
@@ -110,11 +148,16 @@ __device__ __forceinline__ double list_spai_apply(int ns, int64_t o0, const List
     return rz;
 }
 
-// Vectors of one system per row of the batch: x, r, p, q, z, D^-1, forward x, y (SPAI).
-constexpr int LIST_NV = 8;
+// Vectors a system keeps (per row): x, r, p, q, then D^-1 (Jacobi), z and y = G^T r (SPAI),
+// the forward x (adjoint); without SPAI z = D^-1 r is formed where it is used, not stored.
+// In shared memory the system's row offsets follow the vectors.
+__host__ __device__ inline int list_nv(bool jacobi, bool spai, bool adjoint)
+{
+    return 4 + (jacobi ? 1 : 0) + (spai ? 2 : 0) + (adjoint ? 1 : 0);
+}
 
 template <typename V, int S>
-__global__ void __launch_bounds__(LIST_T)
+__global__ void __launch_bounds__(LIST_T, 3)
 k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sys_off, int batch,
            const V *B, V *X, const V *dinv, const V *Xf, V *Gout, double tol, long long maxit_opt,
            sla_pcg_info *info, const ListSpai<V> spai, int use_spai, V *ws)
@@ -122,29 +165,50 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
     extern __shared__ __align__(16) unsigned char s_raw[];
     __shared__ double s_red[2 * (LIST_T / 32) + 2];
     const int tid = threadIdx.x;
+    const bool jac = dinv != nullptr;
+    const int nv = list_nv(jac, use_spai, Xf != nullptr);
     for (int s = blockIdx.x; s < batch; s += gridDim.x) {
         const int64_t o0 = sys_off[s];
         const int ns = (int)(sys_off[s + 1] - o0);
-        V *x = ws ? ws + (int64_t)LIST_NV * o0 : (V *)s_raw;
+        V *x = ws ? ws + (int64_t)nv * o0 : (V *)s_raw;
         V *r = x + ns;
         V *p = r + ns;
         V *q = p + ns;
-        V *z = q + ns;
-        V *dv = z + ns;
-        V *xf = dv + ns;
-        V *y = xf + ns;
+        V *nxt = q + ns;
+        V *dv = nullptr, *z = nullptr, *y = nullptr, *xf = nullptr;
+        if (jac) {
+            dv = nxt;
+            nxt += ns;
+        }
+        if (use_spai) {
+            z = nxt;
+            y = nxt + ns;
+            nxt += 2 * ns;
+        }
+        if (Xf) {
+            xf = nxt;
+            nxt += ns;
+        }
+        // the system's row offsets: staged in shared memory after the vectors
+        const int32_t *rpl = rp + o0;
+        if (!ws) {
+            int32_t *s_rp = (int32_t *)(s_raw + (size_t)nv * ns * sizeof(V));
+            for (int i = tid; i <= ns; i += LIST_T)
+                s_rp[i] = rp[o0 + i];
+            rpl = s_rp;
+        }
         const long long maxit = maxit_opt > 0 ? maxit_opt : 10LL * (ns > 0 ? ns : 1);
 
         double bb = 0.0, rz = 0.0;
         for (int i = tid; i < ns; i += LIST_T) {
             const V bi = B[o0 + i];
-            const V di = dinv ? dinv[o0 + i] : (V)1;
-            const V zi = (V)((double)bi * (double)di);
             x[i] = (V)0;
             r[i] = bi;
-            dv[i] = di;
             if (!use_spai) {
-                z[i] = zi;
+                const V di = jac ? dinv[o0 + i] : (V)1;
+                const V zi = (V)((double)bi * (double)di);
+                if (jac)
+                    dv[i] = di;
                 p[i] = zi;
                 rz += (double)bi * (double)zi;
             }
@@ -152,8 +216,8 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
                 xf[i] = Xf[o0 + i];
             bb += (double)bi * (double)bi;
         }
+        __syncthreads();
         if (use_spai) {
-            __syncthreads();
             rz = list_spai_apply<V, S>(ns, o0, spai, r, y, z);
             for (int i = tid; i < ns; i += LIST_T)
                 p[i] = z[i];
@@ -173,7 +237,7 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
         else {
             while (it < maxit) {
                 ++it;
-                double pq = list_spmv<V, S>(ns, o0, rp, ci, val, p, q), dummy = 0.0;
+                double pq = list_spmv<V, S>(ns, o0, rpl, ci, val, p, q), dummy = 0.0;
                 list_sum2(pq, dummy, s_red);
                 if (!(pq > 0.0) || !isfinite(pq)) {
                     status = SLA_BREAKDOWN;
@@ -187,8 +251,7 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
                     r[i] = rn;
                     rr += (double)rn * (double)rn;
                     if (!use_spai) {
-                        const V zn = (V)((double)rn * (double)dv[i]);
-                        z[i] = zn;
+                        const V zn = jac ? (V)((double)rn * (double)dv[i]) : rn;
                         rzn += (double)rn * (double)zn;
                     }
                 }
@@ -220,8 +283,15 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
                 }
                 const double beta = rzn / rho;
                 rho = rzn;
-                for (int i = tid; i < ns; i += LIST_T)
-                    p[i] = (V)__fma_rn(beta, (double)p[i], (double)z[i]);
+                if (use_spai) {
+                    for (int i = tid; i < ns; i += LIST_T)
+                        p[i] = (V)__fma_rn(beta, (double)p[i], (double)z[i]);
+                } else {
+                    for (int i = tid; i < ns; i += LIST_T) {
+                        const V zi = jac ? (V)((double)r[i] * (double)dv[i]) : r[i];
+                        p[i] = (V)__fma_rn(beta, (double)p[i], (double)zi);
+                    }
+                }
                 __syncthreads();
             }
         }
@@ -233,7 +303,7 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
             const int lane = tid & (S - 1), grp = tid / S;
             for (int i = grp; i < ns; i += LIST_T / S) {
                 const double li = (double)x[i];
-                for (int64_t k = rp[o0 + i] + lane; k < rp[o0 + i + 1]; k += S)
+                for (int64_t k = rpl[i] + lane; k < rpl[i + 1]; k += S)
                     Gout[k] = (V)(-li * (double)xf[ci[k] - o0]);
             }
         }
@@ -247,20 +317,27 @@ k_list_pcg(const int32_t *rp, const int32_t *ci, const V *val, const int64_t *sy
     }
 }
 
-// Shared memory a system's vectors take; above LIST_SMEM_MAX they live in a workspace.
+// Shared memory a system's vectors and row offsets take; above LIST_SMEM_MAX the vectors
+// live in a workspace instead.
 constexpr size_t LIST_SMEM_MAX = 200 * 1024;
+
+static int list_nv_of(const sla_precond *M, bool adjoint)
+{
+    return list_nv(M && M->kind == 1, M && M->kind == 2, adjoint);
+}
 
 static size_t list_smem(const sla_csr *A, int nv)
 {
-    return (size_t)nv * (size_t)A->max_sys_n * (A->dtype == SLA_F32 ? 4 : 8);
+    return (size_t)nv * (size_t)A->max_sys_n * (A->dtype == SLA_F32 ? 4 : 8) +
+           ((size_t)A->max_sys_n + 1) * sizeof(int32_t);
 }
 
 template <typename V, int S>
 static sla_status list_launch(const sla_csr *A, const V *dinv, const ListSpai<V> &spai, int use_spai, V *ws,
                               const void *B, void *X, const void *Xf, void *G, double tol, long long maxit,
-                              sla_pcg_info *d_info, cudaStream_t s)
+                              sla_pcg_info *d_info, bool timed, cudaStream_t s)
 {
-    const size_t shm = ws ? 0 : (size_t)LIST_NV * (size_t)A->max_sys_n * sizeof(V);
+    const size_t shm = ws ? 0 : list_smem(A, list_nv(dinv != nullptr, use_spai != 0, Xf != nullptr));
     auto kern = k_list_pcg<V, S>;
     SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm));
     int per_sm = 0;
@@ -268,16 +345,28 @@ static sla_status list_launch(const sla_csr *A, const V *dinv, const ListSpai<V>
     if (per_sm < 1)
         return fail(SLA_ERR_UNSUPPORTED, "list solve: a system's vectors do not fit in shared memory");
     const int grid = std::min<int64_t>(A->batch, (int64_t)per_sm * A->num_sms);
+    sla_csr *Am = const_cast<sla_csr *>(A);
+    Am->list_ev_recorded = 0;
+    if (timed) {
+        for (cudaEvent_t &ev : Am->list_ev)
+            if (!ev)
+                SLA_CUDA_TRY(cudaEventCreate(&ev));
+        SLA_CUDA_TRY(cudaEventRecord(Am->list_ev[0], s));
+    }
     kern<<<grid, LIST_T, shm, s>>>(A->rp, A->ci, (const V *)A->val, A->d_sys_off, A->batch,
                                    (const V *)B, (V *)X, dinv, (const V *)Xf, (V *)G, tol, maxit,
                                    d_info, spai, use_spai, ws);
     SLA_CUDA_TRY(cudaGetLastError());
+    if (timed) {
+        SLA_CUDA_TRY(cudaEventRecord(Am->list_ev[1], s));
+        Am->list_ev_recorded = 1;
+    }
     return SLA_SUCCESS;
 }
 
 template <typename V>
 static sla_status list_v(const sla_csr *A, const sla_precond *M, V *ws, const void *B, void *X, const void *Xf,
-                         void *G, double tol, long long maxit, sla_pcg_info *d_info, cudaStream_t s)
+                         void *G, double tol, long long maxit, sla_pcg_info *d_info, bool timed, cudaStream_t s)
 {
     const V *dinv = nullptr;
     ListSpai<V> sp{};
@@ -291,12 +380,12 @@ static sla_status list_v(const sla_csr *A, const sla_precond *M, V *ws, const vo
     }
     const double mean = A->n > 0 ? (double)A->nnz / (double)A->n : 0.0;
     if (mean <= 6.0)
-        return list_launch<V, 4>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
+        return list_launch<V, 4>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, timed, s);
     if (mean <= 24.0)
-        return list_launch<V, 8>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
+        return list_launch<V, 8>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, timed, s);
     if (mean <= 64.0)
-        return list_launch<V, 16>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
-    return list_launch<V, 32>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, s);
+        return list_launch<V, 16>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, timed, s);
+    return list_launch<V, 32>(A, dinv, sp, use_spai, ws, B, X, Xf, G, tol, maxit, d_info, timed, s);
 }
 
 static sla_status list_check_precond(const sla_precond *M)
@@ -317,18 +406,19 @@ sla_status run_list_solve(const sla_csr *A, const sla_precond *M, const void *B,
     const long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 0;
     sla_pcg_info *d_info = nullptr;
     SLA_CUDA_TRY(cudaMallocAsync((void **)&d_info, sizeof(sla_pcg_info) * (size_t)A->batch, s));
-    // systems whose vectors do not fit in shared memory: a workspace of LIST_NV values per row
+    // systems whose vectors do not fit in shared memory: a workspace of nv values per row
+    const int nv = list_nv_of(M, Xf != nullptr);
     void *ws = nullptr;
     cudaError_t we = cudaSuccess;
-    if (list_smem(A, LIST_NV) > LIST_SMEM_MAX && A->n > 0)
-        we = cudaMallocAsync(&ws, (size_t)LIST_NV * (size_t)A->n * (A->dtype == SLA_F32 ? 4 : 8), s);
+    if (list_smem(A, nv) > LIST_SMEM_MAX && A->n > 0)
+        we = cudaMallocAsync(&ws, (size_t)nv * (size_t)A->n * (A->dtype == SLA_F32 ? 4 : 8), s);
     sla_status st;
     if (we != cudaSuccess)
         st = fail(SLA_ERR_OOM, "list solve: workspace allocation");
     else if (A->dtype == SLA_F32)
-        st = list_v<float>(A, M, (float *)ws, B, X, Xf, G, tol, maxit, d_info, s);
+        st = list_v<float>(A, M, (float *)ws, B, X, Xf, G, tol, maxit, d_info, true, s);
     else
-        st = list_v<double>(A, M, (double *)ws, B, X, Xf, G, tol, maxit, d_info, s);
+        st = list_v<double>(A, M, (double *)ws, B, X, Xf, G, tol, maxit, d_info, true, s);
     if (ws)
         cudaFreeAsync(ws, s);
     if (st == SLA_SUCCESS) {
@@ -408,13 +498,28 @@ sla_status launch_list_kernel(const sla_csr *A, const sla_precond *M, const void
 {
     SLA_TRY(list_check_precond(M));
     // this path allocates nothing: every system's vectors must fit in shared memory
-    if (list_smem(A, LIST_NV) > LIST_SMEM_MAX)
+    if (list_smem(A, list_nv_of(M, false)) > LIST_SMEM_MAX)
         return fail(SLA_ERR_UNSUPPORTED, "list solve without allocation: largest system exceeds the shared-memory size");
     const double tol = (opts && opts->rtol > 0) ? opts->rtol : (A->dtype == SLA_F32 ? 1e-6 : 1e-10);
     const long long maxit = (opts && opts->maxit > 0) ? opts->maxit : 0;
     if (A->dtype == SLA_F32)
-        return list_v<float>(A, M, (float *)nullptr, B, X, nullptr, nullptr, tol, maxit, d_info, s);
-    return list_v<double>(A, M, (double *)nullptr, B, X, nullptr, nullptr, tol, maxit, d_info, s);
+        return list_v<float>(A, M, (float *)nullptr, B, X, nullptr, nullptr, tol, maxit, d_info, false, s);
+    return list_v<double>(A, M, (double *)nullptr, B, X, nullptr, nullptr, tol, maxit, d_info, false, s);
 }
 
 }  // namespace sla
+
+using namespace sla;
+
+extern "C" sla_status sla_list_kernel_ms(const sla_csr *A, double *h_ms)
+{
+    if (!A || !h_ms)
+        return fail(SLA_ERR_INVALID_ARG, "NULL argument");
+    if (A->batch < 1 || A->sys_off.empty() || !A->list_ev_recorded)
+        return fail(SLA_ERR_INVALID_ARG, "no list solve has run on this handle");
+    SLA_CUDA_TRY(cudaEventSynchronize(A->list_ev[1]));
+    float ms = 0.f;
+    SLA_CUDA_TRY(cudaEventElapsedTime(&ms, A->list_ev[0], A->list_ev[1]));
+    *h_ms = (double)ms;
+    return SLA_SUCCESS;
+}

@@ -203,6 +203,9 @@ struct sla_csr {
     // preconditioners built on this handle (as A or as G); they are detached when it is
     // destroyed, whatever the order the caller destroys handles in
     std::vector<sla_precond *> dependents;
+    // device time of the last list solve's kernel (CUDA events around its launch)
+    cudaEvent_t list_ev[2] = {nullptr, nullptr};
+    int list_ev_recorded = 0;
 };
 
 struct sla_precond {

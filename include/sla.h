@@ -349,6 +349,13 @@ SLA_API sla_status sla_pcg_solve_batched_noalloc(const sla_csr *A, const sla_pre
 SLA_API sla_status sla_pcg_kernel_times(const sla_csr *A, const sla_precond *M, int32_t nrhs,
                                         int32_t vector_f64, int32_t reps, double *h_ms, void *stream);
 
+/* Device time, in ms, of the list kernel of the last list solve on list handle A (forward or
+ * adjoint; CUDA events recorded on the solve's stream right before and after the kernel's
+ * launch, so the time holds that one kernel and nothing the call does around it).
+ * SLA_ERR_INVALID_ARG when A is not a list handle or no list solve has run on it since its
+ * creation (the allocation-free list solve is not timed).  Waits for the end event. */
+SLA_API sla_status sla_list_kernel_ms(const sla_csr *A, double *h_ms);
+
 /* Device time per phase of the last persistent-engine solve of the (A, M, nrhs, vector_f64)
  * solver, measured inside the kernel by block 0 from one grid barrier to the next (so each
  * phase's time includes the barrier that ends it).  h_ms[0..3]: mean ms of a
