@@ -859,34 +859,14 @@ sla_status sla_precond_jacobi(sla_precond **out, const sla_csr *A, void *stream)
     return SLA_SUCCESS;
 }
 
-// G^T by a counting sort of G's entries by column on the host (set-up only): row j of G^T
-// lists the rows i of G holding column j in increasing i.  perm[k] = position in G of the
-// k-th entry of G^T, so a later change of G's values is one device gather.
+// G^T on the device (device_transpose: a stable sort of G's entries by column): row j of
+// G^T lists the rows i of G holding column j in increasing i.  perm[k] = position in G of
+// the k-th entry of G^T, so a later change of G's values is one device gather.  Only G^T's
+// row pointers come back to the host (for the row partitions, like every handle's).
 static sla_status spai_transpose(sla_precond *M, cudaStream_t s)
 {
     const sla_csr *G = M->G;
     const int64_t n = G->n, nnz = G->nnz;
-    std::vector<int32_t> ci((size_t)nnz);
-    if (nnz > 0) {
-        SLA_CUDA_TRY(cudaMemcpyAsync(ci.data(), G->ci, (size_t)nnz * sizeof(int32_t),
-                                     cudaMemcpyDeviceToHost, s));
-        SLA_CUDA_TRY(cudaStreamSynchronize(s));
-    }
-    std::vector<int32_t> rpT((size_t)n + 1, 0), ciT((size_t)nnz), perm((size_t)nnz);
-    for (int64_t k = 0; k < nnz; ++k) {
-        if (ci[(size_t)k] < 0 || ci[(size_t)k] >= n)
-            return fail(SLA_ERR_INVALID_CSR, "G: column index out of range");
-        rpT[(size_t)ci[(size_t)k] + 1] += 1;
-    }
-    for (int64_t j = 0; j < n; ++j)
-        rpT[(size_t)j + 1] += rpT[(size_t)j];
-    std::vector<int32_t> fill(rpT.begin(), rpT.end() - 1);
-    for (int64_t i = 0; i < n; ++i)
-        for (int64_t k = G->h_rp[(size_t)i]; k < G->h_rp[(size_t)i + 1]; ++k) {
-            const int32_t dst = fill[(size_t)ci[(size_t)k]]++;
-            ciT[(size_t)dst] = (int32_t)i;
-            perm[(size_t)dst] = (int32_t)k;
-        }
     sla_csr *GT = new sla_csr();
     GT->n = n;
     GT->nnz = nnz;
@@ -894,12 +874,7 @@ static sla_status spai_transpose(sla_precond *M, cudaStream_t s)
     GT->device = G->device;
     GT->num_sms = G->num_sms;
     GT->max_sys_n = n;
-    GT->h_rp = rpT;
     M->GT = GT;
-    int64_t mx = 0;
-    for (int64_t j = 0; j < n; ++j)
-        mx = std::max<int64_t>(mx, (int64_t)rpT[(size_t)j + 1] - rpT[(size_t)j]);
-    GT->max_row_len = mx;
     SLA_CUDA_TRY(cudaMalloc((void **)&GT->own_rp, ((size_t)n + 1) * sizeof(int32_t)));
     SLA_CUDA_TRY(cudaMalloc((void **)&GT->own_ci, (size_t)std::max<int64_t>(nnz, 1) * sizeof(int32_t)));
     SLA_CUDA_TRY(cudaMalloc(&GT->own_val, (size_t)std::max<int64_t>(nnz, 1) * vbytes(G->dtype)));
@@ -907,16 +882,16 @@ static sla_status spai_transpose(sla_precond *M, cudaStream_t s)
     GT->rp = GT->own_rp;
     GT->ci = GT->own_ci;
     GT->val = GT->own_val;
-    SLA_CUDA_TRY(cudaMemcpyAsync(GT->own_rp, rpT.data(), ((size_t)n + 1) * sizeof(int32_t),
-                                 cudaMemcpyHostToDevice, s));
-    if (nnz > 0) {
-        SLA_CUDA_TRY(cudaMemcpyAsync(GT->own_ci, ciT.data(), (size_t)nnz * sizeof(int32_t),
-                                     cudaMemcpyHostToDevice, s));
-        SLA_CUDA_TRY(cudaMemcpyAsync(M->d_perm, perm.data(), (size_t)nnz * sizeof(int32_t),
-                                     cudaMemcpyHostToDevice, s));
-    }
+    SLA_TRY(device_transpose(G, GT->own_rp, GT->own_ci, M->d_perm, s));
+    GT->h_rp.resize((size_t)n + 1);
+    SLA_CUDA_TRY(cudaMemcpyAsync(GT->h_rp.data(), GT->own_rp, ((size_t)n + 1) * sizeof(int32_t),
+                                 cudaMemcpyDeviceToHost, s));
     SLA_TRY(refresh_transpose_values(G, GT, M->d_perm, s));
     SLA_CUDA_TRY(cudaStreamSynchronize(s));
+    int64_t mx = 0;
+    for (int64_t j = 0; j < n; ++j)
+        mx = std::max<int64_t>(mx, (int64_t)GT->h_rp[(size_t)j + 1] - GT->h_rp[(size_t)j]);
+    GT->max_row_len = mx;
     return SLA_SUCCESS;
 }
 

@@ -1,72 +1,95 @@
-// Set-up of the column-sorted row segments (csb.cuh) on the host, once per matrix pattern.
+// Set-up of the column-sorted row segments (csb.cuh), once per matrix pattern.
 //
-// Segments: contiguous rows with about equal (entries + rows), at most CSB_RMAX rows each
-// (their sums live in shared memory) and as few as that allows -- the larger a segment, the
-// closer its sorted columns lie -- rounded up to a multiple of the SpMV's grid (one block
-// per SM), so that every block takes the same number of segments.  Each segment's
-// entries are sorted by (column, row) -- the segments are independent and are sorted on all
-// host threads -- and cut into chunks of 32; a chunk also ends early when its next column
+// Segments (on the host, from the row pointers): contiguous rows with about equal
+// (entries + rows), at most CSB_RMAX rows each (their sums live in shared memory) and as few
+// as that allows -- the larger a segment, the closer its sorted columns lie -- rounded up to
+// a multiple of the SpMV's grid (one block per SM), so that every block takes the same number
+// of segments.
+//
+// The entries (on the device): every entry gets the key (segment, column, local row), the
+// keys are sorted with the radix sort of radix_sort.cuh, and one warp per segment cuts the
+// segment's sorted entries into chunks of 32; a chunk also ends early when its next column
 // would lie 65536 or more past the chunk's first column (the column offset is 16 bits), and
-// the rest of its slots are padding.
+// the rest of its slots are padding.  A first walk counts each segment's chunks, a second
+// writes them.
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cstring>
 #include <memory>
-#include <thread>
 #include <vector>
 
 #include "sla.h"
 #include "sla_internal.cuh"
 #include "csb.cuh"
+#include "radix_sort.cuh"
 
 namespace sla {
 
 namespace {
 
+constexpr int CSB_RB = 14;                      // bits of a local row in the sort key
+static_assert(CSB_RMAX <= (1 << CSB_RB), "local rows must fit the key's row field");
 
-struct SegOut {
-    std::vector<int32_t> cbase;
-    std::vector<uint32_t> pk;
-    std::vector<int32_t> perm;
-};
-
-// Sort one segment's entries by (column, row) and cut them into chunks.
-void build_segment(const int32_t *rp, const int32_t *ci, int64_t r0, int64_t r1, SegOut &o)
+// key[k] = (segment << (cb + CSB_RB)) | (column << CSB_RB) | local row, val[k] = k; one warp
+// per row, its segment found by binary search over the segments' first rows.
+__global__ void k_csb_keys(int64_t n, const int32_t *rp, const int32_t *ci, const int32_t *seg_row0, int nseg,
+                           int cb, uint64_t *key, int32_t *val)
 {
-    const int64_t k0 = rp[r0], k1 = rp[r1];
-    std::vector<uint64_t> key((size_t)(k1 - k0));
-    for (int64_t r = r0; r < r1; ++r)
-        for (int64_t k = rp[r]; k < rp[r + 1]; ++k)   // column in the high bits, local row below
-            key[(size_t)(k - k0)] = ((uint64_t)(uint32_t)ci[k] << 32) | (uint64_t)(uint32_t)(r - r0);
-    // (column, row) pairs are distinct, so the order is unique
-    std::vector<int64_t> pos((size_t)(k1 - k0));
-    for (size_t i = 0; i < pos.size(); ++i)
-        pos[i] = (int64_t)i;
-    std::sort(pos.begin(), pos.end(), [&](int64_t a, int64_t b) { return key[(size_t)a] < key[(size_t)b]; });
-    o.cbase.clear();
-    o.pk.clear();
-    o.perm.clear();
-    size_t i = 0;
-    while (i < pos.size()) {
-        const int64_t first = pos[i];
-        const uint32_t base = (uint32_t)(key[(size_t)first] >> 32);
-        o.cbase.push_back((int32_t)base);
-        int l = 0;
-        for (; l < 32 && i < pos.size(); ++l) {
-            const int64_t e = pos[i];
-            const uint32_t col = (uint32_t)(key[(size_t)e] >> 32);
-            if (col - base > 0xFFFFu)
-                break;
-            const uint32_t row = (uint32_t)(key[(size_t)e] & 0xFFFFFFFFu);
-            o.pk.push_back(((col - base) << 16) | row);
-            o.perm.push_back((int32_t)(k0 + e));
-            ++i;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; i < n; i += warps) {
+        int lo = 0, hi = nseg - 1;              // last segment whose first row is <= i
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seg_row0[mid] <= i)
+                lo = mid;
+            else
+                hi = mid - 1;
         }
-        for (; l < 32; ++l) {
-            o.pk.push_back(CSB_PAD);
-            o.perm.push_back(-1);
+        const uint64_t hi_bits = ((uint64_t)lo << (cb + CSB_RB)) | (uint64_t)(i - seg_row0[lo]);
+        for (int64_t k = rp[i] + lane; k < rp[i + 1]; k += 32) {
+            key[k] = hi_bits | ((uint64_t)(uint32_t)ci[k] << CSB_RB);
+            val[k] = (int32_t)k;
         }
+    }
+}
+
+// One warp per segment walks its sorted entries chunk by chunk: a chunk takes the next
+// entries up to 32 whose column lies within 65535 of the first one (a prefix of the 32 read,
+// since the columns ascend).  WRITE = false: chunk counts; true: the chunks themselves,
+// from the segment's first chunk ch0[s].
+template <bool WRITE>
+__global__ void k_csb_chunks(int nseg, const int32_t *seg_row0, const int32_t *rp, const uint64_t *key,
+                             const int32_t *val, int cb, int32_t *cnt, const int32_t *ch0, int32_t *cbase,
+                             uint32_t *pk, int32_t *perm)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    const uint64_t colmask = (cb >= 32) ? 0xFFFFFFFFull : ((1ull << cb) - 1ull);
+    for (int64_t sg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; sg < nseg; sg += warps) {
+        const int64_t e0 = rp[seg_row0[sg]], e1 = rp[seg_row0[sg + 1]];
+        int64_t ch = WRITE ? (int64_t)ch0[sg] : 0;
+        for (int64_t pos = e0; pos < e1;) {
+            const int64_t t = pos + lane;
+            const bool in = t < e1;
+            const uint64_t kk = in ? key[t] : 0ull;
+            const uint32_t col = (uint32_t)((kk >> CSB_RB) & colmask);
+            const uint32_t base = __shfl_sync(0xffffffffu, col, 0);
+            const bool ok = in && col - base <= 0xFFFFu;
+            const int take = __popc(__ballot_sync(0xffffffffu, ok));
+            if (WRITE) {
+                const uint32_t lr = (uint32_t)(kk & ((1u << CSB_RB) - 1u));
+                pk[ch * 32 + lane] = lane < take ? ((col - base) << 16) | lr : CSB_PAD;
+                perm[ch * 32 + lane] = lane < take ? val[t] : -1;
+                if (lane == 0)
+                    cbase[ch] = (int32_t)base;
+            }
+            ++ch;
+            pos += take;
+        }
+        if (!WRITE && lane == 0)
+            cnt[sg] = (int32_t)ch;
     }
 }
 
@@ -95,11 +118,6 @@ sla_status ensure_csb(sla_csr *A, cudaStream_t s, const CsbPart **out)
     if (A->bdim != 1 || A->n > 0x7FFFFFFF || A->nnz >= ((int64_t)1 << 31))
         return fail(SLA_ERR_UNSUPPORTED, "column-sorted segments: CSR matrices with int32 sizes only");
     const int64_t n = A->n;
-    std::vector<int32_t> h_ci((size_t)A->nnz);
-    if (A->nnz > 0) {
-        SLA_CUDA_TRY(cudaMemcpyAsync(h_ci.data(), A->ci, (size_t)A->nnz * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
-        SLA_CUDA_TRY(cudaStreamSynchronize(s));
-    }
     const int32_t *rp = A->h_rp.data();
     // segment boundaries: equal shares of (entries + rows), at most CSB_RMAX rows
     const int64_t total = A->nnz + n;
@@ -136,67 +154,76 @@ sla_status ensure_csb(sla_csr *A, cudaStream_t s, const CsbPart **out)
         row0.push_back((int32_t)n);
     }
     nseg = (int64_t)row0.size() - 1;
-    std::vector<SegOut> segs((size_t)nseg);
-    const unsigned hw = std::max(1u, std::thread::hardware_concurrency());
-    const unsigned nth = (unsigned)std::min<int64_t>(hw, nseg);
-    {
-        std::vector<std::thread> th;
-        for (unsigned t = 0; t < nth; ++t)
-            th.emplace_back([&, t] {
-                for (int64_t sgi = t; sgi < nseg; sgi += nth)
-                    build_segment(rp, h_ci.data(), row0[(size_t)sgi], row0[(size_t)sgi + 1], segs[(size_t)sgi]);
-            });
-        for (auto &x : th)
-            x.join();
-    }
-    std::vector<int32_t> ch0((size_t)nseg + 1, 0);
     int rmax = 0;
-    for (int64_t sgi = 0; sgi < nseg; ++sgi) {
-        ch0[(size_t)sgi + 1] = ch0[(size_t)sgi] + (int32_t)segs[(size_t)sgi].cbase.size();
+    for (int64_t sgi = 0; sgi < nseg; ++sgi)
         rmax = std::max(rmax, row0[(size_t)sgi + 1] - row0[(size_t)sgi]);
-    }
-    const int64_t nch = ch0.back();
+    const int cb = std::max(1, bits_for((uint64_t)std::max<int64_t>(n - 1, 0)));
+    const int sb = bits_for((uint64_t)(nseg - 1));
+    if (sb + cb + CSB_RB > 64)
+        return fail(SLA_ERR_UNSUPPORTED, "column-sorted segments: sort key wider than 64 bits");
+    const int64_t nnz = A->nnz;
     auto cp = std::make_unique<CsbPart>();
     cp->n_seg = (int)nseg;
     cp->rmax = rmax;
+    cudaError_t e = cudaMalloc((void **)&cp->d_seg_row0, sizeof(int32_t) * (size_t)(nseg + 1));
+    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_seg_ch0, sizeof(int32_t) * (size_t)(nseg + 1));
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(cp->d_seg_row0, row0.data(), sizeof(int32_t) * row0.size(), cudaMemcpyHostToDevice, s);
+    // sort (segment, column, local row) keys with the entry positions
+    uint64_t *k0 = nullptr, *k1 = nullptr, *ks = nullptr;
+    int32_t *v0 = nullptr, *v1 = nullptr, *vs = nullptr, *d_cnt = nullptr;
+    const size_t ne = (size_t)std::max<int64_t>(nnz, 1);
+    if (e == cudaSuccess) e = cudaMallocAsync((void **)&k0, sizeof(uint64_t) * ne, s);
+    if (e == cudaSuccess) e = cudaMallocAsync((void **)&k1, sizeof(uint64_t) * ne, s);
+    if (e == cudaSuccess) e = cudaMallocAsync((void **)&v0, sizeof(int32_t) * ne, s);
+    if (e == cudaSuccess) e = cudaMallocAsync((void **)&v1, sizeof(int32_t) * ne, s);
+    if (e == cudaSuccess) e = cudaMallocAsync((void **)&d_cnt, sizeof(int32_t) * (size_t)nseg, s);
+    const int rgrid = (int)std::max<int64_t>(1, std::min<int64_t>((n + 7) / 8, (int64_t)A->num_sms * 16));
+    const int sgrid = (int)std::max<int64_t>(1, (nseg + 7) / 8);
+    if (e == cudaSuccess && n > 0) {
+        k_csb_keys<<<rgrid, 256, 0, s>>>(n, A->rp, A->ci, cp->d_seg_row0, (int)nseg, cb, k0, v0);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess)
+        e = radix_sort_pairs<uint64_t>(k0, v0, k1, v1, nnz, sb + cb + CSB_RB, &ks, &vs, s);
+    if (e == cudaSuccess) {
+        k_csb_chunks<false><<<sgrid, 256, 0, s>>>((int)nseg, cp->d_seg_row0, A->rp, ks, vs, cb, d_cnt, nullptr,
+                                                  nullptr, nullptr, nullptr);
+        e = cudaGetLastError();
+    }
+    std::vector<int32_t> cnt((size_t)nseg);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(cnt.data(), d_cnt, sizeof(int32_t) * (size_t)nseg, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    std::vector<int32_t> ch0((size_t)nseg + 1, 0);
+    for (int64_t sgi = 0; sgi < nseg; ++sgi)
+        ch0[(size_t)sgi + 1] = ch0[(size_t)sgi] + cnt[(size_t)sgi];
+    const int64_t nch = ch0.back();
     cp->n_chunks = nch;
     const size_t vb = A->dtype == SLA_F32 ? 4 : 8;
-    auto fail_free = [&](cudaError_t e) {
+    const size_t nc = (size_t)std::max<int64_t>(nch, 1);
+    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_cbase, sizeof(int32_t) * nc);
+    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_pk, sizeof(uint32_t) * 32 * nc);
+    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_perm, sizeof(int32_t) * 32 * nc);
+    if (e == cudaSuccess) e = cudaMalloc(&cp->d_val, vb * 32 * nc);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(cp->d_seg_ch0, ch0.data(), sizeof(int32_t) * ch0.size(), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && nch > 0) {
+        k_csb_chunks<true><<<sgrid, 256, 0, s>>>((int)nseg, cp->d_seg_row0, A->rp, ks, vs, cb, nullptr,
+                                                 cp->d_seg_ch0, cp->d_cbase, cp->d_pk, cp->d_perm);
+        e = cudaGetLastError();
+    }
+    for (void *p : {(void *)k0, (void *)k1, (void *)v0, (void *)v1, (void *)d_cnt})
+        if (p)
+            cudaFreeAsync(p, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
         A->csb = cp.release();
         free_csb(A);
-        return cuda_fail(e, "column-sorted segments: device allocation");
-    };
-    cudaError_t e = cudaSuccess;
-    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_seg_row0, sizeof(int32_t) * (size_t)(nseg + 1));
-    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_seg_ch0, sizeof(int32_t) * (size_t)(nseg + 1));
-    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_cbase, sizeof(int32_t) * (size_t)std::max<int64_t>(nch, 1));
-    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_pk, sizeof(uint32_t) * 32 * (size_t)std::max<int64_t>(nch, 1));
-    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_perm, sizeof(int32_t) * 32 * (size_t)std::max<int64_t>(nch, 1));
-    if (e == cudaSuccess) e = cudaMalloc(&cp->d_val, vb * 32 * (size_t)std::max<int64_t>(nch, 1));
-    if (e != cudaSuccess)
-        return fail_free(e);
-    // gather the per-segment pieces into whole host arrays, then one copy each
-    std::vector<int32_t> cb((size_t)nch);
-    std::vector<uint32_t> pk((size_t)nch * 32);
-    std::vector<int32_t> perm((size_t)nch * 32);
-    for (int64_t sgi = 0; sgi < nseg; ++sgi) {
-        const SegOut &o = segs[(size_t)sgi];
-        const size_t c0 = (size_t)ch0[(size_t)sgi];
-        if (!o.cbase.empty()) {
-            std::memcpy(&cb[c0], o.cbase.data(), o.cbase.size() * sizeof(int32_t));
-            std::memcpy(&pk[c0 * 32], o.pk.data(), o.pk.size() * sizeof(uint32_t));
-            std::memcpy(&perm[c0 * 32], o.perm.data(), o.perm.size() * sizeof(int32_t));
-        }
+        return cuda_fail(e, "column-sorted segments: device build");
     }
-    segs.clear();
-    e = cudaMemcpyAsync(cp->d_seg_row0, row0.data(), sizeof(int32_t) * row0.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(cp->d_seg_ch0, ch0.data(), sizeof(int32_t) * ch0.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && nch) e = cudaMemcpyAsync(cp->d_cbase, cb.data(), sizeof(int32_t) * cb.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && nch) e = cudaMemcpyAsync(cp->d_pk, pk.data(), sizeof(uint32_t) * pk.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && nch) e = cudaMemcpyAsync(cp->d_perm, perm.data(), sizeof(int32_t) * perm.size(), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess)
-        return fail_free(e);
     A->csb = cp.release();
     A->csb_vals_current = 0;
     *out = A->csb;

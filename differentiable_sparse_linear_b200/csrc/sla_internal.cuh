@@ -273,6 +273,10 @@ sla_status launch_pattern_grad(const sla_csr *A, int K, int vec64, const void *l
                                void *g, cudaStream_t s, double scale = -1.0);
 sla_status launch_validate(const sla_csr *A, int *d_err, cudaStream_t s);
 sla_status launch_jacobi_dinv(const sla_csr *A, void *dinv64, void *dinv32, int *d_err, cudaStream_t s);
+// G^T of a CSR matrix on the device: row pointers (n+1), columns and perm (nnz each, perm[t] =
+// position in G of G^T's t-th entry), all caller-allocated.  SLA_ERR_INVALID_CSR for a
+// column of G outside [0, n).  Synchronises s.
+sla_status device_transpose(const sla_csr *G, int32_t *rpT, int32_t *ciT, int32_t *perm, cudaStream_t s);
 sla_status refresh_transpose_values(const sla_csr *G, sla_csr *GT, const int32_t *d_perm,
                                     cudaStream_t s);
 sla_status capture_plan_graph(sla_csr *A, Plan *p);
