@@ -364,14 +364,19 @@ def run_ours(args):
     spai = w.precond == "spai"
     form_a = isinstance(A, W.BSR) or (not is_list and int(np.diff(A.row_ptr).max(initial=0)) > 16)
     form_gt = spai and int(np.bincount(w.G.col, minlength=A.n_rows).max(initial=0)) > 16
-    q_k, us_k = (2 if form_a else 1), (2 if form_gt else 1)
-    # single-RHS long-row matrices run on column-sorted copies whose values are gathered from
-    # the CSR values before every graph-engine solve: one kernel per such matrix
+    # single-RHS long-row matrices run on column-sorted copies whose values (and per-segment
+    # row bounds) are gathered from the CSR values before every graph-engine solve: two
+    # kernels per such matrix; with fp32 values and vectors each of their products is
+    # preceded by the max |v| kernel of its fixed-point row sums
     one_col = nrhs_of(w) == 1 and not is_list and not isinstance(A, W.BSR)
     form_g = spai and int(np.diff(w.G.row_ptr).max(initial=0)) > 16
-    csb_gathers = (int(form_a) + int(form_g) + int(form_gt)) if one_col else 0
-    body_kernels = 2 * (q_k + us_k + 1) if spai else 2 * (q_k + 1)   # two iterations per loop body
-    prologue = us_k + 1 if spai else 1
+    fx = int(one_col and vbytes(w.dtype) == 4)
+    q_k = (2 + fx) if form_a else 1
+    us_k = (2 + fx) if form_gt else 1
+    z_k = 1 + fx * int(form_g)
+    csb_gathers = 2 * (int(form_a) + int(form_g) + int(form_gt)) if one_col else 0
+    body_kernels = 2 * (q_k + us_k + z_k) if spai else 2 * (q_k + 1)   # two iterations per loop body
+    prologue = us_k + z_k if spai else 1
     engines_seen = set()
 
     def launches(iters: int, engine: str) -> int:

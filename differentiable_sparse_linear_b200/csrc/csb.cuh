@@ -17,9 +17,21 @@
 // values may change between solves; the pattern may not).  8 bytes per entry plus 4 per 32
 // entries, as CSR's value + column index.
 //
-// The sums are fp64 in any order (the atomic adds' order varies from launch to launch), so
-// a row sum may differ from one launch to the next by the last bits of an fp64 value, which
-// the rounding to fp32 vectors almost always absorbs.
+// Row sums.  With fp32 values and vectors every product a_ij v_j is rounded to an integer
+// on a per-segment fixed-point scale and the row sums are exact integer sums, kept as three
+// 32-bit words per row: the integer's low lb bits, its next lb bits, and the signed rest,
+// each added with a native 32-bit shared-memory atomic (fp64 shared atomics, a
+// compare-and-swap loop on 8-byte slots that meet more bank conflicts, made the products
+// over half again as slow on B200).  The scale 2^sc is chosen so that bound = (largest sum
+// of |a_ij| over a row of the segment) x max_j |v_j| maps below 2^EB, EB = min(62, 2 lb +
+// 30): every term fits an int64 (one fp64-to-integer conversion per entry) and no word's sum
+// can overflow (lb is set from the longest row, so that row's lower words cannot carry out
+// of 32 bits).  Each term is rounded once, to 2^-(EB+1) of the bound (about 1e-19 of it):
+// rows far below their segment's bound keep about as many digits as fp64 sums give them.
+// The result is the same whatever the order of the adds, so these products are
+// bit-reproducible.  max |v_j| comes from k_vec_absmax launched right before (one partial
+// per block); when it or the bound is not finite the segment falls back to fp64 atomic adds
+// (as fp64-vector products always do), so a NaN or Inf still reaches the result.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -30,7 +42,13 @@
 
 namespace sla {
 
-constexpr int CSB_RMAX = 16384;                // rows per segment (fp64 sums in shared memory)
+constexpr int CSB_RMAX = 16384;                // rows per segment with fp64 sums (8 bytes a row)
+// rows per segment with fp32 values (three 4-byte fixed-point words a row): 128 KB of sums
+// leave the other half of the SM's 256 KB of L1/shared memory to cache the gathered
+// operand lines (with 16384 rows, 192 KB of sums left 60 KB of L1 and the products ran 7 %
+// slower on the power-law 4M system despite the denser segments)
+constexpr int CSB_RMAX_F32 = 10922;
+constexpr int CSB_WORDS = 3;
 constexpr uint32_t CSB_PAD = 0xFFFFu;
 
 template <typename VM>
@@ -42,7 +60,77 @@ struct CsbView {
     const VM *val;                             // per entry slot
     int n_seg;
     int rmax;                                  // rows of the largest segment
+    const double *seg_bound;                   // per segment: max over rows of sum |a_ij|
+    const float *vmax;                         // per-block max |v_j| of the operand, or null
+    int vmax_n;
+    int lb;                                    // bits of the fixed-point low word
 };
+
+constexpr int CSB_VMAX_T = 512;                // threads of k_vec_absmax
+
+// Per-block max |v_i| over v[0, n) into out[blockIdx.x]; +Inf if the block saw a value that
+// is not finite.
+template <typename V>
+__global__ void __launch_bounds__(CSB_VMAX_T) k_vec_absmax(int64_t n, const V *v, float *out, const PcgState *st)
+{
+    __shared__ float s_m[CSB_VMAX_T / 32];
+    if (st && *(volatile const int *)&st->all_done)
+        return;
+    float m = 0.f;
+    bool bad = false;
+    const int64_t stride = (int64_t)gridDim.x * CSB_VMAX_T;
+    for (int64_t i = (int64_t)blockIdx.x * CSB_VMAX_T + threadIdx.x; i < n; i += stride) {
+        const float a = fabsf((float)v[i]);
+        bad |= !(a <= 3.0e38f);
+        m = fmaxf(m, a);
+    }
+    if (bad)
+        m = __int_as_float(0x7f800000);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0)
+        s_m[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int w = 0; w < CSB_VMAX_T / 32; ++w)
+            t = fmaxf(t, s_m[w]);
+        out[blockIdx.x] = t;
+    }
+}
+
+// Per segment the largest row sum of |a_ij| (fp64), from the CSR values: a block per
+// segment, a warp per row.
+template <typename VM>
+__global__ void __launch_bounds__(256) k_csb_bounds(int n_seg, const int32_t *seg_row0, const int32_t *rp,
+                                                    const VM *val, double *bound)
+{
+    __shared__ double s_w[8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int sg = blockIdx.x; sg < n_seg; sg += gridDim.x) {
+        double wm = 0.0;
+        for (int r = seg_row0[sg] + warp; r < seg_row0[sg + 1]; r += 8) {
+            double a = 0.0;
+            for (int k = rp[r] + lane; k < rp[r + 1]; k += 32)
+                a += fabs((double)val[k]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                a += __shfl_xor_sync(0xffffffffu, a, off);
+            wm = fmax(wm, a);
+        }
+        if (lane == 0)
+            s_w[warp] = wm;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t = 0.0;
+            for (int w = 0; w < 8; ++w)
+                t = fmax(t, s_w[w]);
+            bound[sg] = t;
+        }
+        __syncthreads();
+    }
+}
 
 // 4 chunks per warp per round with the next round prefetched measured the same as 2, 6, or
 // 8 without the prefetch (q = A p on the 4M system: 0.773 / 0.773 / 0.786 / 0.783 ms).
@@ -50,6 +138,12 @@ struct CsbCfg {
     static constexpr int T = 1024;             // threads per block (one block per SM)
     static constexpr int U = 4;                // chunks per warp per round
 };
+
+// Shared-memory 32-bit add without a returned value (a native shared-memory atomic).
+__device__ __forceinline__ void red_add_u32(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"((unsigned)__cvta_generic_to_shared(p)), "r"(v) : "memory");
+}
 
 // One round's matrix data of a warp: U chunks (or padding past the segment's end).
 template <typename VM, int U>
@@ -96,12 +190,33 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
     __shared__ double s_scal[Op::NS > 0 ? Op::NS : 1];
     __shared__ double s_sum[NR];
     __shared__ int s_flag;
+    __shared__ float s_vm[NW];
+    // fixed-point row sums (see the top of this file): fp32 values and vectors only
+    constexpr bool FIX = sizeof(VM) == 4 && sizeof(VV) == 4;
+    // fixed point: high words s_w[0, R), middle words s_w[R, 2R), low words s_w[2R, 3R) of
+    // the segment's R rows (s_y[0, R) of the fp64 path shares the first 2R words)
+    uint32_t *s_w = reinterpret_cast<uint32_t *>(s_y);
 
     if (op.skip())
         return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0)
         op.stage(s_scal);
+    float vmax = __int_as_float(0x7f800000);                // +Inf: no usable bound
+    if (FIX && c.vmax) {
+        float m = 0.f;
+        for (int b = tid; b < c.vmax_n; b += T)
+            m = fmaxf(m, c.vmax[b]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0)
+            s_vm[warp] = m;
+        __syncthreads();
+        vmax = 0.f;
+        for (int w = 0; w < NW; ++w)
+            vmax = fmaxf(vmax, s_vm[w]);
+    }
     __syncthreads();
     GlobalRows<Op, 1> rv{op};
     double part[NR];
@@ -114,11 +229,27 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
         const int R = c.seg_row0[s + 1] - r0;
         const int ch1 = c.seg_ch0[s + 1];
         int ch = c.seg_ch0[s] + warp;
+        // this segment's scale 2^sc (block-uniform), or the fp64 path
+        bool fix = false;
+        double scale = 1.0, unscale = 1.0;
+        if (FIX && c.vmax) {
+            const double bound = c.seg_bound[s] * (double)vmax;
+            if (bound == 0.0) {
+                fix = true;
+            } else if (bound <= 1.0e300) {           // finite (and not NaN)
+                const int eb = min(62, 2 * c.lb + 30);
+                const int sc = min(eb - (ilogb(bound) + 1), 1000);
+                scale = ldexp(1.0, sc);
+                unscale = ldexp(1.0, -sc);
+                fix = true;
+            }
+        }
         CsbRound<VM, U> cur;
         cur.load(c, ch, ch1, lane);
-        for (int i = tid; i < R; i += T)
-            s_y[i] = 0.0;
+        for (int i = tid; i < ((FIX && c.vmax) ? CSB_WORDS * R : 2 * R); i += T)
+            s_w[i] = 0u;                               // fixed-point words, or s_y[0, R)
         __syncthreads();
+        const uint32_t lmask = (1u << c.lb) - 1u;
         for (; ch < ch1; ch += U * NW) {
             CsbRound<VM, U> nxt;
             nxt.load(c, ch + U * NW, ch1, lane);
@@ -127,15 +258,35 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
             for (int u = 0; u < U; ++u)
                 g[u] = (cur.w[u] & 0xFFFFu) != CSB_PAD
                            ? op.operand((int64_t)cur.base[u] + (cur.w[u] >> 16), 0, s_scal) : (VV)0;
+            if (FIX && fix) {
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if ((cur.w[u] & 0xFFFFu) != CSB_PAD)
-                    atomicAdd(&s_y[cur.w[u] & 0xFFFFu], (double)cur.a[u] * (double)g[u]);
+                for (int u = 0; u < U; ++u)
+                    if ((cur.w[u] & 0xFFFFu) != CSB_PAD) {
+                        const uint32_t r = cur.w[u] & 0xFFFFu;
+                        const long long v = __double2ll_rn((double)cur.a[u] * (double)g[u] * scale);
+                        red_add_u32(&s_w[r], (uint32_t)(int32_t)(v >> (2 * c.lb)));
+                        red_add_u32(&s_w[R + r], (uint32_t)(v >> c.lb) & lmask);
+                        red_add_u32(&s_w[2 * R + r], (uint32_t)v & lmask);
+                    }
+            } else {
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if ((cur.w[u] & 0xFFFFu) != CSB_PAD)
+                        atomicAdd(&s_y[cur.w[u] & 0xFFFFu], (double)cur.a[u] * (double)g[u]);
+            }
             cur = nxt;
         }
         __syncthreads();
         for (int i = tid; i < R; i += T) {
-            const double acc[1] = {s_y[i]};
+            double acc[1];
+            if (FIX && fix) {
+                // |sum| < 2^62 + 2^52: exact in int64, rounded once to fp64
+                const long long t = (long long)(int32_t)s_w[i] * (1ll << (2 * c.lb)) +
+                                    (long long)s_w[R + i] * (1ll << c.lb) + (long long)s_w[2 * R + i];
+                acc[0] = (double)t * unscale;
+            } else {
+                acc[0] = s_y[i];
+            }
             op.emit((int64_t)(r0 + i), acc, part, s_scal, rv);
         }
         __syncthreads();

@@ -1,10 +1,10 @@
 // Set-up of the column-sorted row segments (csb.cuh), once per matrix pattern.
 //
 // Segments (on the host, from the row pointers): contiguous rows with about equal
-// (entries + rows), at most CSB_RMAX rows each (their sums live in shared memory) and as few
-// as that allows -- the larger a segment, the closer its sorted columns lie -- rounded up to
-// a multiple of the SpMV's grid (one block per SM), so that every block takes the same number
-// of segments.
+// (entries + rows), at most CSB_RMAX rows each (CSB_RMAX_F32 for fp32 values; their sums
+// live in shared memory) and as few as that allows -- the larger a segment, the closer its
+// sorted columns lie -- rounded up to a multiple of the SpMV's grid (one block per SM), so
+// that every block takes the same number of segments.
 //
 // The entries (on the device): every entry gets the key (segment, column, local row), the
 // keys are sorted with the radix sort of radix_sort.cuh, and one warp per segment cuts the
@@ -105,6 +105,8 @@ void free_csb(sla_csr *A)
     cudaFree(A->csb->d_pk);
     cudaFree(A->csb->d_perm);
     cudaFree(A->csb->d_val);
+    cudaFree(A->csb->d_seg_bound);
+    cudaFree(A->csb->d_vmax);
     delete A->csb;
     A->csb = nullptr;
 }
@@ -119,13 +121,14 @@ sla_status ensure_csb(sla_csr *A, cudaStream_t s, const CsbPart **out)
         return fail(SLA_ERR_UNSUPPORTED, "column-sorted segments: CSR matrices with int32 sizes only");
     const int64_t n = A->n;
     const int32_t *rp = A->h_rp.data();
-    // segment boundaries: equal shares of (entries + rows), at most CSB_RMAX rows
+    // segment boundaries: equal shares of (entries + rows), at most RMX rows
     const int64_t total = A->nnz + n;
     const int64_t grid = std::max(1, A->num_sms);
-    const int64_t nseg_min = std::max<int64_t>(1, (n + CSB_RMAX - 1) / CSB_RMAX);
+    const int64_t RMX = A->dtype == SLA_F32 ? CSB_RMAX_F32 : CSB_RMAX;
+    const int64_t nseg_min = std::max<int64_t>(1, (n + RMX - 1) / RMX);
     int64_t nseg = (nseg_min + grid - 1) / grid * grid;
     // segments of the row budget but with a few rows more than an equal share of the
-    // cost would give are still under CSB_RMAX: allow that much slack before splitting
+    // cost would give are still under RMX: allow that much slack before splitting
     nseg = std::min<int64_t>(nseg, std::max<int64_t>(1, n));
     std::vector<int32_t> row0;
     row0.push_back(0);
@@ -142,15 +145,15 @@ sla_status ensure_csb(sla_csr *A, cudaStream_t s, const CsbPart **out)
                     hi = mid;
             }
             int64_t cut = std::max(lo, r + 1);
-            cut = std::min(cut, r + (int64_t)CSB_RMAX);
+            cut = std::min(cut, r + RMX);
             if (cut >= n)
                 break;
             row0.push_back((int32_t)cut);
             r = cut;
         }
-        // the last segment may still exceed CSB_RMAX rows: split it
-        while (n - row0.back() > CSB_RMAX)
-            row0.push_back(row0.back() + CSB_RMAX);
+        // the last segment may still exceed RMX rows: split it
+        while (n - row0.back() > RMX)
+            row0.push_back(row0.back() + (int32_t)RMX);
         row0.push_back((int32_t)n);
     }
     nseg = (int64_t)row0.size() - 1;
@@ -207,6 +210,14 @@ sla_status ensure_csb(sla_csr *A, cudaStream_t s, const CsbPart **out)
     if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_pk, sizeof(uint32_t) * 32 * nc);
     if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_perm, sizeof(int32_t) * 32 * nc);
     if (e == cudaSuccess) e = cudaMalloc(&cp->d_val, vb * 32 * nc);
+    // fixed-point row sums: per-segment bounds (with the values), operand maxima, low-word
+    // bits such that the longest row's low words cannot carry out of 32 bits
+    cp->vmax_n = std::max(1, A->num_sms);
+    cp->lb = std::max(1, std::min(20, 32 - bits_for((uint64_t)std::max<int64_t>(A->max_row_len, 0))));
+    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_seg_bound, sizeof(double) * (size_t)std::max<int64_t>(nseg, 1));
+    if (e == cudaSuccess) e = cudaMalloc((void **)&cp->d_vmax, sizeof(float) * (size_t)cp->vmax_n);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(cp->d_seg_bound, 0, sizeof(double) * (size_t)std::max<int64_t>(nseg, 1), s);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(cp->d_seg_ch0, ch0.data(), sizeof(int32_t) * ch0.size(), cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && nch > 0) {
@@ -237,10 +248,15 @@ sla_status launch_csb_values(const sla_csr *A, cudaStream_t s)
         return SLA_SUCCESS;
     const int64_t slots = cp->n_chunks * 32;
     const int grid = (int)std::min<int64_t>((slots + 255) / 256, (int64_t)A->num_sms * 16);
-    if (A->dtype == SLA_F32)
+    if (A->dtype == SLA_F32) {
         k_csb_values<float><<<grid, 256, 0, s>>>(slots, cp->d_perm, (const float *)A->val, (float *)cp->d_val);
-    else
+        k_csb_bounds<float><<<cp->n_seg, 256, 0, s>>>(cp->n_seg, cp->d_seg_row0, A->rp, (const float *)A->val,
+                                                      cp->d_seg_bound);
+    } else {
         k_csb_values<double><<<grid, 256, 0, s>>>(slots, cp->d_perm, (const double *)A->val, (double *)cp->d_val);
+        k_csb_bounds<double><<<cp->n_seg, 256, 0, s>>>(cp->n_seg, cp->d_seg_row0, A->rp, (const double *)A->val,
+                                                       cp->d_seg_bound);
+    }
     SLA_CUDA_TRY(cudaGetLastError());
     const_cast<sla_csr *>(A)->csb_vals_current = 1;
     return SLA_SUCCESS;

@@ -423,7 +423,13 @@ struct TileLaunch {
                 cv.val = (const VM *)cp->d_val;
                 cv.n_seg = cp->n_seg;
                 cv.rmax = std::max(cp->rmax, 1);
-                csb_smem = (size_t)std::max(cp->rmax, 1) * sizeof(double);
+                cv.seg_bound = cp->d_seg_bound;
+                // exact fixed-point row sums for fp32 values and vectors
+                cv.vmax = (sizeof(VM) == 4 && sizeof(typename Op::VV) == 4) ? cp->d_vmax : nullptr;
+                cv.vmax_n = cp->vmax_n;
+                cv.lb = cp->lb;
+                // fp64 row sums, or three 32-bit fixed-point words per row
+                csb_smem = (size_t)std::max(cp->rmax, 1) * (cv.vmax ? 4 * CSB_WORDS : sizeof(double));
                 auto kern = k_csb<VM, Op>;
                 SLA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csb_smem));
                 SLA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, CsbCfg::T, csb_smem));
@@ -466,8 +472,12 @@ struct TileLaunch {
     {
         if (maxl == -3) {
             if constexpr (K == 1 && Op::NG == 1)
-                if (cv.n_seg > 0)
+                if (cv.n_seg > 0) {
+                    if (cv.vmax)    // max |v_j| of the gathered vector, for the fixed-point scale
+                        k_vec_absmax<typename Op::VV><<<cv.vmax_n, CSB_VMAX_T, 0, s>>>(
+                            m.n, op.gvec(0), const_cast<float *>(cv.vmax), st);
                     k_csb<VM, Op><<<grid, CsbCfg::T, csb_smem, s>>>(cv, op, part, st);
+                }
             return;
         }
         if (maxl < 0 ? gv.n_tasks == 0 : m.n_tiles == 0)

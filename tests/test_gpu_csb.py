@@ -102,3 +102,67 @@ def test_static_values_spmv(ora, cfg, size):
     sla.sla_csr_values_changed(As)
     ys2 = host(sla.sla_spmv(As, dev(x)))
     assert rel(ys2, -0.5 * ref) <= SPMV_TOL[w.dtype]
+
+
+def _fx_slack(A, x):
+    """2^-50 of max_i sum_j |a_ij| x max_j |x_j|: the fixed-point sums round every term once,
+    to 2^-63 of their segment's bound (largest row sum of |a_ij| times max |x_j|), so a row
+    of m <= 8192 terms is off by at most 2^-50 of it."""
+    rows = np.add.reduceat(np.abs(A.val.astype(np.float64)), A.row_ptr[:-1]) * (np.diff(A.row_ptr) > 0)
+    return 2.0 ** -50 * float(rows.max()) * float(np.max(np.abs(x.astype(np.float64))))
+
+
+def test_fixed_point_sums_reproducible_and_rounded(ora):
+    """fp32 products of the segment engine sum exact integers on a per-segment scale: two
+    launches give identical bits, and each row is the fp64 row sum rounded to fp32 up to an
+    error far below the fp32 rounding of a typical row."""
+    import differentiable_sparse_linear_b200 as sla
+    w = W.workload(5, "small")
+    A = w.A
+    As = sla.sla_csr_create(dev(A.row_ptr), dev(A.col), dev(A.val), static_values=True)
+    x = W.rhs_normal(96, A.n_rows, np.float32)
+    y1 = host(sla.sla_spmv(As, dev(x)))
+    y2 = host(sla.sla_spmv(As, dev(x)))
+    assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+    ref = ora.spmv(A, x)
+    ulp = np.spacing(np.abs(ref.astype(np.float32))).astype(np.float64)
+    err = np.abs(y1.astype(np.float64) - ref)
+    assert np.all(err <= 0.5 * ulp + _fx_slack(A, x))
+
+
+def test_fixed_point_wide_range(ora):
+    """Operands spanning the fp32 range (1e-30 .. 1e30): no term or word overflows, every
+    row stays finite, and rows are exact to 2^-50 of the largest |A||x| scale."""
+    import differentiable_sparse_linear_b200 as sla
+    w = W.workload(5, "tiny")
+    A = w.A
+    As = sla.sla_csr_create(dev(A.row_ptr), dev(A.col), dev(A.val), static_values=True)
+    rng = np.random.default_rng(97)
+    x = (rng.standard_normal(A.n_rows) * 10.0 ** rng.uniform(-30, 30, A.n_rows)).astype(np.float32)
+    y = host(sla.sla_spmv(As, dev(x))).astype(np.float64)
+    ref = ora.spmv(A, x)
+    ulp = np.spacing(np.abs(ref.astype(np.float32))).astype(np.float64)
+    assert np.all(np.isfinite(y))
+    assert np.all(np.abs(y - ref) <= 0.5 * ulp + _fx_slack(A, x))
+
+
+@pytest.mark.parametrize("bad", [np.nan, np.inf])
+def test_nonfinite_operand_reaches_the_result(ora, bad):
+    """A NaN or Inf in the operand makes the fixed-point bound unusable: the product falls
+    back to fp64 sums, so the rows that read it are not finite and the others are exact."""
+    import differentiable_sparse_linear_b200 as sla
+    w = W.workload(5, "tiny")
+    A = w.A
+    As = sla.sla_csr_create(dev(A.row_ptr), dev(A.col), dev(A.val), static_values=True)
+    x = W.rhs_normal(98, A.n_rows, np.float32)
+    j = A.n_rows // 3
+    x[j] = bad
+    y = host(sla.sla_spmv(As, dev(x)))
+    reads = np.zeros(A.n_rows, bool)
+    rows = np.repeat(np.arange(A.n_rows), np.diff(A.row_ptr))
+    reads[rows[A.col == j]] = True
+    assert reads.any() and not np.isfinite(y[reads]).any()
+    xs = x.copy()
+    xs[j] = 0.0
+    ref = ora.spmv(A, xs)
+    assert rel(y[~reads], ref[~reads]) <= 1e-6
