@@ -12,7 +12,7 @@
 //
 // Storage (CsbPart): per segment its first row and first chunk; entries in chunks of 32
 // (one warp load), per chunk the smallest column `base`, per entry a 32-bit word
-// (column - base) << 16 | local row, padding marked by local row 0xFFFF, and the entry's
+// (column - base) << 16 | local row, padding marked by a flag bit (csb_pad_word), and the entry's
 // value, gathered from the caller's CSR values by `perm` at the start of every solve (the
 // values may change between solves; the pattern may not).  8 bytes per entry plus 4 per 32
 // entries, as CSR's value + column index.
@@ -43,13 +43,24 @@
 namespace sla {
 
 constexpr int CSB_RMAX = 16384;                // rows per segment with fp64 sums (8 bytes a row)
+static_assert(CSB_RMAX <= 16384, "local rows must fit 14 bits (the pad flag is bit 15)");
 // rows per segment with fp32 values (three 4-byte fixed-point words a row): 128 KB of sums
 // leave the other half of the SM's 256 KB of L1/shared memory to cache the gathered
 // operand lines (with 16384 rows, 192 KB of sums left 60 KB of L1 and the products ran 7 %
 // slower on the power-law 4M system despite the denser segments)
 constexpr int CSB_RMAX_F32 = 10922;
 constexpr int CSB_WORDS = 3;
-constexpr uint32_t CSB_PAD = 0xFFFFu;
+// A padding slot (past a chunk's last entry) has value 0, column offset 0, local row = its
+// lane in a segment of at least 32 rows (else row 0), and the flag CSB_PADF: it gathers a
+// valid operand and, with the fixed-point sums (finite operands only), adds 0 to a row of
+// its own bank without a test; the fp64 sums skip it by the flag (0 x Inf would be NaN).
+// Local rows are below 2^14 (CSB_RMAX), so the flag bit is free.
+constexpr uint32_t CSB_PADF = 0x8000u;
+constexpr uint32_t CSB_ROWM = 0x3FFFu;
+__host__ __device__ inline uint32_t csb_pad_word(int lane, int seg_rows)
+{
+    return (seg_rows >= 32 ? (uint32_t)lane : 0u) | CSB_PADF;
+}
 
 template <typename VM>
 struct CsbView {
@@ -151,7 +162,8 @@ struct CsbRound {
     int base[U];
     uint32_t w[U];
     VM a[U];
-    __device__ __forceinline__ void load(const CsbView<VM> &c, int ch, int ch1, int lane)
+    // chunks past the segment's last one read as padding (`pad` = csb_pad_word)
+    __device__ __forceinline__ void load(const CsbView<VM> &c, int ch, int ch1, int lane, uint32_t pad)
     {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -162,7 +174,7 @@ struct CsbRound {
                 a[u] = __ldg(&c.val[(int64_t)cc * 32 + lane]);
             } else {
                 base[u] = 0;
-                w[u] = CSB_PAD;
+                w[u] = pad;
                 a[u] = (VM)0;
             }
         }
@@ -244,37 +256,40 @@ k_csb(const CsbView<VM> c, const Op op, double *partials, PcgState *st)
                 fix = true;
             }
         }
-        CsbRound<VM, U> cur;
-        cur.load(c, ch, ch1, lane);
+        const uint32_t pad = csb_pad_word(lane, R);
         for (int i = tid; i < ((FIX && c.vmax) ? CSB_WORDS * R : 2 * R); i += T)
             s_w[i] = 0u;                               // fixed-point words, or s_y[0, R)
-        __syncthreads();
         const uint32_t lmask = (1u << c.lb) - 1u;
-        for (; ch < ch1; ch += U * NW) {
-            CsbRound<VM, U> nxt;
-            nxt.load(c, ch + U * NW, ch1, lane);
+        // one round: gather the U chunks' operands, then add their products
+        auto round = [&](const CsbRound<VM, U> &cr) {
             VV g[U];
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                g[u] = (cur.w[u] & 0xFFFFu) != CSB_PAD
-                           ? op.operand((int64_t)cur.base[u] + (cur.w[u] >> 16), 0, s_scal) : (VV)0;
-            if (FIX && fix) {
+                g[u] = op.operand((int64_t)cr.base[u] + (cr.w[u] >> 16), 0, s_scal);
 #pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if ((cur.w[u] & 0xFFFFu) != CSB_PAD) {
-                        const uint32_t r = cur.w[u] & 0xFFFFu;
-                        const long long v = __double2ll_rn((double)cur.a[u] * (double)g[u] * scale);
-                        red_add_u32(&s_w[r], (uint32_t)(int32_t)(v >> (2 * c.lb)));
-                        red_add_u32(&s_w[R + r], (uint32_t)(v >> c.lb) & lmask);
-                        red_add_u32(&s_w[2 * R + r], (uint32_t)v & lmask);
-                    }
-            } else {
-#pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if ((cur.w[u] & 0xFFFFu) != CSB_PAD)
-                        atomicAdd(&s_y[cur.w[u] & 0xFFFFu], (double)cur.a[u] * (double)g[u]);
+            for (int u = 0; u < U; ++u) {
+                const uint32_t r = cr.w[u] & CSB_ROWM;
+                if (FIX && fix) {
+                    const long long v = __double2ll_rn((double)cr.a[u] * (double)g[u] * scale);
+                    red_add_u32(&s_w[r], (uint32_t)(int32_t)(v >> (2 * c.lb)));
+                    red_add_u32(&s_w[R + r], (uint32_t)(v >> c.lb) & lmask);
+                    red_add_u32(&s_w[2 * R + r], (uint32_t)v & lmask);
+                } else if (!(cr.w[u] & CSB_PADF)) {
+                    atomicAdd(&s_y[r], (double)cr.a[u] * (double)g[u]);
+                }
             }
-            cur = nxt;
+        };
+        // two round buffers in turn: the next round's loads go out before this round's work
+        CsbRound<VM, U> ra, rb;
+        ra.load(c, ch, ch1, lane, pad);
+        __syncthreads();
+        for (; ch < ch1; ch += 2 * U * NW) {
+            rb.load(c, ch + U * NW, ch1, lane, pad);
+            round(ra);
+            if (ch + U * NW >= ch1)
+                break;
+            ra.load(c, ch + 2 * U * NW, ch1, lane, pad);
+            round(rb);
         }
         __syncthreads();
         for (int i = tid; i < R; i += T) {

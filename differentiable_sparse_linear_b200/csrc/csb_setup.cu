@@ -69,6 +69,7 @@ __global__ void k_csb_chunks(int nseg, const int32_t *seg_row0, const int32_t *r
     const uint64_t colmask = (cb >= 32) ? 0xFFFFFFFFull : ((1ull << cb) - 1ull);
     for (int64_t sg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; sg < nseg; sg += warps) {
         const int64_t e0 = rp[seg_row0[sg]], e1 = rp[seg_row0[sg + 1]];
+        const int r_seg = seg_row0[sg + 1] - seg_row0[sg];
         int64_t ch = WRITE ? (int64_t)ch0[sg] : 0;
         for (int64_t pos = e0; pos < e1;) {
             const int64_t t = pos + lane;
@@ -80,7 +81,7 @@ __global__ void k_csb_chunks(int nseg, const int32_t *seg_row0, const int32_t *r
             const int take = __popc(__ballot_sync(0xffffffffu, ok));
             if (WRITE) {
                 const uint32_t lr = (uint32_t)(kk & ((1u << CSB_RB) - 1u));
-                pk[ch * 32 + lane] = lane < take ? ((col - base) << 16) | lr : CSB_PAD;
+                pk[ch * 32 + lane] = lane < take ? ((col - base) << 16) | lr : csb_pad_word(lane, r_seg);
                 perm[ch * 32 + lane] = lane < take ? val[t] : -1;
                 if (lane == 0)
                     cbase[ch] = (int32_t)base;
