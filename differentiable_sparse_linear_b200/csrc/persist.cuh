@@ -47,11 +47,13 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
 
 template <typename VM, typename VV, int K, int MAXL>
 struct Persist {
-    static constexpr int TB = 512;    // threads per block
+    // threads per block: one 1024-thread block per SM for one right-hand side (half the grid
+    // barrier's arrivals of two 512-thread blocks: 35.7 against 37.7 us per SPAI iteration on
+    // the 1024^2 problem), 512 for more (their lanes need more than 64 registers)
+    static constexpr int TB = K == 1 ? 1024 : 512;
     static constexpr int NR = 2 * K;
-    // blocks per SM the register budget is cut for (two: 32 warps per SM) where the lane
-    // code fits 64 registers without spills
-    static constexpr int MINB = (K == 1 && MAXL == 8) ? 2 : 1;
+    // blocks per SM the register budget is cut for
+    static constexpr int MINB = 1;
     // slices per warp round (their loads in flight together): two where that fits the registers
     static constexpr int RS = (K == 1 || (K == 2 && sizeof(VV) == 4)) ? 2 : 1;
     // wide rows (K >= 4 right-hand sides): p_new is formed in a phase of its own, so Q
