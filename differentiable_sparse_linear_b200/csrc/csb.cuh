@@ -36,6 +36,8 @@
 
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "sla_internal.cuh"
 #include "pcg_ops.cuh"
 #include "tile_engine.cuh"
@@ -77,10 +79,10 @@ struct CsbView {
     int lb;                                    // bits of the fixed-point low word
 };
 
-constexpr int CSB_VMAX_T = 512;                // threads of k_vec_absmax
+constexpr int CSB_VMAX_T = 1024;               // threads of k_vec_absmax
 
 // Per-block max |v_i| over v[0, n) into out[blockIdx.x]; +Inf if the block saw a value that
-// is not finite.
+// is not finite.  16-byte loads where v is 16-byte aligned, four in flight per thread.
 template <typename V>
 __global__ void __launch_bounds__(CSB_VMAX_T) k_vec_absmax(int64_t n, const V *v, float *out, const PcgState *st)
 {
@@ -89,12 +91,39 @@ __global__ void __launch_bounds__(CSB_VMAX_T) k_vec_absmax(int64_t n, const V *v
         return;
     float m = 0.f;
     bool bad = false;
-    const int64_t stride = (int64_t)gridDim.x * CSB_VMAX_T;
-    for (int64_t i = (int64_t)blockIdx.x * CSB_VMAX_T + threadIdx.x; i < n; i += stride) {
-        const float a = fabsf((float)v[i]);
+    auto take = [&](V x) {
+        const float a = fabsf((float)x);
         bad |= !(a <= 3.0e38f);
         m = fmaxf(m, a);
+    };
+    const int64_t tid = (int64_t)blockIdx.x * CSB_VMAX_T + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * CSB_VMAX_T;
+    constexpr int VW = 16 / sizeof(V);             // values per 16-byte load
+    int64_t done = 0;
+    if (((uintptr_t)v & 15) == 0) {
+        using L = typename std::conditional<sizeof(V) == 4, float4, double2>::type;
+        const L *v4 = reinterpret_cast<const L *>(v);
+        const int64_t n4 = n / VW;
+        constexpr int IL = 4;
+        for (int64_t i = tid; i < n4; i += stride * IL) {
+            L t[IL];
+#pragma unroll
+            for (int k = 0; k < IL; ++k)
+                if (i + k * stride < n4)
+                    t[k] = __ldg(&v4[i + k * stride]);
+#pragma unroll
+            for (int k = 0; k < IL; ++k)
+                if (i + k * stride < n4) {
+                    const V *e = reinterpret_cast<const V *>(&t[k]);
+#pragma unroll
+                    for (int j = 0; j < VW; ++j)
+                        take(e[j]);
+                }
+        }
+        done = n4 * VW;
     }
+    for (int64_t i = done + tid; i < n; i += stride)
+        take(v[i]);
     if (bad)
         m = __int_as_float(0x7f800000);
 #pragma unroll
@@ -112,30 +141,53 @@ __global__ void __launch_bounds__(CSB_VMAX_T) k_vec_absmax(int64_t n, const V *v
 }
 
 // Per segment the largest row sum of |a_ij| (fp64), from the CSR values: a block per
-// segment, a warp per row.
+// segment, a warp per row group of four rows summed together (four rows' loads in flight).
+constexpr int CSB_BND_T = 1024;
 template <typename VM>
-__global__ void __launch_bounds__(256) k_csb_bounds(int n_seg, const int32_t *seg_row0, const int32_t *rp,
-                                                    const VM *val, double *bound)
+__global__ void __launch_bounds__(CSB_BND_T) k_csb_bounds(int n_seg, const int32_t *seg_row0, const int32_t *rp,
+                                                          const VM *val, double *bound)
 {
-    __shared__ double s_w[8];
+    constexpr int NW = CSB_BND_T / 32, RU = 4;
+    __shared__ double s_w[NW];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int sg = blockIdx.x; sg < n_seg; sg += gridDim.x) {
+        const int r0 = seg_row0[sg], r1 = seg_row0[sg + 1];
         double wm = 0.0;
-        for (int r = seg_row0[sg] + warp; r < seg_row0[sg + 1]; r += 8) {
-            double a = 0.0;
-            for (int k = rp[r] + lane; k < rp[r + 1]; k += 32)
-                a += fabs((double)val[k]);
+        for (int rb = r0 + warp * RU; rb < r1; rb += NW * RU) {
+            int k[RU], k1[RU];
+            double a[RU];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                a += __shfl_xor_sync(0xffffffffu, a, off);
-            wm = fmax(wm, a);
+            for (int u = 0; u < RU; ++u) {
+                const int r = rb + u;
+                k[u] = r < r1 ? rp[r] + lane : 0;
+                k1[u] = r < r1 ? rp[r + 1] : 0;
+                a[u] = 0.0;
+            }
+            bool more = true;
+            while (more) {
+                more = false;
+#pragma unroll
+                for (int u = 0; u < RU; ++u)
+                    if (k[u] < k1[u]) {
+                        a[u] += fabs((double)val[k[u]]);
+                        k[u] += 32;
+                        more |= k[u] < k1[u];
+                    }
+            }
+#pragma unroll
+            for (int u = 0; u < RU; ++u) {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    a[u] += __shfl_xor_sync(0xffffffffu, a[u], off);
+                wm = fmax(wm, a[u]);
+            }
         }
         if (lane == 0)
             s_w[warp] = wm;
         __syncthreads();
         if (threadIdx.x == 0) {
             double t = 0.0;
-            for (int w = 0; w < 8; ++w)
+            for (int w = 0; w < NW; ++w)
                 t = fmax(t, s_w[w]);
             bound[sg] = t;
         }
@@ -143,8 +195,9 @@ __global__ void __launch_bounds__(256) k_csb_bounds(int n_seg, const int32_t *se
     }
 }
 
-// 4 chunks per warp per round with the next round prefetched measured the same as 2, 6, or
-// 8 without the prefetch (q = A p on the 4M system: 0.773 / 0.773 / 0.786 / 0.783 ms).
+// 4 chunks per warp per round, the next round's loads in flight during this one's adds:
+// 2 or 8 measured slower with the fixed-point sums (q = A p on the 4M system: 0.644 and
+// 0.657 ms against 0.538).
 struct CsbCfg {
     static constexpr int T = 1024;             // threads per block (one block per SM)
     static constexpr int U = 4;                // chunks per warp per round

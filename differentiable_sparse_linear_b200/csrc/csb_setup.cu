@@ -251,11 +251,11 @@ sla_status launch_csb_values(const sla_csr *A, cudaStream_t s)
     const int grid = (int)std::min<int64_t>((slots + 255) / 256, (int64_t)A->num_sms * 16);
     if (A->dtype == SLA_F32) {
         k_csb_values<float><<<grid, 256, 0, s>>>(slots, cp->d_perm, (const float *)A->val, (float *)cp->d_val);
-        k_csb_bounds<float><<<cp->n_seg, 256, 0, s>>>(cp->n_seg, cp->d_seg_row0, A->rp, (const float *)A->val,
+        k_csb_bounds<float><<<cp->n_seg, CSB_BND_T, 0, s>>>(cp->n_seg, cp->d_seg_row0, A->rp, (const float *)A->val,
                                                       cp->d_seg_bound);
     } else {
         k_csb_values<double><<<grid, 256, 0, s>>>(slots, cp->d_perm, (const double *)A->val, (double *)cp->d_val);
-        k_csb_bounds<double><<<cp->n_seg, 256, 0, s>>>(cp->n_seg, cp->d_seg_row0, A->rp, (const double *)A->val,
+        k_csb_bounds<double><<<cp->n_seg, CSB_BND_T, 0, s>>>(cp->n_seg, cp->d_seg_row0, A->rp, (const double *)A->val,
                                                        cp->d_seg_bound);
     }
     SLA_CUDA_TRY(cudaGetLastError());
