@@ -37,7 +37,14 @@
  *   - Errors: every call returns an sla_status.  Negative values are errors and leave
  *     outputs unspecified; sla_last_error() gives a thread-local message.  Solver outcomes
  *     SLA_NOT_CONVERGED and SLA_BREAKDOWN are positive: the outputs hold the last iterate.
- *   - Handles are not thread-safe: one host thread at a time per handle.
+ *   - Handles are not thread-safe: one host thread at a time per handle.  Work queued on
+ *     one handle to different streams must not overlap in time (order the streams): the
+ *     handle's layout copies and scratch (value copies, per-segment bounds, operand maxima
+ *     of the column-sorted products) are shared by its calls.
+ *   - Products of fp32 values with fp32 vectors on the column-sorted segments (long-row
+ *     single-RHS solves, and sla_spmv on SLA_STATIC_VALUES handles) sum each row exactly in
+ *     fixed point after rounding every term to 2^-63 of its segment's bound (largest row sum
+ *     of |a_ij| times max |v_j|): results are bit-reproducible run to run.
  */
 #ifndef SLA_H
 #define SLA_H
