@@ -406,14 +406,15 @@ def run_ours(args):
             if record:
                 fwd_events[-1][1].record()
                 if not is_list:     # one iteration advances every right-hand side
-                    fwd_iters.append(max(i.iters for i in inf))
+                    fwd_iters.append(int(inf.iters.max()))
             lam, g, ainf = sla.sla_pcg_adjoint_batched(Ad, M, x, wv, rtol=w.tol, engine=args.engine,
                                                        dLdB=lam_buf, dLdA=g_buf)
-            engines_seen.update(i.engine for i in inf + ainf)
+            # the per-system results are read as arrays (PcgInfoList), not system by system
+            engines_seen.update(inf.engines | ainf.engines)
             if is_list:
-                return sum(i.iters for i in inf) + sum(i.iters for i in ainf), 2, x, lam
-            it = max(i.iters for i in inf), max(i.iters for i in ainf)
-            return (sum(i.iters for i in inf) + sum(i.iters for i in ainf),
+                return int(inf.iters.sum()) + int(ainf.iters.sum()), 2, x, lam
+            it = int(inf.iters.max()), int(ainf.iters.max())
+            return (int(inf.iters.sum()) + int(ainf.iters.sum()),
                     launches(it[0], inf[0].engine) + launches(it[1], ainf[0].engine) + 1, x, lam)
         x, inf = sla.sla_pcg_solve(Ad, M, bv, x_out, rtol=w.tol, engine=args.engine)
         if record:
@@ -592,7 +593,7 @@ def run_ours(args):
             if r >= 1:
                 tot += sla.sla_list_kernel_ms(Ad)
         launch_ms = tot / reps
-        its = np.array([i.iters for i in infos], dtype=np.int64)
+        its = np.asarray(infos.iters, dtype=np.int64)
         launch_bytes = int((per_iter * its).sum())
         ach = launch_bytes / (launch_ms * 1e6)
         roofline = {"bound": "hbm", "kernel": "k_list_pcg", "achieved": ach, "peak": peak, "unit": "GB/s",

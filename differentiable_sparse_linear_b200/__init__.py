@@ -12,10 +12,12 @@ dL/db = lambda, dL/dA_ij = -lambda_i x_j on A's pattern; only x is saved for bac
 """
 from __future__ import annotations
 
+import collections.abc as _abc
 import ctypes as C
 from dataclasses import dataclass
 from typing import Optional, Sequence
 
+import numpy as np
 import torch
 
 from . import _lib
@@ -24,7 +26,7 @@ from ._lib import (SLA_BREAKDOWN, SLA_ERR_CUDA, SLA_ERR_INVALID_ARG, SLA_ERR_INV
                    SLA_SPD, SLA_STATIC_VALUES, SLA_SUCCESS, SLA_VALIDATE)
 
 __all__ = [
-    "SlaError", "Matrix", "Preconditioner", "PcgInfo", "lib",
+    "SlaError", "Matrix", "Preconditioner", "PcgInfo", "PcgInfoList", "lib",
     "sla_version", "sla_csr_create", "sla_csr_values_changed", "sla_bsr_create", "sla_csr_create_list", "sla_spmv", "sla_spmv_multi",
     "sla_precond_jacobi", "sla_precond_spai", "sla_pcg_solve", "sla_pcg_adjoint",
     "sla_pcg_solve_batched", "sla_pcg_adjoint_batched", "sla_pattern_grad",
@@ -95,9 +97,47 @@ class PcgInfo:
         return self.status == SLA_SUCCESS
 
 
-def _infos(arr) -> list[PcgInfo]:
-    return [PcgInfo(int(a.iters), float(a.relres), int(a.status), _ENGINE_NAMES.get(int(a.engine), "?"))
-            for a in arr]
+class PcgInfoList(_abc.Sequence):
+    """Per-system (or per-right-hand-side) results of a batched solve: a sequence of PcgInfo,
+    each made when it is read, over the arrays `iters`, `relres`, `status` and `engine_codes`
+    copied once from the library's result structs (a list of thousands of systems reads them
+    in bulk, not one Python object per system)."""
+
+    __slots__ = ("iters", "relres", "status", "engine_codes")
+
+    def __init__(self, arr):
+        a = np.ctypeslib.as_array(arr)
+        self.iters = a["iters"].astype(np.int64)
+        self.relres = a["relres"].astype(np.float64)
+        self.status = a["status"].astype(np.int32)
+        self.engine_codes = a["engine"].astype(np.int32)
+
+    def __len__(self) -> int:
+        return int(self.iters.shape[0])
+
+    def __getitem__(self, i):
+        if isinstance(i, slice):
+            return [self[j] for j in range(*i.indices(len(self)))]
+        return PcgInfo(int(self.iters[i]), float(self.relres[i]), int(self.status[i]),
+                       _ENGINE_NAMES.get(int(self.engine_codes[i]), "?"))
+
+    def __add__(self, other):
+        return list(self) + list(other)
+
+    def __radd__(self, other):
+        return list(other) + list(self)
+
+    @property
+    def engines(self) -> set:
+        return {_ENGINE_NAMES.get(int(e), "?") for e in np.unique(self.engine_codes)}
+
+
+def _infos(arr) -> PcgInfoList:
+    return PcgInfoList(arr)
+
+
+def _info1(a) -> PcgInfo:
+    return PcgInfo(int(a.iters), float(a.relres), int(a.status), _ENGINE_NAMES.get(int(a.engine), "?"))
 
 
 def _opts(rtol: float, maxit: int, vector_f64: bool = False, engine: str = "auto") -> _lib.sla_pcg_opts:
@@ -277,7 +317,7 @@ def sla_pcg_solve(A: Matrix, M: Optional[Preconditioner], b: torch.Tensor,
     opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_solve(A.handle, _mh(M), _ptr(b), _ptr(x), C.byref(opts), C.byref(info),
                                _stream(stream)), "sla_pcg_solve")
-    return x, _infos([info])[0]
+    return x, _info1(info)
 
 
 def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLdx: torch.Tensor, *,
@@ -295,12 +335,12 @@ def sla_pcg_adjoint(A: Matrix, M: Optional[Preconditioner], x: torch.Tensor, dLd
     opts = _opts(rtol, maxit, vector_f64, engine)
     _check(lib().sla_pcg_adjoint(A.handle, _mh(M), _ptr(x), _ptr(dLdx), _ptr(dLdb), _ptr(dLdA),
                                  C.byref(opts), C.byref(info), _stream(stream)), "sla_pcg_adjoint")
-    return dLdb, dLdA, _infos([info])[0]
+    return dLdb, dLdA, _info1(info)
 
 
 def sla_pcg_solve_batched(A: Matrix, M: Optional[Preconditioner], B: torch.Tensor,
                           X: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
-                          vector_f64: bool = False, engine: str = "auto", stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
+                          vector_f64: bool = False, engine: str = "auto", stream=None) -> tuple[torch.Tensor, PcgInfoList]:
     """Shared matrix: B is [n, nrhs].  List handle: B is the concatenated [n_total] vector."""
     _check_vec(A, B, vector_f64)
     nrhs = 1 if (B.dim() == 1 or A.batch > 1) else B.shape[1]
@@ -322,7 +362,7 @@ def sla_list_kernel_ms(A: Matrix) -> float:
 
 def sla_pcg_solve_batched_noalloc(A: Matrix, M: Optional[Preconditioner], B: torch.Tensor,
                                   X: Optional[torch.Tensor] = None, *, rtol: float = 0.0, maxit: int = 0,
-                                  stream=None) -> tuple[torch.Tensor, list[PcgInfo]]:
+                                  stream=None) -> tuple[torch.Tensor, PcgInfoList]:
     """List-handle solve that allocates no device memory inside the call (X must be given
     by callers that cannot allocate either; here it is created when omitted)."""
     X = torch.empty_like(B) if X is None else X
@@ -399,7 +439,7 @@ def sla_nonlinear_adjoint(J: Matrix, M: Optional[Preconditioner], A: Optional[Ma
     _check(lib().sla_nonlinear_adjoint(J.handle, _mh(M), None if A is None else A.handle, _ptr(u), _ptr(dLdu),
                                        _ptr(lam), _ptr(dLdA), C.byref(opts), C.byref(info), _stream(stream)),
            "sla_nonlinear_adjoint")
-    return lam, dLdA, _infos([info])[0]
+    return lam, dLdA, _info1(info)
 
 
 def sla_vec_dot(x: torch.Tensor, y: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
