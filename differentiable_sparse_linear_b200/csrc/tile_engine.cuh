@@ -236,7 +236,8 @@ __device__ __forceinline__ void span_tail(const Span<S> &sp, int64_t e, E *smem,
 }
 
 // ------------------------------------------------------------------ the load-and-gather tile kernel
-// Same tiles, merge-path split and fused epilogues as k_tile, without a producer: every
+// Fixed-size tiles of entries with a merge-path split over their rows and the fused
+// epilogues, without a producer warp: every
 // thread loads entries tid, tid + T, ... of the tile (coalesced) and gathers each operand
 // as soon as its column is in a register, so a thread has all of its matrix loads and then
 // all of its gathers in flight; the products go to shared memory for the merge-path sums.

@@ -334,10 +334,9 @@ SLA_API sla_status sla_vec_scatter_add(int32_t dtype, int64_t n, const int32_t *
  * fixed array in the library's own device memory (1.5 MiB, held by every GPU that loads
  * the library until the process exits), and at most 65536 systems are accepted per call
  * (SLA_ERR_INVALID_ARG beyond that).  Every call looks up that array's device address in
- * the current context (cudaGetSymbolAddress, a host-side lookup; on a device's first call it
- * can load the library's device code, so make that first call before any stream capture
- * begins), fills this call's slots with status -1 and synchronises `stream` to read the
- * results back into h_info.  All calls on a device share the array: calls that overlap on
+ * the current context (cudaGetSymbolAddress, a host-side lookup), fills this call's slots
+ * with status -1 and synchronises `stream` to read the results back into h_info, so the
+ * call cannot be captured into a CUDA graph.  All calls on a device share the array: calls that overlap on
  * the GPU race on it.  The matrix and preconditioner handles
  * are created beforehand with the usual calls.  There is no counterpart on the pages this
  * library follows: it is an interface variant, not a different method. */
