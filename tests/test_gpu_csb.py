@@ -166,3 +166,30 @@ def test_nonfinite_operand_reaches_the_result(ora, bad):
     xs[j] = 0.0
     ref = ora.spmv(A, xs)
     assert rel(y[~reads], ref[~reads]) <= 1e-6
+
+
+@pytest.mark.parametrize("dtype", [np.float32, np.float64])
+def test_csb_small_dense_solve(ora, dtype):
+    """A dense 20 x 20 SPD system: every row is long, so the solve runs on the column-sorted
+    copy with one segment per row group smaller than a warp (padding rows fall back to row
+    0); lockstep iterates and the converged solve against the oracle."""
+    import differentiable_sparse_linear_b200 as sla
+    rng = np.random.default_rng(99)
+    n = 20
+    B = rng.standard_normal((n, n))
+    D = B @ B.T + n * np.eye(n)
+    rp = np.arange(0, n * n + 1, n, dtype=np.int32)
+    col = np.tile(np.arange(n, dtype=np.int32), n)
+    A = W.CSR(n, n, rp, col, D.ravel().astype(dtype))
+    Ad = matrix(A)
+    M = sla.sla_precond_jacobi(Ad)
+    b = rng.standard_normal(n).astype(dtype)
+    tight = 1e-11 if dtype == np.float64 else 1e-5
+    for k in (1, 3):
+        x, info = sla.sla_pcg_solve(Ad, M, dev(b), rtol=1e-300, maxit=k, engine="graph")
+        ref = ora.pcg(A, b, precond="jacobi", fixed_iters=k)
+        assert info.iters == k and rel(host(x), ref.x) <= tight, (k, rel(host(x), ref.x))
+    tol = 1e-10 if dtype == np.float64 else 1e-6
+    x, info = sla.sla_pcg_solve(Ad, M, dev(b), rtol=tol, engine="graph")
+    ref = ora.pcg(A, b, precond="jacobi", tol=tol)
+    assert info.status == 0 and rel(host(x), ref.x) <= SOL_TOL[dtype]

@@ -68,6 +68,9 @@ def _special(kind, dtype):
     elif kind == "dense_row_block":
         n = 700
         lens = np.full(n, 700)
+    elif kind == "dense_small":       # fewer rows than a warp's lanes, all long
+        n = 20
+        lens = np.full(n, 20)
     rp = np.zeros(n + 1, np.int64)
     np.cumsum(lens, out=rp[1:])
     col = np.concatenate([np.sort(rng.choice(n, size=l, replace=False)) if l else np.zeros(0, np.int64)
@@ -77,11 +80,15 @@ def _special(kind, dtype):
 
 
 @pytest.mark.parametrize("dtype", [np.float32, np.float64])
-@pytest.mark.parametrize("kind", ["long_rows", "empty_rows", "one_row", "dense_row_block"])
-def test_spmv_edge_patterns(ora, kind, dtype):
+@pytest.mark.parametrize("kind", ["long_rows", "empty_rows", "one_row", "dense_row_block", "dense_small"])
+@pytest.mark.parametrize("static", [False, True])
+def test_spmv_edge_patterns(ora, kind, dtype, static):
+    """static=True: long-row single-vector products run on the column-sorted copy (its
+    padding rows, segments smaller than a warp, fixed-point sums for fp32)."""
     import differentiable_sparse_linear_b200 as sla
     A = _special(kind, dtype)
-    Ad = matrix(A)
+    Ad = (sla.sla_csr_create(dev(A.row_ptr), dev(A.col), dev(A.val), static_values=True) if static
+          else matrix(A))
     for k in (1, 4):
         X = _x(A.n_rows, k, dtype, 11)
         if k == 1:
