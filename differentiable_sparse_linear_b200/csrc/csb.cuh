@@ -210,30 +210,9 @@ __device__ __forceinline__ void red_add_u32(uint32_t *p, uint32_t v)
 }
 
 // The matrix stream (chunk bases, packed words, values) is read once: loaded without L1
-// allocation, so L1 keeps the gathered operand lines (q = A p on the power-law 4M system:
-// 0.514 against 0.530 ms with L1-allocating loads; an L2 evict-first hint on top was
-// slower, 0.579).
-__device__ __forceinline__ uint32_t ld_stream_b32(const void *q)
-{
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(q));
-    return v;
-}
-__device__ __forceinline__ uint64_t ld_stream_b64(const void *q)
-{
-    uint64_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.b64 %0, [%1];" : "=l"(v) : "l"(q));
-    return v;
-}
-template <typename VM>
-__device__ __forceinline__ VM ld_stream_val(const VM *q)
-{
-    if constexpr (sizeof(VM) == 4)
-        return __uint_as_float(ld_stream_b32(q));
-    else
-        return __longlong_as_double((long long)ld_stream_b64(q));
-}
-
+// allocation (ld_stream_*), so L1 keeps the gathered operand lines (q = A p on the
+// power-law 4M system: 0.514 against 0.530 ms with L1-allocating loads; an L2 evict-first
+// hint on top was slower, 0.579).
 // One round's matrix data of a warp: U chunks (or padding past the segment's end).
 template <typename VM, int U>
 struct CsbRound {

@@ -36,6 +36,19 @@ struct LaneVals {
     __device__ __forceinline__ VV get(int vi, int64_t, int c) const { return v[vi][c]; }
 };
 
+// A slot's value: with 4 or more right-hand sides loaded without L1 allocation (the operand
+// rows are wide and L1 is better left to them: the 8-RHS heat solve ran 59.0 against 61.4 us
+// per iteration); with fewer, an L1-allocating load (the L2-resident 1024^2 SPAI solve ran
+// 36.3 against 47.7 us with no-allocate loads).
+template <int K, typename VM>
+__device__ __forceinline__ VM sell_val(const VM *q)
+{
+    if constexpr (K >= 4)
+        return ld_stream_val(q);
+    else
+        return *q;
+}
+
 // The slices [s0, s1) of this block, warps round-robin over consecutive slices, RS slices
 // per round (their loads all in flight together); `part` takes the epilogue's dot-product
 // partials in a fixed order.  In a diagonal slice the operand rows are row + offs[u]
@@ -96,7 +109,7 @@ __device__ __forceinline__ void sell_phase(const SellView<VM> &m, const Op &op, 
                 for (int u = 0; u < MAXL; ++u) {
                     if (u < L) {
                         const int32_t j = min(max(row + of[u], 0), nlast);
-                        const Acc av = (Acc)m.val[e0 + u * 32];
+                        const Acc av = (Acc)sell_val<K>(&m.val[e0 + u * 32]);
                         VV o[K];
                         op.operand_row(j, o, s_scal);
 #pragma unroll
@@ -111,7 +124,7 @@ __device__ __forceinline__ void sell_phase(const SellView<VM> &m, const Op &op, 
                     if (u < len) {
                         const int32_t j =
                             m.idx16 ? row + (int32_t)m.idx16[e0 + u * 32] : m.idx32[e0 + u * 32];
-                        const Acc av = (Acc)m.val[e0 + u * 32];
+                        const Acc av = (Acc)sell_val<K>(&m.val[e0 + u * 32]);
                         VV o[K];
                         op.operand_row(j, o, s_scal);
 #pragma unroll

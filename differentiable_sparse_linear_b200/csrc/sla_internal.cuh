@@ -144,6 +144,29 @@ struct SellPart {
 // 32 entry slots, its entries in ascending (column, row) order; per chunk the smallest
 // column, per slot (column - base) << 16 | local row (0xFFFF: padding), the CSR position of
 // the entry (-1: padding) and its value (gathered from the CSR values before each solve).
+// Loads of data read once (a matrix stream), without L1 allocation: L1 is left to data that
+// is read again (gathered operand lines).
+__device__ __forceinline__ uint32_t ld_stream_b32(const void *q)
+{
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(q));
+    return v;
+}
+__device__ __forceinline__ uint64_t ld_stream_b64(const void *q)
+{
+    uint64_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.b64 %0, [%1];" : "=l"(v) : "l"(q));
+    return v;
+}
+template <typename VM>
+__device__ __forceinline__ VM ld_stream_val(const VM *q)
+{
+    if constexpr (sizeof(VM) == 4)
+        return __uint_as_float(ld_stream_b32(q));
+    else
+        return __longlong_as_double((long long)ld_stream_b64(q));
+}
+
 struct CsbPart {
     int n_seg = 0;
     int rmax = 0;                        // rows of the largest segment
