@@ -17,6 +17,8 @@
 #include "bsr.cuh"
 #include "csb.cuh"
 
+#include <type_traits>
+
 namespace sla {
 
 // ------------------------------------------------------------------ elementwise kernels
@@ -76,7 +78,26 @@ k_ep(int64_t n, const V *z, const V *p_old, V *p_new, PcgState *st)
     __syncthreads();
     using IO = RowIO<V, K>;
     const int64_t stride = (int64_t)gridDim.x * VEC_T;
-    for (int64_t i = (int64_t)blockIdx.x * VEC_T + threadIdx.x; i < n; i += stride) {
+    int64_t i0 = (int64_t)blockIdx.x * VEC_T + threadIdx.x;
+    if constexpr (K == 1) {
+        // one right-hand side: 16-byte loads and stores where the vectors allow them
+        using L = typename std::conditional<sizeof(V) == 4, float4, double2>::type;
+        constexpr int VW = 16 / sizeof(V);
+        if ((((uintptr_t)z | (uintptr_t)p_old | (uintptr_t)p_new) & 15) == 0) {
+            const int64_t n4 = n / VW;
+            for (int64_t j = i0; j < n4; j += stride) {
+                L zz = reinterpret_cast<const L *>(z)[j], pp = reinterpret_cast<const L *>(p_old)[j], pn;
+                const V *zv = reinterpret_cast<const V *>(&zz), *pv = reinterpret_cast<const V *>(&pp);
+                V *nv = reinterpret_cast<V *>(&pn);
+#pragma unroll
+                for (int e = 0; e < VW; ++e)
+                    nv[e] = vfma<V>(s_b[0], pv[e], zv[e]);
+                reinterpret_cast<L *>(p_new)[j] = pn;
+            }
+            i0 += n4 * VW;
+        }
+    }
+    for (int64_t i = i0; i < n; i += stride) {
         V zz[K], pp[K], pn[K];
         IO::load(z + i * K, zz);
         IO::load(p_old + i * K, pp);
@@ -120,7 +141,37 @@ k_er(int64_t n, const V *r_old, const V *q, const V *p, V *x, V *r_new, double *
     for (int c = 0; c < K; ++c)
         part[c] = 0.0;
     const int64_t stride = (int64_t)gridDim.x * VEC_T;
-    for (int64_t i = (int64_t)blockIdx.x * VEC_T + threadIdx.x; i < n; i += stride) {
+    int64_t i0 = (int64_t)blockIdx.x * VEC_T + threadIdx.x;
+    if constexpr (K == 1) {
+        // one right-hand side: 16-byte loads and stores where the vectors allow them
+        using L = typename std::conditional<sizeof(V) == 4, float4, double2>::type;
+        constexpr int VW = 16 / sizeof(V);
+        if ((((uintptr_t)r_old | (uintptr_t)q | (uintptr_t)p | (uintptr_t)x | (uintptr_t)r_new) & 15) == 0) {
+            const int64_t n4 = n / VW;
+            const bool on = s_on[0] != 0.0;
+            for (int64_t j = i0; j < n4; j += stride) {
+                L ro = reinterpret_cast<const L *>(r_old)[j], qq = reinterpret_cast<const L *>(q)[j];
+                L pp = reinterpret_cast<const L *>(p)[j], xx = reinterpret_cast<const L *>(x)[j], rn;
+                const V *rov = reinterpret_cast<const V *>(&ro), *qv = reinterpret_cast<const V *>(&qq);
+                const V *pv = reinterpret_cast<const V *>(&pp);
+                V *xv = reinterpret_cast<V *>(&xx), *rnv = reinterpret_cast<V *>(&rn);
+#pragma unroll
+                for (int e = 0; e < VW; ++e) {
+                    if (on) {
+                        rnv[e] = vfma<V>(-s_a[0], qv[e], rov[e]);
+                        xv[e] = vfma<V>(s_a[0], pv[e], xv[e]);
+                    } else {
+                        rnv[e] = rov[e];
+                    }
+                    part[0] += (double)rnv[e] * (double)rnv[e];
+                }
+                reinterpret_cast<L *>(r_new)[j] = rn;
+                reinterpret_cast<L *>(x)[j] = xx;
+            }
+            i0 += n4 * VW;
+        }
+    }
+    for (int64_t i = i0; i < n; i += stride) {
         V ro[K], qq[K], pp[K], xx[K], rn[K];
         IO::load(r_old + i * K, ro);
         IO::load(q + i * K, qq);
