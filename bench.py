@@ -194,12 +194,17 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the sources that define a kernel (its ncu traffic is tied to it)."""
+    """Hash of the code that defines a kernel (its ncu traffic is tied to it): the listed
+    sources with their // comments and blank lines left out, so an edit of a comment does
+    not detach a capture from the code it measured."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differentiable_sparse_linear_b200", "csrc")
     for fn in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -4,18 +4,19 @@
 // In CSR order every stored entry gathers one operand from a random column, so each entry
 // costs its own L2 request; measured on B200, a random 4-byte gather stream tops out near
 // 270 G gathers/s, a third of what the matrix stream alone would allow.  Here the rows are
-// cut into segments of at most CSB_RMAX consecutive rows, and each segment's entries are
-// stored in COLUMN order: the 32 lanes of a warp then gather from a few hundred neighbouring
-// columns instead of 32 random ones, so one L2 request serves several entries.  The row sums
-// are accumulated in shared memory (one slot per row of the segment, fp64, atomic adds), and
-// the fused row epilogue of the operation runs once the segment's entries are done.
+// cut into segments of consecutive rows (CSB_RMAX, or CSB_RMAX_F32 for fp32 values), and
+// each segment's entries are stored in COLUMN order: the 32 lanes of a warp then gather from
+// a few hundred neighbouring columns instead of 32 random ones, so one L2 request serves
+// several entries.  The row sums are accumulated in shared memory (atomic adds into the
+// segment's row slots, see "Row sums" below), and the fused row epilogue of the operation
+// runs once the segment's entries are done.
 //
 // Storage (CsbPart): per segment its first row and first chunk; entries in chunks of 32
 // (one warp load), per chunk the smallest column `base`, per entry a 32-bit word
-// (column - base) << 16 | local row, padding marked by a flag bit (csb_pad_word), and the entry's
-// value, gathered from the caller's CSR values by `perm` at the start of every solve (the
-// values may change between solves; the pattern may not).  8 bytes per entry plus 4 per 32
-// entries, as CSR's value + column index.
+// (column - base) << 16 | local row, padding marked by a flag bit (csb_pad_word), and the
+// entry's value, gathered from the caller's CSR values by `perm` at the start of every
+// solve (the values may change between solves; the pattern may not).  8 bytes per entry
+// plus 4 per 32 entries, as CSR's value + column index.
 //
 // Row sums.  With fp32 values and vectors every product a_ij v_j is rounded to an integer
 // on a per-segment fixed-point scale and the row sums are exact integer sums, kept as three
