@@ -131,12 +131,6 @@ struct SellPart {
     void *d_idx = nullptr;               // int16 offsets (rel16) or int32 columns
     int32_t *d_perm = nullptr;
     void *d_val = nullptr;               // the matrix's type
-    // exact fixed-point row sums (csb.cuh): per segment the largest row sum of |a_ij| (with
-    // the values), the operand's per-block |v| maxima, the low word's bits
-    double *d_seg_bound = nullptr;
-    float *d_vmax = nullptr;
-    int vmax_n = 0;
-    int lb = 20;
 };
 
 // Column-sorted row segments of a long-row matrix (csb.cuh): segment s holds rows
